@@ -1,0 +1,97 @@
+/*
+ * oracle.h -- plain, slow, fp64 CPU oracle for exact scaled dot-product
+ * attention forward.  TEST INFRASTRUCTURE ONLY: only tests/, the package's
+ * smoke() entry and bench.py's cpu_baseline / reference leg may load it.  It
+ * shares no code, header, table or helper with the CUDA library.
+ *
+ * Every function takes bf16 inputs as raw 16-bit patterns (exactly widened to
+ * double) and computes in double precision.  Sources (page title, section):
+ *
+ *   [CIA] "Coding interview (14): attention from scratch" (arganzheng.life),
+ *         sections 3.1 softmax, 3.2 sdpa, 3.4 GQA, 3.5 RoPE, 3.6 KV cache,
+ *         3.7 online softmax.
+ *   [TAB] "Transformer Architecture Breakdown: Self-Attention, MHA/GQA/MQA,
+ *         RoPE & FlashAttention 1/2/3" (airsota.com), sections 1.2, 3.1, 4.2.
+ *   [AME] "Attention mechanisms: from alignment to efficient long context"
+ *         (fahimfaisal.info), sections 3, 5, 9, 19.
+ *   [TAD] "Transformer Architecture Deconstructed: Attention, Geometric
+ *         Scaling, and Memory IO" (byronfinn.github.io), "Online Softmax and
+ *         Blocked Incremental Computation".
+ *
+ * Parity status: every function here is pinned by tests/test_oracle.py
+ * (closed forms, invariants, library special cases, printed worked values).
+ */
+#ifndef ATTN_ORACLE_H
+#define ATTN_ORACLE_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Stable softmax of x[0..n) into out ([CIA] 3.1: subtract the max, then
+ * exponentiate and normalise).  n >= 1. */
+void oracle_softmax(const double* x, int64_t n, double* out);
+
+/* log(sum(exp(x))) computed as max + log(sum(exp(x - max))) ([CIA] 3.1).
+ * Returns -inf for n == 0. */
+double oracle_logsumexp(const double* x, int64_t n);
+
+/* RoPE: out[b,h,t,:] = R(pos_offset + t) * x[b,h,t,:] in fp64 ([TAB] 3.1,
+ * [CIA] 3.5).  theta_i = base^(-2i/d), i = 0..d/2-1.  pairing 0 rotates
+ * (x_i, x_{i+d/2}); pairing 1 rotates (x_{2i}, x_{2i+1}).  Each pair (a, b)
+ * becomes (a cos - b sin, a sin + b cos) with angle t * theta_i. */
+void oracle_rope(const uint16_t* x, double* out, int64_t B, int64_t H,
+                 int64_t N, int64_t d, double base, int64_t pos_offset,
+                 int pairing);
+
+/* Number of keys visible to query row i: keys j in [0, result) are visible.
+ * L = key_len clamped to [0, Nk]; causal adds j <= i + (Nk - Nq)
+ * (bottom-right alignment, [CIA] self-test 5).  Result may be 0. */
+int64_t oracle_visible_prefix(int64_t i, int64_t Nq, int64_t Nk, int causal,
+                              int64_t key_len);
+
+/* Definition of the result ([AME] 3, 5, 9; [CIA] 3.2, 3.4):
+ *   g = h / (Hq / Hkv);  s_j = scale * <q_i, k_j> for visible j;
+ *   m = max s; p_j = exp(s_j - m); l = sum p; O_i = sum p_j v_j / l;
+ *   lse_i = m + log(l).  No visible key: O_i = 0, lse_i = -inf.
+ * Layout: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] row-major bf16 bits.
+ * rows: flat row ids r = (b*Hq + h)*Nq + i, or NULL for every row in order.
+ * o: [nrows, d] doubles; lse: [nrows] (may be NULL).
+ * rope != 0 rotates q at position q_pos_offset + i and k at k_pos_offset + j
+ * (unrounded fp64) before the dot product.
+ * key_lens: int32[B] or NULL (= Nk).  nthreads >= 1.
+ * Returns 0, or -1 on invalid arguments. */
+int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
+                     int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
+                     int64_t Nk, int64_t d, int causal, double scale,
+                     const int32_t* key_lens, int rope, double rope_base,
+                     int rope_pairing, int64_t q_pos_offset,
+                     int64_t k_pos_offset, const int64_t* rows, int64_t nrows,
+                     double* o, double* lse, int nthreads);
+
+/* Same result through the one-query-at-a-time online recurrence ([CIA] 3.7,
+ * [AME] 19, [TAD] online softmax): keys visited in blocks of `block`, with a
+ * running max m, running sum l and unnormalised accumulator rescaled by
+ * exp(m_old - m_new) whenever the max grows.  No RoPE. */
+int oracle_attn_online_rows(const uint16_t* q, const uint16_t* k,
+                            const uint16_t* v, int64_t B, int64_t Hq,
+                            int64_t Hkv, int64_t Nq, int64_t Nk, int64_t d,
+                            int causal, double scale, const int32_t* key_lens,
+                            int64_t block, const int64_t* rows, int64_t nrows,
+                            double* o, double* lse, int nthreads);
+
+/* Which KV tiles a query tile touches, by brute force over the visibility
+ * predicate: tile jt (keys [jt*Bc, min((jt+1)*Bc, Nk))) is touched by query
+ * tile qt (rows [qt*Br, min((qt+1)*Br, Nq))) iff some row of the query tile
+ * sees some key of the KV tile.  Writes the first and last touched tile and
+ * the count (first = last = -1, count = 0 when none). */
+void oracle_kv_tiles(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
+                     int64_t Br, int64_t Bc, int64_t qt, int64_t* first,
+                     int64_t* last, int64_t* count);
+
+#ifdef __cplusplus
+}
+#endif
+#endif
