@@ -1,0 +1,456 @@
+#!/usr/bin/env python
+"""Benchmark of the exact attention forward hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
+
+One step = one attn_fwd call over one batch of the workload (default: causal
+MHA prefill, B=4, H=16, N=2048, d=128).  Inputs are resident in HBM; each
+step reads one of several input copies whose total exceeds the 126 MB L2, so
+no step finds its inputs in cache.  W untimed warm-up steps precede K timed
+steps bracketed by a barrier and a device synchronisation; the time is the
+maximum over ranks of CUDA-event time on the launching stream.  For N > 1
+(torchrun) every rank runs an independent batch (weak scaling, no
+collective on the data path).
+
+The JSON line also carries: the roofline of the dominant kernel, the
+end-to-end figure through the public API with host buffers, the oracle timed
+on host cores (rank 0, N=1, bounded sample), SM clocks sampled during the
+timed region, and the decode workload (MQA over a ragged KV cache) in GB/s.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from exact_scaled_dot_fwd_b200 import synth  # noqa: E402
+
+METRIC = "attention fwd TFLOPS (bf16, causal) and decode GB/s; % of B200 roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_BYTES = 126 * 1024 * 1024
+
+# DRAM traffic per launch of the dominant kernels, from one ncu capture each
+# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload; None when
+# the kernel changed after the capture.
+NCU_TRAFFIC_BYTES = {
+    "mha_prefill": None,
+    "mqa_decode": None,
+}
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=None)
+    p.add_argument("--warmup", type=int, default=5)
+    p.add_argument("--config", default="mha_prefill", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-cpu", action="store_true")
+    p.add_argument("--cpu-seconds", type=float, default=12.0)
+    return p.parse_args()
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            j = json.load(f)
+        return {k: float(j[k]) for k in FALLBACK_PEAKS}, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ------------------------------------------------------------------ clocks --
+
+def gpu_selector(torch, device):
+    """nvidia-smi -i argument for the torch device: its PCI bus id."""
+    try:
+        p = torch.cuda.get_device_properties(device)
+        return "%08X:%02X:%02X.0" % (p.pci_domain_id, p.pci_bus_id, p.pci_device_id)
+    except Exception:
+        return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during a region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, bus_id=None):
+        self.bus_id = bus_id
+        self.proc = None
+        self.out = None
+
+    def start(self):
+        cmd = ["nvidia-smi", "--query-gpu=" + self.FIELDS, "--format=csv,noheader,nounits",
+               "-lms", "100"]
+        if self.bus_id:
+            cmd[1:1] = ["-i", self.bus_id]
+        try:
+            self.out = tempfile.TemporaryFile(mode="w+")
+            self.proc = subprocess.Popen(cmd, stdout=self.out, stderr=subprocess.DEVNULL)
+        except Exception as e:  # noqa: BLE001
+            self.proc = None
+            self.err = repr(e)
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None,
+                    "reasons": ["nvidia-smi unavailable: " + getattr(self, "err", "")]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.out.seek(0)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.out.read().splitlines():
+            parts = [x.strip() for x in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ------------------------------------------------------------------ oracle --
+
+def oracle_sample(w, seconds, seed=12345, rows_per_batch=None):
+    """Time the fp64 oracle on uniformly sampled rows of workload w.
+    Returns (useful_flops, elapsed_s, rows, threads)."""
+    import oracle
+    x = synth.make_inputs(w)
+    total_rows = w.B * w.Hq * w.Nq
+    rng = np.random.Generator(np.random.PCG64(seed))
+    threads = oracle.default_threads()
+    kl = x["key_lens"]
+
+    def flops(rows):
+        f = 0.0
+        for r in rows:
+            i = int(r % w.Nq)
+            b = int(r // (w.Nq * w.Hq))
+            L = w.Nk if kl is None else int(kl[b])
+            f += 4.0 * w.d * oracle.visible_prefix(i, w.Nq, w.Nk, w.causal, L)
+        return f
+
+    rope = (dict(base=synth.ROPE_BASE, pairing=0, q_pos_offset=0, k_pos_offset=0)
+            if w.rope else None)
+    n = rows_per_batch or 8 * threads
+    used_f, used_t, used_rows = 0.0, 0.0, 0
+    while used_t < seconds:
+        rows = np.sort(rng.integers(0, total_rows, size=n)).astype(np.int64)
+        t0 = time.perf_counter()
+        oracle.attn_rows(x["q"], x["k"], x["v"], w.causal, w.scale, key_lens=kl, rows=rows,
+                         rope_cfg=rope, nthreads=threads)
+        dt = time.perf_counter() - t0
+        used_f += flops(rows)
+        used_t += dt
+        used_rows += n
+        if dt < 0.5 * seconds:
+            n = min(n * 2, 1 << 16)
+    return used_f, used_t, used_rows, threads
+
+
+# ------------------------------------------------------------------- ours ---
+
+def to_dev(bits, torch, device):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
+
+
+def decode_bytes(w, key_lens):
+    kv = float(np.clip(key_lens, 0, w.Nk).sum()) * w.Hkv * w.d * 2 * 2
+    return kv + w.B * w.Hq * w.d * 2 * 2 + w.B * w.Hq * 4
+
+
+def time_steps(fn, steps, torch, dist, stream):
+    """Barrier + sync, events around `steps` calls of fn(i), sync + barrier;
+    returns the max over ranks of the elapsed ms."""
+    if dist is not None:
+        dist.barrier()
+    torch.cuda.synchronize()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(steps):
+        fn(i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    if dist is not None:
+        dist.barrier()
+    ms = e0.elapsed_time(e1)
+    if dist is not None:
+        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms
+
+
+def run_ours(args):
+    import torch
+    import exact_scaled_dot_fwd_b200 as eb
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    dist = None
+    if world > 1:
+        import datetime
+        import torch.distributed as tdist
+        torch.cuda.set_device(local)
+        tdist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                 device_id=torch.device("cuda", local))
+        dist = tdist
+    else:
+        torch.cuda.set_device(0)
+    device = torch.device("cuda", torch.cuda.current_device())
+    eb.lib()
+    peaks, peak_src = load_peaks()
+    stream = torch.cuda.current_stream()
+
+    w = synth.WORKLOADS[args.config]
+    # every rank processes its own batch: shift the seed by the rank
+    wr = synth.Workload(**{**w.__dict__, "number": w.number + 100 * rank}) if rank else w
+    x = synth.make_inputs(wr)
+    per_copy = sum(x[n].nbytes for n in ("q", "k", "v"))
+    copies = max(1, min(8, math.ceil(2 * L2_BYTES / per_copy)))
+    Q = [to_dev(x["q"], torch, device) for _ in range(copies)]
+    K = [to_dev(x["k"], torch, device) for _ in range(copies)]
+    V = [to_dev(x["v"], torch, device) for _ in range(copies)]
+    kl = None if x["key_lens"] is None else torch.from_numpy(x["key_lens"]).to(device)
+    O = torch.empty_like(Q[0])
+    LSE = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
+    ws = None
+    if w.Nq == 1:
+        ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, 1, w.Nk, w.d),
+                         dtype=torch.uint8, device=device)
+
+    def step(i):
+        c = i % copies
+        eb.attn_fwd_ws(Q[c], K[c], V[c], ws, causal=w.causal, scale=w.scale, key_lens=kl,
+                       out=O, lse=LSE)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    # size K so that the timed region lasts about two seconds by default
+    probe = time_steps(step, 3, torch, dist, stream) / 3
+    steps = args.steps or max(10, int(2000.0 / max(probe, 1e-3)))
+    sampler = ClockSampler(gpu_selector(torch, device))
+    sampler.start()
+    time.sleep(0.3)
+    ms = time_steps(step, steps, torch, dist, stream)
+    clocks = sampler.stop()
+    ms_step = ms / steps
+    launches_per_step = 2 if w.Nq == 1 else 1
+    if w.Nq == 1:
+        unit, work = "GB/s", decode_bytes(w, x["key_lens"])
+        value = world * work * steps / (ms / 1e3) / 1e9
+        roof = {"bound": "hbm", "achieved": value / world, "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": value / world / peaks["hbm_gbs"],
+                "traffic": NCU_TRAFFIC_BYTES.get(w.name), "peak_source": peak_src}
+    else:
+        unit, work = "TFLOP/s", w.flops()
+        value = world * work * steps / (ms / 1e3) / 1e12
+        roof = {"bound": "tensor", "achieved": value / world, "peak": peaks["bf16_tflops"],
+                "unit": "TFLOP/s", "frac": value / world / peaks["bf16_tflops"],
+                "traffic": NCU_TRAFFIC_BYTES.get(w.name), "peak_source": peak_src}
+    line = {
+        "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
+                   "Nk": w.Nk, "d": w.d, "causal": w.causal, "rope": w.rope,
+                   "key_lens": list(w.key_lens) if w.key_lens else None,
+                   "l2": f"{copies} rotating input copies ({copies * per_copy / 1e6:.0f} MB > "
+                         f"126 MB L2)",
+                   "parallelism": f"replicas x{world} (independent batch per GPU)"},
+        "roofline": roof,
+        "gpu_launches": steps * launches_per_step,
+        "clocks": clocks,
+    }
+
+    # ---- end to end through the public API with pinned host buffers
+    if not args.no_e2e:
+        hq = torch.from_numpy(x["q"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        hk = torch.from_numpy(x["k"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        hv = torch.from_numpy(x["v"].view(np.int16)).view(torch.bfloat16).pin_memory()
+        ho = torch.empty(O.shape, dtype=torch.bfloat16).pin_memory()
+        hl = torch.empty(LSE.shape, dtype=torch.float32).pin_memory()
+
+        def e2e_step(i):
+            Q[0].copy_(hq, non_blocking=True)
+            K[0].copy_(hk, non_blocking=True)
+            V[0].copy_(hv, non_blocking=True)
+            eb.attn_fwd_ws(Q[0], K[0], V[0], ws, causal=w.causal, scale=w.scale, key_lens=kl,
+                           out=O, lse=LSE)
+            ho.copy_(O, non_blocking=True)
+            hl.copy_(LSE, non_blocking=True)
+
+        for i in range(2):
+            e2e_step(i)
+        e_steps = max(3, min(steps, 20))
+        ems = time_steps(e2e_step, e_steps, torch, dist, stream)
+        h2d = hq.numel() * 2 + hk.numel() * 2 + hv.numel() * 2
+        d2h = ho.numel() * 2 + hl.numel() * 4
+        ev = world * work * e_steps / (ems / 1e3) / (1e9 if unit == "GB/s" else 1e12)
+        line["e2e"] = {"value": ev, "unit": unit, "h2d_bytes_per_step": h2d,
+                       "d2h_bytes_per_step": d2h, "steps": e_steps}
+
+    # ---- decode workload (HBM-bound half of the metric), same run
+    if not args.no_decode and w.Nq != 1 and rank == 0 and world == 1:
+        line["decode"] = run_decode(torch, eb, device, stream, peaks, peak_src)
+
+    # ---- oracle on host cores (rank 0, N=1 only)
+    if not args.no_cpu and rank == 0 and world == 1:
+        f, t, rows, thr = oracle_sample(w, args.cpu_seconds)
+        line["cpu_baseline"] = {
+            "value": (f / t) / (1e12 if unit == "TFLOP/s" else 1.0) if unit == "TFLOP/s"
+            else None,
+            "unit": "TFLOP/s (useful, sampled rows)" if unit == "TFLOP/s" else "n/a",
+            "cores": thr, "kind": "oracle",
+            "sample": f"{rows} uniformly drawn query rows of {w.name}, fp64, {t:.1f} s"}
+        if unit == "GB/s":
+            # bytes the sampled rows read (K and V of the visible keys)
+            line["cpu_baseline"]["value"] = (f / (4.0 * w.d)) * w.d * 4 / t / 1e9
+            line["cpu_baseline"]["unit"] = "GB/s (K/V bytes of sampled rows)"
+
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if dist is not None:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None):
+    w = synth.WORKLOADS["mqa_decode"]
+    x = synth.make_inputs(w)
+    per_copy = x["k"].nbytes + x["v"].nbytes
+    copies = 2
+    Q = to_dev(x["q"], torch, device)
+    K = [to_dev(x["k"], torch, device) for _ in range(copies)]
+    V = [to_dev(x["v"], torch, device) for _ in range(copies)]
+    kl = torch.from_numpy(x["key_lens"]).to(device)
+    O = torch.empty_like(Q)
+    LSE = torch.empty((w.B, w.Hq, 1), dtype=torch.float32, device=device)
+    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, 1, w.Nk, w.d), dtype=torch.uint8,
+                     device=device)
+
+    def step(i):
+        eb.attn_fwd_ws(Q, K[i % copies], V[i % copies], ws, scale=w.scale, key_lens=kl, out=O,
+                       lse=LSE)
+
+    for i in range(5):
+        step(i)
+    probe = time_steps(step, 5, torch, None, stream) / 5
+    n = steps or max(20, int(1000.0 / max(probe, 1e-3)))
+    ms = time_steps(step, n, torch, None, stream)
+    gbs = decode_bytes(w, x["key_lens"]) * n / (ms / 1e3) / 1e9
+    return {"metric": "decode GB/s (algorithmic bytes: K/V of valid keys + Q + O + lse)",
+            "value": gbs, "unit": "GB/s", "workload": w.name, "steps": n, "ms_per_step": ms / n,
+            "algorithmic_bytes": decode_bytes(w, x["key_lens"]),
+            "l2": f"{copies} rotating KV caches ({copies * per_copy / 1e6:.0f} MB allocated)",
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"],
+                         "traffic": NCU_TRAFFIC_BYTES.get(w.name), "peak_source": peak_src},
+            "gpu_launches": 2 * n}
+
+
+# -------------------------------------------------------------- reference ---
+
+def run_reference(args):
+    """The oracle as the reference arm: each step is a bounded sample of rows
+    of the same workload, timed on the host cores."""
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if rank != 0:
+        return
+    import oracle
+    w = synth.WORKLOADS[args.config]
+    threads = oracle.default_threads()
+    x = synth.make_inputs(w)
+    kl = x["key_lens"]
+    rng = np.random.Generator(np.random.PCG64(777))
+    rope = (dict(base=synth.ROPE_BASE, pairing=0, q_pos_offset=0, k_pos_offset=0)
+            if w.rope else None)
+    rows_per_step = 4 * threads
+    total_rows = w.B * w.Hq * w.Nq
+
+    def one(rows):
+        oracle.attn_rows(x["q"], x["k"], x["v"], w.causal, w.scale, key_lens=kl, rows=rows,
+                         rope_cfg=rope, nthreads=threads)
+
+    def flops(rows):
+        f = 0.0
+        for r in rows:
+            i = int(r % w.Nq)
+            b = int(r // (w.Nq * w.Hq))
+            L = w.Nk if kl is None else int(kl[b])
+            f += 4.0 * w.d * oracle.visible_prefix(i, w.Nq, w.Nk, w.causal, L)
+        return f
+
+    steps = args.steps or 5
+    for _ in range(args.warmup):
+        one(np.sort(rng.integers(0, total_rows, size=rows_per_step)))
+    t_total, f_total = 0.0, 0.0
+    for _ in range(steps):
+        rows = np.sort(rng.integers(0, total_rows, size=rows_per_step)).astype(np.int64)
+        t0 = time.perf_counter()
+        one(rows)
+        t_total += time.perf_counter() - t0
+        f_total += flops(rows)
+    if w.Nq == 1:
+        unit = "GB/s"
+        value = (f_total / (4.0 * w.d)) * w.d * 4 / t_total / 1e9
+    else:
+        unit = "TFLOP/s"
+        value = f_total / t_total / 1e12
+    sample = f"{rows_per_step} uniformly drawn query rows of {w.name} per step, fp64 oracle"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": unit,
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * t_total / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
+                       "Nk": w.Nk, "d": w.d, "causal": w.causal},
+            "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_ours(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,200 @@
+"""exact_scaled_dot_fwd_b200 -- exact scaled dot-product attention forward on
+B200 (sm_100a).
+
+Thin Python binding over the C ABI of libattn_b200.so (include/attn.h).  It
+only marshals arguments: torch tensors supply device pointers and the current
+CUDA stream; every step of the computation runs in the library's kernels.
+There is no CPU or library fallback: if the shared library is missing or a
+call fails, an exception is raised.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "rope_apply",
+           "prefill_tile_shape", "tile_plan", "device_status", "AttnError", "lib",
+           "STATUS_NAMES"]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
+
+STATUS_NAMES = {0: "ATTN_OK", 1: "ATTN_EINVAL", 2: "ATTN_EUNSUPPORTED", 3: "ATTN_EALIGN",
+                4: "ATTN_EWORKSPACE", 5: "ATTN_ECUDA", 6: "ATTN_ETIMEOUT"}
+
+_lib = None
+
+
+class AttnError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        super().__init__(f"{what}: {STATUS_NAMES.get(status, status)}")
+
+
+def lib():
+    """Load libattn_b200.so (raises OSError when it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise OSError(f"{LIB_PATH} is missing: build it with "
+                          "`python -m exact_scaled_dot_fwd_b200.build`")
+        L = ctypes.CDLL(LIB_PATH)
+        vp, i, f, sz = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
+        L.attn_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp]
+        L.attn_fwd.restype = i
+        L.attn_fwd_ws.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, vp, sz, vp]
+        L.attn_fwd_ws.restype = i
+        L.attn_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.attn_workspace_size.restype = sz
+        L.rope_apply.argtypes = [vp, vp, i, i, i, i, f, i, i, vp]
+        L.rope_apply.restype = i
+        L.attn_prefill_tile_shape.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(i)]
+        L.attn_prefill_tile_shape.restype = i
+        L.attn_fwd_tile_plan.argtypes = [i, i, i, i, i, vp, vp, vp, vp]
+        L.attn_fwd_tile_plan.restype = i
+        L.attn_device_status.argtypes = [vp, i]
+        L.attn_device_status.restype = i
+        L.attn_strerror.argtypes = [i]
+        L.attn_strerror.restype = ctypes.c_char_p
+        L.attn_abi_version.argtypes = []
+        L.attn_abi_version.restype = i
+        _lib = L
+    return _lib
+
+
+def _torch():
+    import torch
+    return torch
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream):
+    torch = _torch()
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check_tensor(t, name, dtype, ndim=None):
+    torch = _torch()
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions")
+
+
+def _raise(rc, what):
+    if rc != 0:
+        raise AttnError(rc, what)
+
+
+def _shapes(q, k, v):
+    B, Hq, Nq, d = q.shape
+    Bk, Hkv, Nk, dk = k.shape
+    if tuple(v.shape) != tuple(k.shape) or Bk != B or dk != d:
+        raise ValueError(f"shape mismatch q{tuple(q.shape)} k{tuple(k.shape)} v{tuple(v.shape)}")
+    return B, Hq, Hkv, Nq, Nk, d
+
+
+def attn_fwd(q, k, v, causal=False, scale=None, key_lens=None, out=None, lse=None,
+             return_lse=True, stream=None):
+    """O = softmax(Q K^T * scale + M) V on the GPU.
+
+    q: bf16 [B, Hq, Nq, d]; k, v: bf16 [B, Hkv, Nk, d]; key_lens: int32 [B]
+    (device) or None.  Returns (o, lse) (lse fp32 [B, Hq, Nq], natural log) or
+    o alone when return_lse is False.
+    """
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n, torch.bfloat16, 4)
+    B, Hq, Hkv, Nq, Nk, d = _shapes(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if key_lens is not None:
+        _check_tensor(key_lens, "key_lens", torch.int32, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse if return_lse else None),
+                        B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale), _ptr(key_lens),
+                        _stream(stream))
+    _raise(rc, "attn_fwd")
+    return (out, lse) if return_lse else out
+
+
+def attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) -> int:
+    return int(lib().attn_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+
+
+def attn_fwd_ws(q, k, v, workspace, causal=False, scale=None, key_lens=None, out=None,
+                lse=None, return_lse=True, stream=None):
+    """attn_fwd with a caller-owned workspace (uint8 CUDA tensor)."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n, torch.bfloat16, 4)
+    B, Hq, Hkv, Nq, Nk, d = _shapes(q, k, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if key_lens is not None:
+        _check_tensor(key_lens, "key_lens", torch.int32, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
+    rc = lib().attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                           _ptr(lse if return_lse else None), B, Hq, Hkv, Nq, Nk, d,
+                           int(bool(causal)), float(scale), _ptr(key_lens), _ptr(workspace),
+                           ws_bytes, _stream(stream))
+    _raise(rc, "attn_fwd_ws")
+    return (out, lse) if return_lse else out
+
+
+def rope_apply(x, base=10000.0, pos_offset=0, pairing=0, out=None, stream=None):
+    """RoPE on bf16 [B, H, N, d]; out=x rotates in place."""
+    torch = _torch()
+    _check_tensor(x, "x", torch.bfloat16, 4)
+    if out is None:
+        out = torch.empty_like(x)
+    B, H, N, d = x.shape
+    rc = lib().rope_apply(_ptr(x), _ptr(out), B, H, N, d, float(base), int(pos_offset),
+                          int(pairing), _stream(stream))
+    _raise(rc, "rope_apply")
+    return out
+
+
+def prefill_tile_shape(d):
+    br, bc = ctypes.c_int(), ctypes.c_int()
+    _raise(lib().attn_prefill_tile_shape(d, ctypes.byref(br), ctypes.byref(bc)),
+           "attn_prefill_tile_shape")
+    return br.value, bc.value
+
+
+def tile_plan(B, Nq, Nk, d, causal, key_lens=None, device="cuda", stream=None):
+    """(first, count) int32 [B, nqt] tensors: the KV tiles the prefill kernel
+    visits for each (b, query tile)."""
+    torch = _torch()
+    br, _ = prefill_tile_shape(d)
+    nqt = -(-Nq // br)
+    first = torch.empty((B, nqt), dtype=torch.int32, device=device)
+    count = torch.empty((B, nqt), dtype=torch.int32, device=device)
+    rc = lib().attn_fwd_tile_plan(B, Nq, Nk, d, int(bool(causal)), _ptr(key_lens), _ptr(first),
+                                  _ptr(count), _stream(stream))
+    _raise(rc, "attn_fwd_tile_plan")
+    return first, count
+
+
+def device_status(reset=True, stream=None) -> int:
+    """Synchronise and read the library's device status word (0 = OK)."""
+    return int(lib().attn_device_status(_stream(stream), int(bool(reset))))

@@ -1,0 +1,224 @@
+// api.cu -- the C ABI of libattn_b200.so: argument checks, dispatch, the
+// library-owned decode workspace, TMA descriptor encoding and the device
+// status word.  Declarations and contracts are in include/attn.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "attn.h"
+#include "common.cuh"
+#include "kernels.h"
+
+namespace attn {
+
+__device__ int g_device_status = 0;
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*,
+                                   const cuuint64_t*, const cuuint64_t*, const cuuint32_t*,
+                                   const cuuint32_t*, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                   CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+int current_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+// Library-owned decode workspace, one per device, grown on demand.
+struct OwnedWorkspace {
+  void* ptr = nullptr;
+  size_t bytes = 0;
+};
+constexpr int kMaxDevices = 64;
+OwnedWorkspace g_ws[kMaxDevices];
+std::mutex g_ws_mu;
+
+struct WorkspaceReaper {
+  ~WorkspaceReaper() {
+    // process exit: the driver may already be tearing down; ignore errors
+    for (auto& w : g_ws)
+      if (w.ptr) cudaFree(w.ptr);
+  }
+} g_reaper;
+
+int check_common(const void* q, const void* k, const void* v, const void* o, int B, int Hq, int Hkv,
+                 int Nq, int Nk, int d, int causal, float scale) {
+  if (!q || !k || !v || !o) return ATTN_EINVAL;
+  if (B <= 0 || Hq <= 0 || Hkv <= 0 || Nq <= 0 || Nk <= 0 || d <= 0) return ATTN_EINVAL;
+  if (Hq % Hkv != 0) return ATTN_EINVAL;
+  if (causal != 0 && causal != 1) return ATTN_EINVAL;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return ATTN_EINVAL;
+  if (d != 64 && d != 128) return ATTN_EUNSUPPORTED;
+  if ((long long)B * Hq * Nq >= (1ll << 31) || (long long)B * Hkv * Nk >= (1ll << 31))
+    return ATTN_EUNSUPPORTED;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_EALIGN;
+  return ATTN_OK;
+}
+
+}  // namespace
+
+int make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                      uint32_t box_cols, uint32_t box_rows) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn) return ATTN_ECUDA;
+  cuuint64_t dims[2] = {cols, rows};
+  cuuint64_t strides[1] = {cols * 2};
+  cuuint32_t box[2] = {box_cols, box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ECUDA;
+}
+
+}  // namespace attn
+
+using namespace attn;
+
+extern "C" {
+
+int attn_abi_version(void) { return ATTN_ABI_VERSION; }
+
+const char* attn_strerror(int status) {
+  switch (status) {
+    case ATTN_OK: return "ATTN_OK";
+    case ATTN_EINVAL: return "ATTN_EINVAL: invalid argument";
+    case ATTN_EUNSUPPORTED: return "ATTN_EUNSUPPORTED: shape not supported by this build";
+    case ATTN_EALIGN: return "ATTN_EALIGN: pointer not 16-byte aligned";
+    case ATTN_EWORKSPACE: return "ATTN_EWORKSPACE: workspace missing or too small";
+    case ATTN_ECUDA: return "ATTN_ECUDA: CUDA call failed";
+    case ATTN_ETIMEOUT: return "ATTN_ETIMEOUT: a kernel gave up waiting on a barrier";
+    default: return "unknown attn status";
+  }
+}
+
+size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  (void)Nk;
+  if (Nq != 1 || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
+  const int sms = current_sms();
+  if (sms <= 0) return 0;
+  return decode_plan(B, Hq, Hkv, d, sms).workspace_bytes;
+}
+
+int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int d, int causal, float scale, const int32_t* key_lens,
+                void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != ATTN_OK) return rc;
+  if (lse && !aligned16(lse)) return ATTN_EALIGN;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (Nq == 1) {
+    if (!decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
+    const int sms = current_sms();
+    if (sms <= 0) return ATTN_ECUDA;
+    const DecodePlan p = decode_plan(B, Hq, Hkv, d, sms);
+    if (!workspace || workspace_bytes < p.workspace_bytes) return ATTN_EWORKSPACE;
+    if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
+    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nk, d, scale, key_lens, workspace, p, st);
+  }
+  if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, st);
+}
+
+int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+             int Hkv, int Nq, int Nk, int d, int causal, float scale, const int32_t* key_lens,
+             void* stream) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != ATTN_OK) return rc;
+  void* ws = nullptr;
+  size_t ws_bytes = 0;
+  if (Nq == 1) {
+    if (!decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
+    const size_t need = attn_workspace_size(B, Hq, Hkv, Nq, Nk, d);
+    if (need == 0) return ATTN_ECUDA;
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ECUDA;
+    std::lock_guard<std::mutex> lock(g_ws_mu);
+    OwnedWorkspace& w = g_ws[dev];
+    if (w.bytes < need) {
+      // the old buffer may still be in use by queued work on some stream
+      if (w.ptr && cudaDeviceSynchronize() != cudaSuccess) return ATTN_ECUDA;
+      if (w.ptr) cudaFree(w.ptr);
+      w.ptr = nullptr;
+      w.bytes = 0;
+      if (cudaMalloc(&w.ptr, need) != cudaSuccess) {
+        w.ptr = nullptr;
+        return ATTN_ECUDA;
+      }
+      w.bytes = need;
+    }
+    ws = w.ptr;
+    ws_bytes = w.bytes;
+  }
+  return attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, ws, ws_bytes,
+                     stream);
+}
+
+int rope_apply(const void* x_in, void* x_out, int B, int H, int N, int d, float base,
+               int pos_offset, int pairing, void* stream) {
+  if (!x_in || !x_out) return ATTN_EINVAL;
+  if (B <= 0 || H <= 0 || N <= 0 || d < 2 || d % 2 != 0) return ATTN_EINVAL;
+  if (!std::isfinite(base) || !(base > 0.f)) return ATTN_EINVAL;
+  if (pairing != 0 && pairing != 1) return ATTN_EINVAL;
+  if (pos_offset < 0) return ATTN_EINVAL;
+  if (d > 256) return ATTN_EUNSUPPORTED;
+  if ((long long)pos_offset + N > (1ll << 31) - 1) return ATTN_EINVAL;
+  if ((long long)B * H > 65535ll * 16) return ATTN_EUNSUPPORTED;
+  if (!aligned16(x_in) || !aligned16(x_out)) return ATTN_EALIGN;
+  const size_t bytes = (size_t)B * H * N * d * 2;
+  const uintptr_t a0 = reinterpret_cast<uintptr_t>(x_in), b0 = reinterpret_cast<uintptr_t>(x_out);
+  if (a0 != b0 && a0 < b0 + bytes && b0 < a0 + bytes) return ATTN_EINVAL;   // partial overlap
+  return launch_rope(x_in, x_out, B, H, N, d, base, pos_offset, pairing,
+                     static_cast<cudaStream_t>(stream));
+}
+
+int attn_prefill_tile_shape(int d, int* Br, int* Bc) {
+  if (!Br || !Bc) return ATTN_EINVAL;
+  if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
+  prefill_tile_shape(d, Br, Bc);
+  return ATTN_OK;
+}
+
+int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal, const int32_t* key_lens,
+                       int32_t* first, int32_t* count, void* stream) {
+  if (!first || !count) return ATTN_EINVAL;
+  if (B <= 0 || Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1)) return ATTN_EINVAL;
+  if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
+  return launch_tile_plan(B, Nq, Nk, d, causal, key_lens, first, count,
+                          static_cast<cudaStream_t>(stream));
+}
+
+int attn_device_status(void* stream, int reset) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return ATTN_ECUDA;
+  int v = 0;
+  if (cudaMemcpyFromSymbol(&v, g_device_status, sizeof v) != cudaSuccess) return ATTN_ECUDA;
+  if (reset) {
+    const int z = 0;
+    if (cudaMemcpyToSymbol(g_device_status, &z, sizeof z) != cudaSuccess) return ATTN_ECUDA;
+  }
+  return v == 0 ? ATTN_OK : v;
+}
+
+}  // extern "C"

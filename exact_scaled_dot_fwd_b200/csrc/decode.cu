@@ -1,0 +1,524 @@
+// decode.cu -- split-KV decode (Nq == 1) and its log-sum-exp combine pass.
+//
+// One new query token per sequence reads the whole KV cache of its sequence
+// ("Coding interview (14): attention from scratch", section 3.6: the newest
+// token needs no causal mask, only the cache length; "Transformer
+// Architecture Deconstructed ...", KV cache section: decode is a
+// bandwidth-bound matrix-vector product).  All Hq/Hkv query heads that share
+// a kv head are processed together, so every K/V byte is read from HBM once.
+//
+// Work split.  Unit u = (b, kv head h) owns len_u = clamp(key_lens[b], 0, Nk)
+// keys.  The units' keys are laid end to end (T keys in total) and CTA c of a
+// one-wave grid takes the global key range [c*T/G, (c+1)*T/G), which may cover
+// the tail of one unit and the head of the next.  Each (CTA, unit) piece is a
+// segment: the CTA runs the online-softmax recurrence over it and writes a
+// partial (O_s / l_s, log2 l_s + m_s) into slot c + u (unique: a later CTA
+// never touches an earlier unit).  The combine pass merges the slots of each
+// unit with the two-block merge rule of the online softmax ("Transformer
+// Architecture Breakdown ...", section 4.2), generalised to n blocks.
+//
+// Data movement.  K and V tiles of 64 keys arrive by TMA (2D tensor map over
+// the [B*Hkv*Nk, d] cache, 128-byte swizzle) into a 4-stage shared-memory ring
+// filled by a dedicated producer warp.  Consumer warps own 16 query heads
+// (one m16 tile) and a quarter (16 keys) of every tile; they use
+// ldmatrix + mma.sync.m16n8k16 (bf16 in, fp32 accumulate) for S = Q K^T and
+// O += P V.  At 32 heads per kv head the path needs ~32 FLOP per byte, well
+// inside what the tensor pipe sustains, so the kernel stays HBM-bound.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace attn {
+
+namespace {
+
+constexpr int kTileKeys = 64;
+constexpr int kStages = 4;
+constexpr int kMaxScanB = 2048;
+
+template <int D>
+struct DecodeSmem {
+  static constexpr int kTileBytes = kTileKeys * D * 2;   // one of K or V
+  static constexpr int kStageBytes = 2 * kTileBytes;
+  // layout (from a 1024-byte aligned base)
+  static constexpr int kRing = 0;
+  static constexpr int kBars = kRing + kStages * kStageBytes;   // full[S], empty[S]
+  static constexpr int kScan = kBars + 2 * kStages * 8;          // int64 [kMaxScanB + 1]
+  static constexpr int kLens = kScan + (kMaxScanB + 1) * 8;      // int [kMaxScanB]
+  static constexpr int kMbuf = kLens + kMaxScanB * 4;             // float [4 kq][4 mt][16]
+  static constexpr int kLbuf = kMbuf + 4 * 4 * 16 * 4;           // float [4 mt][16]
+  static constexpr int kObuf = kLbuf + 4 * 16 * 4;               // float [4 mt][16][D]
+  static constexpr int kAbort = kObuf + 4 * 16 * D * 4;
+  static constexpr int kTotal = kAbort + 16 + 1024;              // + alignment slack
+};
+
+struct Seg {
+  int u, lo, hi;
+};
+
+// Prefix of unit u: keys of all units before u (units are b-major, h-minor).
+__device__ __forceinline__ long long unit_prefix(const long long* pb, const int* lens, int u,
+                                                 int Hkv) {
+  const int b = u / Hkv, h = u - b * Hkv;
+  return (long long)Hkv * pb[b] + (long long)h * lens[b];
+}
+
+}  // namespace
+
+struct DecodeArgs {
+  const __nv_bfloat16* q;
+  const int32_t* key_lens;
+  float* part_o;
+  float* part_lse;
+  int B, Hq, Hkv, Nk, G, grid;
+  float scale_log2;
+};
+
+template <int D, int MT>
+__global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
+    decode_split_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                        const __grid_constant__ CUtensorMap tmap_v, DecodeArgs a) {
+  using L = DecodeSmem<D>;
+  constexpr int kConsumerWarps = MT * 4;
+  constexpr int kConsumerThreads = kConsumerWarps * 32;
+  constexpr int kBoxes = D / 64;             // 128-byte swizzle boxes per row
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + L::kBars);
+  uint64_t* empty = full + kStages;
+  long long* pb = reinterpret_cast<long long*>(smem + L::kScan);
+  float* mbuf = reinterpret_cast<float*>(smem + L::kMbuf);
+  float* lbuf = reinterpret_cast<float*>(smem + L::kLbuf);
+  float* obuf = reinterpret_cast<float*>(smem + L::kObuf);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  int* lens_s = reinterpret_cast<int*>(smem + L::kLens);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int B = a.B, Hkv = a.Hkv, U = B * Hkv;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], kConsumerWarps);
+    }
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  // key lengths (clamped) and their exclusive prefix over b, by warp 0
+  if (warp == 0) {
+    long long carry = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int b = base + lane;
+      int len = 0;
+      if (b < B) {
+        len = a.key_lens ? a.key_lens[b] : a.Nk;
+        len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+        lens_s[b] = len;
+      }
+      long long x = len;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (b < B) pb[b] = carry + x - len;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) pb[B] = carry;
+  }
+  __syncthreads();
+
+  const long long T = (long long)Hkv * pb[B];
+  const long long start = T * blockIdx.x / a.grid;
+  const long long end = T * (blockIdx.x + 1) / a.grid;
+  // first unit whose key range contains `start`
+  int u0 = 0;
+  if (start < end) {
+    int lo = 0, hi = U - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (unit_prefix(pb, lens_s, mid, Hkv) <= start) lo = mid; else hi = mid - 1;
+    }
+    u0 = lo;
+  }
+  auto next_seg = [&](int& u, Seg& s) -> bool {
+    while (u < U) {
+      const long long p0 = unit_prefix(pb, lens_s, u, Hkv);
+      if (p0 >= end) return false;
+      const long long p1 = p0 + lens_s[u / Hkv];
+      const long long lo = start > p0 ? start : p0, hi = end < p1 ? end : p1;
+      const int cur = u++;
+      if (hi > lo) {
+        s.u = cur; s.lo = (int)(lo - p0); s.hi = (int)(hi - p0);
+        return true;
+      }
+    }
+    return false;
+  };
+
+  if (warp == kConsumerWarps) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && start < end) {
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      int u = u0, it = 0;
+      Seg s;
+      bool ok = true;
+      while (ok && next_seg(u, s)) {
+        for (int t = s.lo; t < s.hi; t += kTileKeys, ++it) {
+          const int st = it % kStages;
+          const uint32_t ph = (it / kStages) & 1;
+          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
+          uint8_t* kt = smem + L::kRing + st * L::kStageBytes;
+          uint8_t* vt = kt + L::kTileBytes;
+          mbar_arrive_expect_tx(&full[st], L::kStageBytes);
+          const int row = s.u * a.Nk + t;
+#pragma unroll
+          for (int bx = 0; bx < kBoxes; ++bx) {
+            tma_load_2d(kt + bx * (kTileKeys * 128), &tmap_k, bx * 64, row, &full[st]);
+            tma_load_2d(vt + bx * (kTileKeys * 128), &tmap_v, bx * 64, row, &full[st]);
+          }
+        }
+      }
+      // drain: every issued stage must land before the CTA may exit
+      const int issued = it;
+      for (int j = issued - kStages > 0 ? issued - kStages : 0; j < issued; ++j)
+        mbar_wait(&full[j % kStages], (j / kStages) & 1, nullptr);
+    }
+    return;
+  }
+
+  // -------------------------------------------------------------- consumers
+  const int mt = warp % MT, kq = warp / MT;
+  const int g = lane >> 2, t4 = lane & 3;
+  int u = u0, it = 0;
+  Seg s;
+  bool alive = start < end;
+  while (alive && next_seg(u, s)) {
+    const int b = s.u / Hkv, h = s.u - b * Hkv;
+    // Q fragments for heads mt*16 .. mt*16+15 of this unit's group
+    uint32_t qa[D / 16][4];
+    {
+      const int r0 = mt * 16 + g, r1 = r0 + 8;
+      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(
+          a.q + ((size_t)b * a.Hq + (size_t)h * a.G + r0) * D);
+      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(
+          a.q + ((size_t)b * a.Hq + (size_t)h * a.G + r1) * D);
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        qa[ks][0] = r0 < a.G ? q0[ks * 8 + t4] : 0u;
+        qa[ks][1] = r1 < a.G ? q1[ks * 8 + t4] : 0u;
+        qa[ks][2] = r0 < a.G ? q0[ks * 8 + 4 + t4] : 0u;
+        qa[ks][3] = r1 < a.G ? q1[ks * 8 + 4 + t4] : 0u;
+      }
+    }
+    float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
+    float acc[D / 8][4];
+#pragma unroll
+    for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
+
+    for (int t = s.lo; t < s.hi; t += kTileKeys, ++it) {
+      const int st = it % kStages;
+      if (!mbar_wait(&full[st], (it / kStages) & 1, abort_flag)) { alive = false; break; }
+      const uint32_t kbase = smem_u32(smem + L::kRing + st * L::kStageBytes);
+      const uint32_t vbase = kbase + L::kTileBytes;
+      // ---- S = Q K^T for keys kq*16 .. kq*16+15 of the tile
+      float sc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+#pragma unroll
+      for (int ks = 0; ks < D / 16; ++ks) {
+        // matrices: (keys +0..7, d chunk 2ks), (keys +0..7, chunk 2ks+1),
+        //           (keys +8..15, chunk 2ks), (keys +8..15, chunk 2ks+1)
+        const int mi = lane >> 3, r = lane & 7;
+        const uint32_t key = kq * 16 + (mi >> 1) * 8 + r;
+        const uint32_t chunk = 2 * ks + (mi & 1);
+        const uint32_t addr = kbase + (chunk >> 3) * (kTileKeys * 128) + sw128_offset(key, chunk & 7);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(addr, b0, b1, b2, b3);
+        mma_bf16_16816(sc[0], qa[ks], b0, b1);
+        mma_bf16_16816(sc[1], qa[ks], b2, b3);
+      }
+      // ---- mask, scale (log2 domain), online softmax
+      const int kfirst = t + kq * 16;
+      float mx[2] = {-INFINITY, -INFINITY};
+#pragma unroll
+      for (int n = 0; n < 2; ++n)
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const int key = kfirst + n * 8 + 2 * t4 + (e & 1);
+          const float v = key < s.hi ? sc[n][e] * a.scale_log2 : -INFINITY;
+          sc[n][e] = v;
+          mx[e >> 1] = fmaxf(mx[e >> 1], v);
+        }
+      float alpha[2], mu[2];
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 1));
+        mx[r] = fmaxf(mx[r], __shfl_xor_sync(0xffffffffu, mx[r], 2));
+        const float mn = fmaxf(m[r], mx[r]);
+        mu[r] = mn == -INFINITY ? 0.f : mn;
+        alpha[r] = exp2_approx(m[r] - mu[r]);
+        m[r] = mn;
+      }
+      uint32_t pa[4];
+      float rs[2] = {0.f, 0.f};
+#pragma unroll
+      for (int n = 0; n < 2; ++n) {
+        const float p0 = exp2_approx(sc[n][0] - mu[0]);
+        const float p1 = exp2_approx(sc[n][1] - mu[0]);
+        const float p2 = exp2_approx(sc[n][2] - mu[1]);
+        const float p3 = exp2_approx(sc[n][3] - mu[1]);
+        rs[0] += p0 + p1;
+        rs[1] += p2 + p3;
+        pa[2 * n + 0] = pack_bf16x2(p0, p1);
+        pa[2 * n + 1] = pack_bf16x2(p2, p3);
+      }
+      l[0] = l[0] * alpha[0] + rs[0];
+      l[1] = l[1] * alpha[1] + rs[1];
+#pragma unroll
+      for (int n = 0; n < D / 8; ++n) {
+        acc[n][0] *= alpha[0]; acc[n][1] *= alpha[0];
+        acc[n][2] *= alpha[1]; acc[n][3] *= alpha[1];
+      }
+      // ---- O += P V over keys kq*16 .. +15 (V rows), d in steps of 16
+#pragma unroll
+      for (int dn = 0; dn < D / 16; ++dn) {
+        // matrices: (keys +0..7, chunk 2dn), (keys +8..15, chunk 2dn),
+        //           (keys +0..7, chunk 2dn+1), (keys +8..15, chunk 2dn+1)
+        const int mi = lane >> 3, r = lane & 7;
+        const uint32_t key = kq * 16 + (mi & 1) * 8 + r;
+        const uint32_t chunk = 2 * dn + (mi >> 1);
+        const uint32_t addr = vbase + (chunk >> 3) * (kTileKeys * 128) + sw128_offset(key, chunk & 7);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(addr, b0, b1, b2, b3);
+        mma_bf16_16816(acc[2 * dn], pa, b0, b1);
+        mma_bf16_16816(acc[2 * dn + 1], pa, b2, b3);
+      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&empty[st]);
+    }
+    if (!alive) break;
+
+    // ---- merge the four key quarters of each head tile
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      l[r] += __shfl_xor_sync(0xffffffffu, l[r], 1);
+      l[r] += __shfl_xor_sync(0xffffffffu, l[r], 2);
+    }
+    if (t4 == 0) {
+      mbuf[(kq * 4 + mt) * 16 + g] = m[0];
+      mbuf[(kq * 4 + mt) * 16 + g + 8] = m[1];
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads));
+    float f[2], M[2];
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      float mm = -INFINITY;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) mm = fmaxf(mm, mbuf[(q * 4 + mt) * 16 + g + 8 * r]);
+      M[r] = mm;
+      f[r] = mm == -INFINITY ? 0.f : exp2_approx(m[r] - mm);
+    }
+    float* ob = obuf + mt * 16 * D;
+    for (int q = 0; q < 4; ++q) {
+      if (kq == q) {
+#pragma unroll
+        for (int n = 0; n < D / 8; ++n) {
+          const int c = n * 8 + 2 * t4;
+          float* o0 = ob + g * D + c;
+          float* o1 = ob + (g + 8) * D + c;
+          if (q == 0) {
+            o0[0] = acc[n][0] * f[0]; o0[1] = acc[n][1] * f[0];
+            o1[0] = acc[n][2] * f[1]; o1[1] = acc[n][3] * f[1];
+          } else {
+            o0[0] += acc[n][0] * f[0]; o0[1] += acc[n][1] * f[0];
+            o1[0] += acc[n][2] * f[1]; o1[1] += acc[n][3] * f[1];
+          }
+        }
+        if (t4 == 0) {
+          if (q == 0) { lbuf[mt * 16 + g] = l[0] * f[0]; lbuf[mt * 16 + g + 8] = l[1] * f[1]; }
+          else { lbuf[mt * 16 + g] += l[0] * f[0]; lbuf[mt * 16 + g + 8] += l[1] * f[1]; }
+        }
+      }
+      asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads));
+    }
+    // ---- write the partial of slot (blockIdx.x + unit)
+    const size_t slot = (size_t)blockIdx.x + s.u;
+    for (int idx = threadIdx.x; idx < MT * 16 * D; idx += kConsumerThreads) {
+      const int row = idx / D, c = idx - row * D;   // row = mt*16 + r
+      if (row < a.G) {
+        const float lv = lbuf[row];
+        a.part_o[(slot * a.G + row) * D + c] = lv > 0.f ? obuf[idx] / lv : 0.f;
+      }
+    }
+    if (kq == 0 && t4 == 0) {
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = mt * 16 + g + 8 * r;
+        if (row < a.G) {
+          const float lv = lbuf[row];
+          a.part_lse[slot * a.G + row] = lv > 0.f ? M[r] + __log2f(lv) : -INFINITY;
+        }
+      }
+    }
+    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads));   // obuf/mbuf reused next segment
+  }
+}
+
+// Combine: one CTA per (unit, 16 heads); reads the slots of the unit.
+struct CombineArgs {
+  const int32_t* key_lens;
+  const float* part_o;
+  const float* part_lse;
+  __nv_bfloat16* o;
+  float* lse;
+  int B, Hq, Hkv, Nk, G, grid;
+};
+
+template <int D>
+__global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
+  __shared__ long long s_pb[2];
+  __shared__ int s_len;
+  __shared__ float s_w[64][16];   // per slot weight for each of 16 heads
+  __shared__ float s_lse[16];
+  const int u = blockIdx.x, b = u / a.Hkv, h = u - b * a.Hkv;
+  const int g0 = blockIdx.y * 16;
+  if (threadIdx.x == 0) {
+    long long pb = 0;
+    for (int bb = 0; bb < b; ++bb) {
+      int len = a.key_lens ? a.key_lens[bb] : a.Nk;
+      pb += len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+    }
+    long long tot = pb;
+    int lenb = 0;
+    for (int bb = b; bb < a.B; ++bb) {
+      int len = a.key_lens ? a.key_lens[bb] : a.Nk;
+      len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+      if (bb == b) lenb = len;
+      tot += len;
+    }
+    s_pb[0] = (long long)a.Hkv * pb + (long long)h * lenb;   // unit start
+    s_pb[1] = (long long)a.Hkv * tot;                        // T
+    s_len = lenb;
+  }
+  __syncthreads();
+  const long long p0 = s_pb[0], T = s_pb[1];
+  const int len = s_len;
+  const int rows = (a.G - g0) < 16 ? (a.G - g0) : 16;
+  if (len == 0) {
+    for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
+      const int r = idx / D, c = idx - r * D;
+      a.o[(((size_t)b * a.Hq) + (size_t)h * a.G + g0 + r) * D + c] = __float2bfloat16(0.f);
+    }
+    if (a.lse && threadIdx.x < rows) a.lse[(size_t)b * a.Hq + h * a.G + g0 + threadIdx.x] = -INFINITY;
+    return;
+  }
+  // CTAs whose ranges intersect [p0, p0 + len)
+  auto cta_of = [&](long long x) -> int {
+    long long c = (x * a.grid) / T;
+    while (c + 1 < a.grid && T * (c + 1) / a.grid <= x) ++c;
+    while (c > 0 && T * c / a.grid > x) --c;
+    return (int)c;
+  };
+  const int c0 = cta_of(p0), c1 = cta_of(p0 + len - 1);
+  const int ns = c1 - c0 + 1;
+  // weights: lse over slots, per head (thread r < rows handles head r)
+  if (threadIdx.x < rows) {
+    const int r = threadIdx.x;
+    float mx = -INFINITY;
+    for (int c = c0; c <= c1; ++c)
+      mx = fmaxf(mx, a.part_lse[((size_t)c + u) * a.G + g0 + r]);
+    float sum = 0.f;
+    for (int c = c0; c <= c1; ++c)
+      sum += exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - mx);
+    const float L2 = mx + __log2f(sum);
+    s_lse[r] = L2;
+    for (int c = c0; c <= c1 && c - c0 < 64; ++c)
+      s_w[c - c0][r] = exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - L2);
+    if (a.lse) a.lse[(size_t)b * a.Hq + h * a.G + g0 + r] = L2 * kLn2;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
+    const int r = idx / D, c = idx - r * D;
+    float accv = 0.f;
+    for (int k = 0; k < ns; ++k) {
+      const float w = k < 64 ? s_w[k][r]
+                             : exp2_approx(a.part_lse[((size_t)(c0 + k) + u) * a.G + g0 + r] - s_lse[r]);
+      accv += w * a.part_o[(((size_t)(c0 + k) + u) * a.G + g0 + r) * D + c];
+    }
+    a.o[(((size_t)b * a.Hq) + (size_t)h * a.G + g0 + r) * D + c] = __float2bfloat16(accv);
+  }
+}
+
+// ------------------------------------------------------------------ host side
+
+namespace {
+template <int D, int MT>
+int launch_decode_t(const DecodePlan& p, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const DecodeArgs& a, cudaStream_t st) {
+  auto kern = decode_split_kernel<D, MT>;
+  const int smem = DecodeSmem<D>::kTotal;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ECUDA;
+  kern<<<p.grid, (MT * 4 + 1) * 32, smem, st>>>(tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+}  // namespace
+
+DecodePlan decode_plan(int B, int Hq, int Hkv, int d, int num_sms) {
+  DecodePlan p;
+  p.grid = num_sms;   // one CTA per SM (the ring takes most of shared memory)
+  p.G = Hq / Hkv;
+  p.slots = (size_t)p.grid + (size_t)B * Hkv;
+  p.part_o_bytes = ((p.slots * p.G * d * sizeof(float)) + 255) & ~size_t(255);
+  p.part_lse_bytes = ((p.slots * p.G * sizeof(float)) + 255) & ~size_t(255);
+  p.workspace_bytes = p.part_o_bytes + p.part_lse_bytes;
+  return p;
+}
+
+bool decode_supported(int B, int Hq, int Hkv, int d) {
+  const int G = Hq / Hkv;
+  return (d == 64 || d == 128) && G >= 1 && G <= 64 && B <= kMaxScanB;
+}
+
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                  int Hkv, int Nk, int d, float scale, const int32_t* key_lens, void* workspace,
+                  const DecodePlan& p, cudaStream_t st) {
+  CUtensorMap tk, tv;
+  const uint64_t rows = (uint64_t)B * Hkv * Nk;
+  if (make_tmap_2d_bf16(&tk, k, d, rows, 64, kTileKeys) != ATTN_OK) return ATTN_ECUDA;
+  if (make_tmap_2d_bf16(&tv, v, d, rows, 64, kTileKeys) != ATTN_OK) return ATTN_ECUDA;
+  DecodeArgs a;
+  a.q = static_cast<const __nv_bfloat16*>(q);
+  a.key_lens = key_lens;
+  a.part_o = static_cast<float*>(workspace);
+  a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.part_o_bytes);
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = p.G; a.grid = p.grid;
+  a.scale_log2 = scale * kLog2e;
+  const int MT = (p.G + 15) / 16;
+  int rc;
+  if (d == 128) {
+    rc = MT == 1 ? launch_decode_t<128, 1>(p, tk, tv, a, st)
+       : MT == 2 ? launch_decode_t<128, 2>(p, tk, tv, a, st)
+                 : launch_decode_t<128, 4>(p, tk, tv, a, st);
+  } else {
+    rc = MT == 1 ? launch_decode_t<64, 1>(p, tk, tv, a, st)
+       : MT == 2 ? launch_decode_t<64, 2>(p, tk, tv, a, st)
+                 : launch_decode_t<64, 4>(p, tk, tv, a, st);
+  }
+  if (rc != ATTN_OK) return rc;
+  CombineArgs c;
+  c.key_lens = key_lens;
+  c.part_o = a.part_o;
+  c.part_lse = a.part_lse;
+  c.o = static_cast<__nv_bfloat16*>(o);
+  c.lse = lse;
+  c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.Nk = Nk; c.G = p.G; c.grid = p.grid;
+  dim3 cg(B * Hkv, (p.G + 15) / 16);
+  if (d == 128) decode_combine_kernel<128><<<cg, 256, 0, st>>>(c);
+  else decode_combine_kernel<64><<<cg, 256, 0, st>>>(c);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+}  // namespace attn

@@ -1,0 +1,136 @@
+/*
+ * attn.h -- C ABI of the B200 (sm_100a) exact scaled-dot-product attention
+ * forward library (libattn_b200.so).
+ *
+ * The operation ("Attention mechanisms: from alignment to efficient long
+ * context", sections 3, 5, 9 and 19; "Transformer Architecture Breakdown ...",
+ * section 1.2):
+ *
+ *     O = softmax(Q K^T * scale + M) V,    lse = log(sum(exp(Q K^T * scale + M)))
+ *
+ * computed tile by tile with the online-softmax recurrence (running max m,
+ * running sum l, rescale factor alpha; "Coding interview (14): attention from
+ * scratch", section 3.7; "Transformer Architecture Deconstructed ...", online
+ * softmax), so the Nq x Nk score matrix never reaches device memory.
+ *
+ * Conventions shared by every entry point
+ *   - Tensors are caller-owned DEVICE memory, row-major and contiguous:
+ *       q   bf16 [B, Hq,  Nq, d]      k, v  bf16 [B, Hkv, Nk, d]
+ *       o   bf16 [B, Hq,  Nq, d]      lse   fp32 [B, Hq, Nq]   (natural log)
+ *     Query head h reads kv head h / (Hq / Hkv) (MHA: Hkv = Hq, MQA: Hkv = 1;
+ *     "Attention mechanisms ...", sections 8 and 9).
+ *   - The mask M is never materialised.  Key j is visible to query row i of
+ *     batch b iff j < key_lens[b] and, when causal, j <= i + (Nk - Nq)
+ *     (lower-triangular for Nq == Nk; bottom-right aligned otherwise, as in
+ *     the multi-token decode mask of "Coding interview (14)", self-test 5).
+ *     Masked entries get exactly zero weight (-inf).  A row with no visible
+ *     key gets O = 0 and lse = -inf.
+ *   - key_lens: DEVICE int32 [B] or NULL (= Nk for every batch).  Values are
+ *     clamped to [0, Nk] by the kernels; keys at or beyond key_lens[b] must
+ *     hold finite values (they are read by whole tiles, then masked).
+ *   - stream: a cudaStream_t passed as void*.  Calls only enqueue work on it
+ *     and never synchronise; results are valid once the stream reaches them.
+ *   - Pointers must be 16-byte aligned.  No call retains or frees a caller
+ *     pointer.
+ *   - Return value: an attn_status.  Argument checks happen on the host
+ *     before any launch; nothing is printed and nothing throws.
+ */
+#ifndef ATTN_B200_H
+#define ATTN_B200_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define ATTN_API __attribute__((visibility("default")))
+#else
+#define ATTN_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  ATTN_OK = 0,
+  ATTN_EINVAL = 1,        /* null required pointer, bad size, Hq % Hkv != 0, bad scale */
+  ATTN_EUNSUPPORTED = 2,  /* a shape this build does not implement (e.g. d not 64/128) */
+  ATTN_EALIGN = 3,        /* a pointer not 16-byte aligned */
+  ATTN_EWORKSPACE = 4,    /* workspace missing or smaller than attn_workspace_size() */
+  ATTN_ECUDA = 5,         /* a CUDA runtime / driver call failed (launch, attribute) */
+  ATTN_ETIMEOUT = 6       /* a kernel gave up waiting on a barrier (device status) */
+} attn_status;
+
+/* Exact attention forward.  Dispatch: Nq == 1 runs the split-KV decode kernel
+ * followed by the log-sum-exp combine pass; Nq > 1 runs the tiled prefill
+ * kernel (TMA + tcgen05/TMEM).
+ *   d: 64 or 128.  scale: finite and > 0 (usually 1/sqrt(d); "Transformer
+ *   Architecture Breakdown ...", section 1.2).  causal: 0 or 1 (ignored in
+ *   effect for Nq == 1, where j <= Nk - 1 always holds).
+ *   lse may be NULL.  The decode path needs scratch for its partial results:
+ *   this entry point uses a workspace owned by the library (allocated on
+ *   first use per device, grown on demand, released at process exit); decode
+ *   calls that overlap on the GPU share it and must not run concurrently --
+ *   use attn_fwd_ws for concurrent streams.
+ * Errors: ATTN_EINVAL / EUNSUPPORTED / EALIGN before any launch; ATTN_ECUDA
+ * if a launch or the workspace allocation fails. */
+ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+             int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+             float scale, const int32_t* key_lens, void* stream);
+
+/* attn_fwd with a caller-owned device workspace of at least
+ * attn_workspace_size(...) bytes (256-byte aligned).  The prefill path uses
+ * none (workspace may be NULL when Nq > 1).  The workspace must stay
+ * untouched until the stream has passed this call. */
+ATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* o,
+                float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                int causal, float scale, const int32_t* key_lens,
+                void* workspace, size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_fwd_ws needs for these sizes on the current device
+ * (0 for Nq > 1). */
+ATTN_API size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
+/* RoPE prologue ("Transformer Architecture Breakdown ...", section 3.1;
+ * "Coding interview (14)", section 3.5): for each row x of x_in at position
+ * t = pos_offset + row index along N, and i = 0..d/2-1,
+ *     theta_i = base^(-2i/d),  (a, b) -> (a cos t*theta_i - b sin t*theta_i,
+ *                                         a sin t*theta_i + b cos t*theta_i)
+ * pairing 0: (a, b) = (x_i, x_{i+d/2});  pairing 1: (a, b) = (x_{2i}, x_{2i+1}).
+ *   x_in, x_out: DEVICE bf16 [B, H, N, d]; x_out == x_in (in place) allowed,
+ *   partial overlap is not.  d even, 2 <= d <= 256.  base > 0, finite.
+ *   The angle is formed and reduced in fp64; the rotation runs in fp32; the
+ *   result is rounded to bf16 (nearest even). */
+ATTN_API int rope_apply(const void* x_in, void* x_out, int B, int H, int N, int d,
+               float base, int pos_offset, int pairing, void* stream);
+
+/* Tile shape (query rows Br, keys Bc) the prefill kernel uses for head
+ * dimension d.  Returns ATTN_EUNSUPPORTED for other d. */
+ATTN_API int attn_prefill_tile_shape(int d, int* Br, int* Bc);
+
+/* The KV-tile range the prefill kernel visits for every (b, query tile):
+ * writes first[b * nqt + qt] and count[b * nqt + qt] (nqt = ceil(Nq / Br);
+ * first = -1, count = 0 when the tile sees no key).  Runs the same device
+ * function the prefill kernel uses.  first/count: DEVICE int32 [B * nqt]. */
+ATTN_API int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal,
+                       const int32_t* key_lens, int32_t* first,
+                       int32_t* count, void* stream);
+
+/* Synchronises `stream`, then returns ATTN_ETIMEOUT if any kernel of this
+ * library on the current device gave up on a barrier wait since the last
+ * reset, else ATTN_OK (ATTN_ECUDA if the synchronisation failed).  reset != 0
+ * clears the device status word. */
+ATTN_API int attn_device_status(void* stream, int reset);
+
+/* Human-readable name of a status code (static string). */
+ATTN_API const char* attn_strerror(int status);
+
+/* ABI version of this header (incremented on incompatible changes). */
+ATTN_API int attn_abi_version(void);
+
+#define ATTN_ABI_VERSION 1
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -35,7 +35,7 @@ def lib():
         L.oracle_visible_prefix.argtypes = [i64, i64, i64, i32, i64]
         L.oracle_visible_prefix.restype = i64
         L.oracle_attn_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f64,
-                                       vp, i32, f64, i32, i64, i64, vp, i64, vp, vp, i32]
+                                       vp, i32, f64, i32, i32, i64, i64, vp, i64, vp, vp, i32]
         L.oracle_attn_rows.restype = i32
         L.oracle_attn_online_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32,
                                               f64, vp, i64, vp, i64, vp, vp, i32]
@@ -106,7 +106,9 @@ def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
     """Naive fp64 attention for the listed flat rows (all rows if None).
 
     q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] as bf16 bit patterns.  rope_cfg: None or
-    dict(base=, pairing=, q_pos_offset=, k_pos_offset=).  Returns (o [n,d], lse [n]).
+    dict(base=, pairing=, q_pos_offset=, k_pos_offset=, round_bf16=) -- round_bf16
+    rounds the rotated rows to bf16 (a RoPE pass with bf16 output feeding the
+    attention).  Returns (o [n,d], lse [n]).
     """
     q, k, v, kl, r, (B, Hq, Hkv, Nq, Nk, d), nrows = _prep(q, k, v, key_lens, rows)
     o = np.empty((nrows, d), np.float64)
@@ -115,7 +117,8 @@ def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
     st = lib().oracle_attn_rows(
         _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale),
         _ptr(kl), int(rope_cfg is not None), float(rc.get("base", 10000.0)),
-        int(rc.get("pairing", 0)), int(rc.get("q_pos_offset", 0)), int(rc.get("k_pos_offset", 0)),
+        int(rc.get("pairing", 0)), int(bool(rc.get("round_bf16", False))),
+        int(rc.get("q_pos_offset", 0)), int(rc.get("k_pos_offset", 0)),
         _ptr(r), nrows, _ptr(o), _ptr(lse), int(nthreads or default_threads()))
     if st != 0:
         raise ValueError("oracle_attn_rows rejected its arguments")

@@ -22,6 +22,17 @@ static double bf16_bits_to_double(uint16_t h) {
   return (double)f;
 }
 
+/* double -> nearest bf16 value (via fp32, then round-to-nearest-even on the
+ * upper 16 bits), returned as a double.  Models a bf16 store. */
+static double round_to_bf16(double x) {
+  float f = (float)x;
+  uint32_t u;
+  memcpy(&u, &f, sizeof u);
+  u = (u + 0x7FFFu + ((u >> 16) & 1u)) & 0xFFFF0000u;
+  memcpy(&f, &u, sizeof f);
+  return (double)f;
+}
+
 /* ---- softmax / logsumexp ([CIA] 3.1) ---------------------------------- */
 
 void oracle_softmax(const double* x, int64_t n, double* out) {
@@ -117,6 +128,7 @@ typedef struct {
   int rope;
   double rope_base;
   int rope_pairing;
+  int rope_round; /* round rotated q/k rows to bf16 (composed-pipeline check) */
   int64_t q_pos_offset, k_pos_offset;
   int64_t block; /* > 0: online recurrence with this block size */
   const int64_t* rows;
@@ -142,6 +154,8 @@ static void load_key(job_t* J, const uint16_t* base_ptr, int64_t b,
         double* row = J->kcache + jj * d;
         for (int64_t c = 0; c < d; ++c) row[c] = bf16_bits_to_double(src[c]);
         rope_row(row, d, J->k_pos_offset + jj, J->rope_base, J->rope_pairing);
+        if (J->rope_round)
+          for (int64_t c = 0; c < d; ++c) row[c] = round_to_bf16(row[c]);
       }
       J->kcache_bg = bg;
     }
@@ -150,8 +164,11 @@ static void load_key(job_t* J, const uint16_t* base_ptr, int64_t b,
   }
   const uint16_t* src = base_ptr + ((b * J->Hkv + g) * J->Nk + j) * d;
   for (int64_t c = 0; c < d; ++c) dst[c] = bf16_bits_to_double(src[c]);
-  if (rotate)
+  if (rotate) {
     rope_row(dst, d, J->k_pos_offset + j, J->rope_base, J->rope_pairing);
+    if (J->rope_round)
+      for (int64_t c = 0; c < d; ++c) dst[c] = round_to_bf16(dst[c]);
+  }
 }
 
 /* One output row, naive definition: all visible scores, stable softmax,
@@ -168,8 +185,11 @@ static void row_naive(job_t* J, int64_t r, double* qrow, double* krow,
 
   const uint16_t* qsrc = J->q + r * d;
   for (int64_t c = 0; c < d; ++c) qrow[c] = bf16_bits_to_double(qsrc[c]);
-  if (J->rope)
+  if (J->rope) {
     rope_row(qrow, d, J->q_pos_offset + i, J->rope_base, J->rope_pairing);
+    if (J->rope_round)
+      for (int64_t c = 0; c < d; ++c) qrow[c] = round_to_bf16(qrow[c]);
+  }
 
   for (int64_t j = 0; j < n; ++j) {
     load_key(J, J->k, b, g, j, J->rope, krow);
@@ -301,7 +321,7 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                      int64_t Nk, int64_t d, int causal, double scale,
                      const int32_t* key_lens, int rope, double rope_base,
-                     int rope_pairing, int64_t q_pos_offset,
+                     int rope_pairing, int rope_round, int64_t q_pos_offset,
                      int64_t k_pos_offset, const int64_t* rows, int64_t nrows,
                      double* o, double* lse, int nthreads) {
   job_t J;
@@ -310,6 +330,7 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d;
   J.causal = causal; J.scale = scale; J.key_lens = key_lens;
   J.rope = rope; J.rope_base = rope_base; J.rope_pairing = rope_pairing;
+  J.rope_round = rope_round;
   J.q_pos_offset = q_pos_offset; J.k_pos_offset = k_pos_offset;
   J.block = 0; J.rows = rows; J.nrows = nrows; J.o = o; J.lse = lse;
   return run_rows(&J, nthreads);

@@ -60,14 +60,16 @@ int64_t oracle_visible_prefix(int64_t i, int64_t Nq, int64_t Nk, int causal,
  * rows: flat row ids r = (b*Hq + h)*Nq + i, or NULL for every row in order.
  * o: [nrows, d] doubles; lse: [nrows] (may be NULL).
  * rope != 0 rotates q at position q_pos_offset + i and k at k_pos_offset + j
- * (unrounded fp64) before the dot product.
+ * in fp64 before the dot product; rope_round != 0 then rounds the rotated
+ * rows to bf16 (nearest even), which models a RoPE pass that stores bf16
+ * before the attention reads it.
  * key_lens: int32[B] or NULL (= Nk).  nthreads >= 1.
  * Returns 0, or -1 on invalid arguments. */
 int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                      int64_t Nk, int64_t d, int causal, double scale,
                      const int32_t* key_lens, int rope, double rope_base,
-                     int rope_pairing, int64_t q_pos_offset,
+                     int rope_pairing, int rope_round, int64_t q_pos_offset,
                      int64_t k_pos_offset, const int64_t* rows, int64_t nrows,
                      double* o, double* lse, int nthreads);
 

@@ -1,0 +1,103 @@
+"""The C ABI without a GPU: the library loads, exports every function that
+include/attn.h declares, and rejects bad arguments on the host before any
+CUDA call."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import exact_scaled_dot_fwd_b200 as eb
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_functions():
+    names = []
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            src = open(os.path.join(ROOT, "include", fn)).read()
+            names += re.findall(r"ATTN_API\s+[\w\s\*]+?\b(\w+)\s*\(", src)
+    return sorted(set(names))
+
+
+@pytest.fixture(scope="module")
+def L():
+    from exact_scaled_dot_fwd_b200 import build
+    build.build()
+    return eb.lib()
+
+
+def test_every_declared_symbol_is_exported(L):
+    names = declared_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+    assert L.attn_abi_version() == 1
+
+
+def test_strerror(L):
+    for code, name in eb.STATUS_NAMES.items():
+        assert L.attn_strerror(code).decode().startswith(name)
+    assert L.attn_strerror(99) == b"unknown attn status"
+
+
+P = ctypes.c_void_p(0x1000)      # aligned, never dereferenced by these calls
+U = ctypes.c_void_p(0x1001)      # misaligned
+
+
+def fwd(L, q=P, k=P, v=P, o=P, lse=None, B=1, Hq=2, Hkv=2, Nq=8, Nk=8, d=64, causal=0,
+        scale=0.125, key_lens=None):
+    return L.attn_fwd(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, None)
+
+
+def test_attn_fwd_rejects_bad_arguments_on_host(L):
+    assert fwd(L, q=None) == 1
+    assert fwd(L, o=None) == 1
+    assert fwd(L, B=0) == 1
+    assert fwd(L, Nk=-1) == 1
+    assert fwd(L, Hq=3, Hkv=2) == 1
+    assert fwd(L, causal=2) == 1
+    assert fwd(L, scale=0.0) == 1
+    assert fwd(L, scale=float("nan")) == 1
+    assert fwd(L, scale=float("inf")) == 1
+    assert fwd(L, d=96) == 2
+    assert fwd(L, d=32) == 2
+    assert fwd(L, q=U) == 3
+    assert fwd(L, v=U) == 3
+
+
+def test_attn_fwd_ws_rejects_missing_workspace(L):
+    # decode needs a workspace; the size query needs a device, so on a
+    # CPU-only host the call fails before any launch either way
+    rc = L.attn_fwd_ws(P, P, P, P, None, 2, 4, 1, 1, 64, 64, 0, 0.125, None, None, 0, None)
+    assert rc in (4, 5)
+
+
+def test_rope_rejects_bad_arguments_on_host(L):
+    r = L.rope_apply
+    assert r(None, P, 1, 1, 8, 64, 1e4, 0, 0, None) == 1
+    assert r(P, P, 1, 1, 8, 63, 1e4, 0, 0, None) == 1       # odd d
+    assert r(P, P, 1, 1, 8, 64, -1.0, 0, 0, None) == 1      # base
+    assert r(P, P, 1, 1, 8, 64, 1e4, 0, 2, None) == 1       # pairing
+    assert r(P, P, 1, 1, 8, 64, 1e4, -1, 0, None) == 1      # negative position
+    assert r(P, P, 1, 1, 8, 512, 1e4, 0, 0, None) == 2
+    assert r(U, U, 1, 1, 8, 64, 1e4, 0, 0, None) == 3
+    # partial overlap of input and output
+    assert r(ctypes.c_void_p(0x1000), ctypes.c_void_p(0x1010), 1, 1, 8, 64, 1e4, 0, 0, None) == 1
+
+
+def test_tile_shape_and_plan_args(L):
+    br, bc = ctypes.c_int(), ctypes.c_int()
+    assert L.attn_prefill_tile_shape(128, ctypes.byref(br), ctypes.byref(bc)) == 0
+    assert br.value > 0 and bc.value > 0
+    assert L.attn_prefill_tile_shape(96, ctypes.byref(br), ctypes.byref(bc)) == 2
+    assert L.attn_fwd_tile_plan(1, 8, 8, 64, 0, None, None, P, None) == 1
+    assert L.attn_fwd_tile_plan(1, 8, 8, 64, 3, None, P, P, None) == 1
+
+
+def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
+    monkeypatch.setattr(eb, "LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(eb, "_lib", None)
+    with pytest.raises(OSError):
+        eb.lib()

@@ -417,6 +417,18 @@ def test_attention_with_rope_matches_library_on_rotated_inputs():
         V = f64(v).repeat_interleave(2, 1)
         O = F.scaled_dot_product_attention(Q, K, V, is_causal=True, scale=1 / math.sqrt(d))
         assert np.max(np.abs(o - O.numpy().reshape(-1, d))) < 1e-13
+        # round_bf16: the rotated rows pass through a bf16 store first
+        cfg["round_bf16"] = True
+        o_r, _ = oracle.attn_rows(q, k, v, True, 1 / math.sqrt(d), rope_cfg=cfg)
+
+        def rnd(a):
+            return torch.from_numpy(synth.bf16_bits_to_f32(
+                synth.bf16_bits_from_f32(a.astype(np.float32))).astype(np.float64))
+        Qr = rnd(oracle.rope(q, pos_offset=5, pairing=pairing))
+        Kr = rnd(oracle.rope(k, pos_offset=5, pairing=pairing)).repeat_interleave(2, 1)
+        Or = F.scaled_dot_product_attention(Qr, Kr, V, is_causal=True, scale=1 / math.sqrt(d))
+        assert np.max(np.abs(o_r - Or.numpy().reshape(-1, d))) < 1e-13
+        assert np.max(np.abs(o_r - o)) > 1e-6
 
 
 # ------------------------------------------------------------- tile plan ----
