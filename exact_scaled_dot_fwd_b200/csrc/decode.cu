@@ -384,23 +384,31 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
   __shared__ float s_lse[16];
   const int u = blockIdx.x, b = u / a.Hkv, h = u - b * a.Hkv;
   const int g0 = blockIdx.y * 16;
+  // unit start and total key count: block-wide sums over the key lengths
+  __shared__ long long s_red[2][8];
+  long long before = 0, total = 0;
+  for (int bb = threadIdx.x; bb < a.B; bb += blockDim.x) {
+    int len = a.key_lens ? a.key_lens[bb] : a.Nk;
+    len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+    total += len;
+    if (bb < b) before += len;
+    if (bb == b) s_len = len;
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    before += __shfl_xor_sync(0xffffffffu, before, o);
+    total += __shfl_xor_sync(0xffffffffu, total, o);
+  }
+  if ((threadIdx.x & 31) == 0) {
+    s_red[0][threadIdx.x >> 5] = before;
+    s_red[1][threadIdx.x >> 5] = total;
+  }
+  __syncthreads();
   if (threadIdx.x == 0) {
-    long long pb = 0;
-    for (int bb = 0; bb < b; ++bb) {
-      int len = a.key_lens ? a.key_lens[bb] : a.Nk;
-      pb += len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
-    }
-    long long tot = pb;
-    int lenb = 0;
-    for (int bb = b; bb < a.B; ++bb) {
-      int len = a.key_lens ? a.key_lens[bb] : a.Nk;
-      len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
-      if (bb == b) lenb = len;
-      tot += len;
-    }
-    s_pb[0] = (long long)a.Hkv * pb + (long long)h * lenb;   // unit start
-    s_pb[1] = (long long)a.Hkv * tot;                        // T
-    s_len = lenb;
+    long long pb = 0, tot = 0;
+    for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { pb += s_red[0][w]; tot += s_red[1][w]; }
+    s_pb[0] = (long long)a.Hkv * pb + (long long)h * s_len;   // unit start
+    s_pb[1] = (long long)a.Hkv * tot;                         // T
   }
   __syncthreads();
   const long long p0 = s_pb[0], T = s_pb[1];
@@ -423,19 +431,22 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
   };
   const int c0 = cta_of(p0), c1 = cta_of(p0 + len - 1);
   const int ns = c1 - c0 + 1;
+  // CTAs whose global range is empty (T < grid) wrote no slot: weight 0
+  auto nonempty = [&](int c) -> bool { return T * c / a.grid < T * (c + 1) / a.grid; };
   // weights: lse over slots, per head (thread r < rows handles head r)
   if (threadIdx.x < rows) {
     const int r = threadIdx.x;
     float mx = -INFINITY;
     for (int c = c0; c <= c1; ++c)
-      mx = fmaxf(mx, a.part_lse[((size_t)c + u) * a.G + g0 + r]);
+      if (nonempty(c)) mx = fmaxf(mx, a.part_lse[((size_t)c + u) * a.G + g0 + r]);
     float sum = 0.f;
     for (int c = c0; c <= c1; ++c)
-      sum += exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - mx);
+      if (nonempty(c)) sum += exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - mx);
     const float L2 = mx + __log2f(sum);
     s_lse[r] = L2;
     for (int c = c0; c <= c1 && c - c0 < 64; ++c)
-      s_w[c - c0][r] = exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - L2);
+      s_w[c - c0][r] =
+          nonempty(c) ? exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - L2) : 0.f;
     if (a.lse) a.lse[(size_t)b * a.Hq + h * a.G + g0 + r] = L2 * kLn2;
   }
   __syncthreads();
@@ -443,9 +454,14 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
     const int r = idx / D, c = idx - r * D;
     float accv = 0.f;
     for (int k = 0; k < ns; ++k) {
-      const float w = k < 64 ? s_w[k][r]
-                             : exp2_approx(a.part_lse[((size_t)(c0 + k) + u) * a.G + g0 + r] - s_lse[r]);
-      accv += w * a.part_o[(((size_t)(c0 + k) + u) * a.G + g0 + r) * D + c];
+      float w;
+      if (k < 64) {
+        w = s_w[k][r];
+      } else {
+        if (!nonempty(c0 + k)) continue;
+        w = exp2_approx(a.part_lse[((size_t)(c0 + k) + u) * a.G + g0 + r] - s_lse[r]);
+      }
+      if (w != 0.f) accv += w * a.part_o[(((size_t)(c0 + k) + u) * a.G + g0 + r) * D + c];
     }
     a.o[(((size_t)b * a.Hq) + (size_t)h * a.G + g0 + r) * D + c] = __float2bfloat16(accv);
   }

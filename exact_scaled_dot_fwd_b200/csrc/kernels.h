@@ -16,6 +16,12 @@ namespace attn {
 int make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                       uint32_t box_cols, uint32_t box_rows);
 
+// 3D bf16 tensor map over [mats, rows, cols] (row-major) with a box of
+// box_cols x box_rows x 1 and 128-byte swizzling; loads and stores clip at
+// the end of each matrix.
+int make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
+                      uint64_t mats, uint32_t box_cols, uint32_t box_rows);
+
 // ---- decode (Nq == 1)
 struct DecodePlan {
   int grid = 0;          // CTAs of the split kernel (one wave)

@@ -115,6 +115,7 @@ DECODE = [
     (2, 64, 1, 3000, 128, [3000, 2048]),       # 64 query heads on one kv head
     (5, 12, 3, 700, 128, None),                # group of 4, not a multiple of 16
     (300, 32, 1, 50, 128, None),               # more units than CTAs
+    (2, 4, 4, 300, 128, [2, 2]),               # fewer keys than CTAs: empty ranges
 ]
 
 
