@@ -74,6 +74,34 @@ struct Tile {
   int row_tile, head, count, first_masked;
 };
 
+// Of every 8 consecutive score columns, the last kPolyPer8 take 2^x from
+// exp2_poly on the FMA pipe instead of the SFU, which is the scarcer unit:
+// one exponential per score against ~512 tensor FLOPs per score at d = 128.
+constexpr int kPolyPer8 = 3;
+
+__device__ __forceinline__ float max3(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for finite x <= 64 by Cody-Waite range reduction and a polynomial:
+// x = n + f with n = round(x) (the 1.5 * 2^23 shifter leaves n in the low
+// mantissa bits), f in [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted
+// here for minimum maximum relative error on that interval (7.5e-5 in fp32
+// Horner form, far below the bf16 rounding of P); n is added to the
+// exponent field.  x is clamped at -126 so the exponent cannot wrap.
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.f);
+  const float t = x + 12582912.f;
+  const float n = t - 12582912.f;
+  const float f = x - n;
+  const float p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111400127411f), f,
+                            0.6932609677314758f),
+                       f, 0.9999280571937561f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
+}
+
 }  // namespace pf
 
 struct FwdArgs {
@@ -276,14 +304,25 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const int lim = nvis - j * kN;   // keys [0, lim) of this tile are visible
       // pass 1: row max of the (masked) scores
       float mx = -INFINITY;
+      if (!masked) {
 #pragma unroll
-      for (int c4 = 0; c4 < kN / 32; ++c4) {
-        float sv[32];
-        tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
-        tc::wait_ld();
+        for (int c8 = 0; c8 < kN / 64; ++c8) {
+          float sv[64];
+          tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
+          tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
+          tc::wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e)
-          mx = fmaxf(mx, (masked && 32 * c4 + e >= lim) ? -INFINITY : sv[e]);
+          for (int e = 0; e < 32; ++e) mx = max3(mx, sv[2 * e], sv[2 * e + 1]);
+        }
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < kN / 32; ++c4) {
+          float sv[32];
+          tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
+          tc::wait_ld();
+#pragma unroll
+          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, 32 * c4 + e >= lim ? -INFINITY : sv[e]);
+        }
       }
       const float m_tile = mx * a.scale_log2;
       const bool need = m_tile > m_run + kRescaleLog2;
@@ -305,27 +344,52 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         m_run = m_new;
       }
       // pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs over the first
-      // 64 columns of S (chunk c4 reads S columns [32 c4, 32 c4 + 32) and
-      // writes P columns [16 c4, 16 c4 + 16), which were already read)
+      // 64 columns of S (chunk c reads S columns [32 c, 32 c + 32) and
+      // writes P columns [16 c, 16 c + 16), which were already read)
       const float m_use = m_run == -INFINITY ? 0.f : m_run;
+      const float sl2 = a.scale_log2;
       float rs = 0.f;
+      if (!masked) {
 #pragma unroll
-      for (int c4 = 0; c4 < kN / 32; ++c4) {
-        float sv[32];
-        tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
-        tc::wait_ld();
-        uint32_t pk[16];
+        for (int c8 = 0; c8 < kN / 64; ++c8) {
+          float sv[64];
+          tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
+          tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
+          tc::wait_ld();
+          uint32_t pk[32];
 #pragma unroll
-        for (int e = 0; e < 16; ++e) {
-          const int c = 32 * c4 + 2 * e;
-          const float x0 = (masked && c >= lim) ? -INFINITY : sv[2 * e];
-          const float x1 = (masked && c + 1 >= lim) ? -INFINITY : sv[2 * e + 1];
-          const float p0 = exp2_approx(fmaf(x0, a.scale_log2, -m_use));
-          const float p1 = exp2_approx(fmaf(x1, a.scale_log2, -m_use));
-          rs += p0 + p1;
-          pk[e] = pack_bf16x2(p0, p1);
+          for (int e = 0; e < 32; ++e) {
+            const float x0 = fmaf(sv[2 * e], sl2, -m_use);
+            const float x1 = fmaf(sv[2 * e + 1], sl2, -m_use);
+            const bool poly0 = ((2 * e) & 7) >= 8 - kPolyPer8;
+            const bool poly1 = ((2 * e + 1) & 7) >= 8 - kPolyPer8;
+            const float p0 = poly0 ? exp2_poly(x0) : exp2_approx(x0);
+            const float p1 = poly1 ? exp2_poly(x1) : exp2_approx(x1);
+            rs += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tc::st16(tmem + lane_off + scol + 32 * c8, pk);
+          tc::st16(tmem + lane_off + scol + 32 * c8 + 16, pk + 16);
         }
-        tc::st16(tmem + lane_off + scol + 16 * c4, pk);
+      } else {
+#pragma unroll
+        for (int c4 = 0; c4 < kN / 32; ++c4) {
+          float sv[32];
+          tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
+          tc::wait_ld();
+          uint32_t pk[16];
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int c = 32 * c4 + 2 * e;
+            const float x0 = c >= lim ? -INFINITY : sv[2 * e];
+            const float x1 = c + 1 >= lim ? -INFINITY : sv[2 * e + 1];
+            const float p0 = exp2_approx(fmaf(x0, sl2, -m_use));
+            const float p1 = exp2_approx(fmaf(x1, sl2, -m_use));
+            rs += p0 + p1;
+            pk[e] = pack_bf16x2(p0, p1);
+          }
+          tc::st16(tmem + lane_off + scol + 16 * c4, pk);
+        }
       }
       l_run += rs;
       tc::wait_st();
