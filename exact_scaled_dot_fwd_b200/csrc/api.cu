@@ -153,7 +153,9 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
     return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nk, d, scale, key_lens, workspace, p, st);
   }
   if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
-  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, st);
+  const int sms = current_sms();
+  if (sms <= 0) return ATTN_ECUDA;
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, sms, st);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,

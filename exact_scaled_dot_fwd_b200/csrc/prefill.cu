@@ -9,9 +9,12 @@
 // 2^(m_old - m_new); divide by l at the end.  The score tile lives only in
 // TMEM and registers.
 //
-// CTA = two query tiles of 128 rows that share one kv head (rows 2p, 2p+1 of
-// one head, or -- when a kv head serves an even number of query heads -- the
-// same rows of two query heads).  Warp roles:
+// Work item = two query tiles of 128 rows that share one kv head (rows 2p,
+// 2p+1 of one head, or -- when a kv head serves an even number of query heads
+// -- the same rows of two query heads).  The kernel is persistent: one CTA
+// per SM walks the items in a snake order over a list sorted by cost (causal:
+// most KV tiles first), so every SM gets a near-equal share and the next
+// item's loads and first MMAs overlap the current item's tail.  Warp roles:
 //   warps 0-3  softmax for query tile 0 (one row per thread = one TMEM lane)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    tcgen05.mma issuer (one thread) and TMEM allocator
@@ -23,6 +26,9 @@
 // query tile.  tcgen05 MMAs of one thread execute in issue order, so S(j+1)
 // overwrites P(j) only after PV(j) has read it, and the commit after S(j+1)
 // also covers PV(j) -- the softmax may rescale O as soon as S(j+1) is ready.
+//
+// Barrier phases run on across items; each role derives the same item
+// sequence and tile counts, so the counters stay in step.
 //
 // Lazy rescale: O and l are rescaled only when a row's max grows by more
 // than 8 (log2 units); otherwise the stale max is kept (P <= 2^8, exact in
@@ -49,13 +55,14 @@ template <int D>
 struct Smem {
   static constexpr int kBox = 128 * 128;          // one 64-column box of a 128-row tile
   static constexpr int kTile = 128 * D * 2;       // Q, K or V tile
-  static constexpr int kQ = 0;                    // Q[2] (reused as output staging)
+  static constexpr int kQ = 0;                    // Q[2]
   static constexpr int kK = kQ + 2 * kTile;       // K[kKS]
   static constexpr int kV = kK + kKS * kTile;     // V[kVS]
   static constexpr int kBar = kV + kVS * kTile;
   enum {
-    Q_FULL = 0,
-    K_FULL = 1,
+    Q_FULL = 0,                 // [2]
+    Q_EMPTY = 2,                // [2] committed after the last S MMA of a tile
+    K_FULL = 4,
     K_EMPTY = K_FULL + kKS,
     V_FULL = K_EMPTY + kKS,
     V_EMPTY = V_FULL + kVS,
@@ -105,19 +112,81 @@ __device__ __forceinline__ float exp2_poly(float x) {
 }  // namespace pf
 
 struct FwdArgs {
+  __nv_bfloat16* o;
   float* lse;
   const int32_t* key_lens;
   int B, Hq, Hkv, Nq, Nk, causal;
   int head_pairs;   // 1: tiles are heads (2p, 2p+1) at one row tile; 0: row tiles 2p, 2p+1
   int ntq;          // ceil(Nq / 128)
+  int units;        // items per cost rank (head_pairs: B*Hq/2, else B*Hq)
+  int total;        // number of items
   float scale_log2;
 };
+
+namespace pf {
+
+struct Item {
+  Tile tl[2];       // tl[0] has the fewer KV tiles
+  int b, n, kv_row0, L;
+};
+
+// Item `idx` of the cost-sorted list: rank = idx / units walks the row tiles
+// (row pairs) from the most KV tiles to the fewest when causal.
+__device__ __forceinline__ Item make_item(const FwdArgs& a, int idx) {
+  Item it;
+  const int rank = idx / a.units, unit = idx - rank * a.units;
+  if (a.head_pairs) {
+    const int rt = a.causal ? (a.ntq - 1 - rank) : rank;
+    const int hp2 = a.Hq >> 1;
+    it.b = unit / hp2;
+    const int hp = unit - it.b * hp2;
+    it.tl[0].row_tile = it.tl[1].row_tile = rt;
+    it.tl[0].head = 2 * hp;
+    it.tl[1].head = 2 * hp + 1;
+  } else {
+    const int np = (a.ntq + 1) >> 1;
+    const int p = a.causal ? (np - 1 - rank) : rank;
+    it.b = unit / a.Hq;
+    const int h = unit - it.b * a.Hq;
+    it.tl[0].row_tile = 2 * p;
+    it.tl[1].row_tile = 2 * p + 1;
+    it.tl[0].head = it.tl[1].head = h;
+  }
+  it.L = clamp_len(a.key_lens ? a.key_lens[it.b] : a.Nk, a.Nk);
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    if (it.tl[t].row_tile < a.ntq) {
+      const KvRange r = kv_tile_range(it.tl[t].row_tile, kM, kN, a.Nq, a.Nk, a.causal, it.L);
+      it.tl[t].count = r.count;
+      it.tl[t].first_masked = r.first_masked;
+    } else {
+      it.tl[t].count = 0;
+      it.tl[t].first_masked = 0;
+    }
+  }
+  if (it.tl[0].count > it.tl[1].count) {
+    const Tile x = it.tl[0];
+    it.tl[0] = it.tl[1];
+    it.tl[1] = x;
+  }
+  it.n = it.tl[1].count;
+  const int hk = it.tl[1].head / (a.Hq / a.Hkv);
+  it.kv_row0 = (it.b * a.Hkv + hk) * a.Nk;
+  return it;
+}
+
+// k-th item of CTA c in the snake order (or -1 past the end).
+__device__ __forceinline__ int snake_item(int k, int c, int grid, int total) {
+  const int idx = k * grid + ((k & 1) ? (grid - 1 - c) : c);
+  return idx < total ? idx : -1;
+}
+
+}  // namespace pf
 
 template <int D>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
-                      const __grid_constant__ CUtensorMap tv, const __grid_constant__ CUtensorMap to,
-                      FwdArgs a) {
+                      const __grid_constant__ CUtensorMap tv, FwdArgs a) {
   using namespace pf;
   using L = Smem<D>;
   constexpr int kBoxes = D / 64;
@@ -133,43 +202,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int b = blockIdx.z;
-  const int G = a.Hq / a.Hkv;
-  const int L_b = clamp_len(a.key_lens ? a.key_lens[b] : a.Nk, a.Nk);
-
-  // ---- the two query tiles of this CTA (heaviest CTAs first when causal)
-  Tile tl[2];
-  if (a.head_pairs) {
-    const int rt = a.causal ? (a.ntq - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-    tl[0].row_tile = tl[1].row_tile = rt;
-    tl[0].head = 2 * blockIdx.y;
-    tl[1].head = 2 * blockIdx.y + 1;
-  } else {
-    const int np = (a.ntq + 1) >> 1;
-    const int p = a.causal ? (np - 1 - (int)blockIdx.x) : (int)blockIdx.x;
-    tl[0].row_tile = 2 * p;
-    tl[1].row_tile = 2 * p + 1;
-    tl[0].head = tl[1].head = blockIdx.y;
-  }
-#pragma unroll
-  for (int t = 0; t < 2; ++t) {
-    if (tl[t].row_tile < a.ntq) {
-      const KvRange r = kv_tile_range(tl[t].row_tile, kM, kN, a.Nq, a.Nk, a.causal, L_b);
-      tl[t].count = r.count;
-      tl[t].first_masked = r.first_masked;
-    } else {
-      tl[t].count = 0;
-      tl[t].first_masked = 0;
-    }
-  }
-  if (tl[0].count > tl[1].count) {   // tile 0 is the one with fewer KV tiles
-    const Tile x = tl[0];
-    tl[0] = tl[1];
-    tl[1] = x;
-  }
-  const int n = tl[1].count;
-  const int hk = tl[1].head / G;
-  const int kv_row0 = (b * a.Hkv + hk) * a.Nk;
+  const int cta = blockIdx.x, grid = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
@@ -191,95 +224,115 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 
   if (warp == 9) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      uint32_t qbytes = 0;
-      for (int t = 0; t < 2; ++t) qbytes += tl[t].count > 0 ? L::kTile : 0;
-      mbar_arrive_expect_tx(&bars[L::Q_FULL], qbytes);
-      for (int t = 0; t < 2; ++t) {
-        if (tl[t].count == 0) continue;
-        for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_3d(smem + L::kQ + t * L::kTile + bx * L::kBox, &tq, bx * 64,
-                      tl[t].row_tile * kM, b * a.Hq + tl[t].head, &bars[L::Q_FULL]);
-      }
-      for (int j = 0; j < n; ++j) {
-        const int ks = j % kKS;
-        if (!mbar_wait(&bars[L::K_EMPTY + ks], ((j / kKS) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kTile);
-        for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(smem + L::kK + ks * L::kTile + bx * L::kBox, &tk, bx * 64, kv_row0 + j * kN,
-                      &bars[L::K_FULL + ks]);
-        const int vs = j % kVS;
-        if (!mbar_wait(&bars[L::V_EMPTY + vs], ((j / kVS) & 1) ^ 1, abort_flag)) break;
-        mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kTile);
-        for (int bx = 0; bx < kBoxes; ++bx)
-          tma_load_2d(smem + L::kV + vs * L::kTile + bx * L::kBox, &tv, bx * 64, kv_row0 + j * kN,
-                      &bars[L::V_FULL + vs]);
+      int qn[2] = {0, 0}, g = 0;
+      bool ok = true;
+      for (int k = 0, idx; ok && (idx = snake_item(k, cta, grid, a.total)) >= 0; ++k) {
+        const Item it = make_item(a, idx);
+        if (it.n == 0) continue;
+        for (int t = 0; t < 2 && ok; ++t) {
+          if (it.tl[t].count == 0) continue;
+          if (qn[t] > 0 && !mbar_wait(&bars[L::Q_EMPTY + t], (qn[t] - 1) & 1, abort_flag)) {
+            ok = false;
+            break;
+          }
+          ++qn[t];
+          mbar_arrive_expect_tx(&bars[L::Q_FULL + t], L::kTile);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_3d(smem + L::kQ + t * L::kTile + bx * L::kBox, &tq, bx * 64,
+                        it.tl[t].row_tile * kM, it.b * a.Hq + it.tl[t].head, &bars[L::Q_FULL + t]);
+        }
+        for (int j = 0; ok && j < it.n; ++j, ++g) {
+          const int ks = g % kKS;
+          if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / kKS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kTile);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(smem + L::kK + ks * L::kTile + bx * L::kBox, &tk, bx * 64,
+                        it.kv_row0 + j * kN, &bars[L::K_FULL + ks]);
+          const int vs = g % kVS;
+          if (!mbar_wait(&bars[L::V_EMPTY + vs], ((g / kVS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kTile);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(smem + L::kV + vs * L::kTile + bx * L::kBox, &tv, bx * 64,
+                        it.kv_row0 + j * kN, &bars[L::V_FULL + vs]);
+        }
       }
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && n > 0) {
+    if (lane == 0) {
       const uint32_t q_base = smem_u32(smem + L::kQ);
       const uint32_t k_base = smem_u32(smem + L::kK);
       const uint32_t v_base = smem_u32(smem + L::kV);
       auto issue_s = [&](int t, int ks) {
         const uint32_t qa = q_base + t * L::kTile, kb = k_base + ks * L::kTile;
 #pragma unroll
-        for (int k = 0; k < D / 16; ++k) {
-          const uint32_t off = (k >> 2) * L::kBox + (k & 3) * 32;
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
           tc::mma_ss(tmem + 128u * t, tc::smem_desc_sw128(qa + off, 16, 1024),
-                     tc::smem_desc_sw128(kb + off, 16, 1024), kIdescS, k > 0 ? 1u : 0u);
+                     tc::smem_desc_sw128(kb + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
         }
       };
       auto issue_pv = [&](int t, int vs, bool acc) {
         const uint32_t vb = v_base + vs * L::kTile;
 #pragma unroll
-        for (int k = 0; k < kN / 16; ++k) {
-          tc::mma_ts(tmem + 256u + D * t, tmem + 128u * t + k * 8,
-                     tc::smem_desc_sw128(vb + k * 16 * 128, L::kBox, 1024), kIdescPV,
-                     (acc || k > 0) ? 1u : 0u);
+        for (int kk = 0; kk < kN / 16; ++kk) {
+          tc::mma_ts(tmem + 256u + D * t, tmem + 128u * t + kk * 8,
+                     tc::smem_desc_sw128(vb + kk * 16 * 128, L::kBox, 1024), kIdescPV,
+                     (acc || kk > 0) ? 1u : 0u);
         }
       };
-      bool ok = mbar_wait(&bars[L::Q_FULL], 0, abort_flag) &&
-                mbar_wait(&bars[L::K_FULL + 0], 0, abort_flag);
-      if (ok) {
-        tc::fence_after();
-        for (int t = 0; t < 2; ++t)
-          if (tl[t].count > 0) {
-            issue_s(t, 0);
-            tc::commit(&bars[L::S_FULL + t]);
-          }
-        tc::commit(&bars[L::K_EMPTY + 0]);
-      }
-      for (int j = 0; ok && j < n; ++j) {
-        const int vs = j % kVS, ksn = (j + 1) % kKS;
-        if (!mbar_wait(&bars[L::V_FULL + vs], (j / kVS) & 1, abort_flag)) { ok = false; break; }
-        bool k_next = false;
+      int qf[2] = {0, 0}, pw[2] = {0, 0}, g = 0;
+      bool ok = true;
+      for (int k = 0, idx; ok && (idx = snake_item(k, cta, grid, a.total)) >= 0; ++k) {
+        const Item it = make_item(a, idx);
+        if (it.n == 0) continue;
+        const int g0 = g;
+        if (!mbar_wait(&bars[L::K_FULL + g0 % kKS], (g0 / kKS) & 1, abort_flag)) { ok = false; break; }
         for (int t = 0; t < 2 && ok; ++t) {
-          if (j >= tl[t].count) continue;
-          if (!mbar_wait(&bars[L::P_FULL + t], j & 1, abort_flag)) { ok = false; break; }
+          if (it.tl[t].count == 0) continue;
+          if (!mbar_wait(&bars[L::Q_FULL + t], qf[t] & 1, abort_flag)) { ok = false; break; }
+          ++qf[t];
           tc::fence_after();
-          issue_pv(t, vs, j > 0);
-          if (j + 1 < tl[t].count) {
-            if (!k_next) {
-              if (!mbar_wait(&bars[L::K_FULL + ksn], ((j + 1) / kKS) & 1, abort_flag)) {
-                ok = false;
-                break;
-              }
-              tc::fence_after();
-              k_next = true;
-            }
-            issue_s(t, ksn);
-            tc::commit(&bars[L::S_FULL + t]);
-          } else {
-            tc::commit(&bars[L::O_FULL + t]);
-          }
+          issue_s(t, g0 % kKS);
+          tc::commit(&bars[L::S_FULL + t]);
+          if (it.tl[t].count == 1) tc::commit(&bars[L::Q_EMPTY + t]);
         }
-        tc::commit(&bars[L::V_EMPTY + vs]);
-        if (k_next) tc::commit(&bars[L::K_EMPTY + ksn]);
+        if (!ok) break;
+        tc::commit(&bars[L::K_EMPTY + g0 % kKS]);
+        for (int j = 0; ok && j < it.n; ++j, ++g) {
+          const int vs = g % kVS, ksn = (g + 1) % kKS;
+          if (!mbar_wait(&bars[L::V_FULL + vs], (g / kVS) & 1, abort_flag)) { ok = false; break; }
+          bool k_next = false;
+          for (int t = 0; t < 2 && ok; ++t) {
+            const int cnt = it.tl[t].count;
+            if (j >= cnt) continue;
+            if (!mbar_wait(&bars[L::P_FULL + t], pw[t] & 1, abort_flag)) { ok = false; break; }
+            ++pw[t];
+            tc::fence_after();
+            issue_pv(t, vs, j > 0);
+            if (j + 1 < cnt) {
+              if (!k_next) {
+                if (!mbar_wait(&bars[L::K_FULL + ksn], ((g + 1) / kKS) & 1, abort_flag)) {
+                  ok = false;
+                  break;
+                }
+                tc::fence_after();
+                k_next = true;
+              }
+              issue_s(t, ksn);
+              tc::commit(&bars[L::S_FULL + t]);
+              if (j + 2 == cnt) tc::commit(&bars[L::Q_EMPTY + t]);
+            } else {
+              tc::commit(&bars[L::O_FULL + t]);
+            }
+          }
+          tc::commit(&bars[L::V_EMPTY + vs]);
+          if (k_next) tc::commit(&bars[L::K_EMPTY + ksn]);
+        }
       }
       // every MMA of this CTA must be complete before TMEM is released
       tc::commit(&bars[L::MMA_DONE]);
@@ -287,123 +340,131 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax
-    const int t = warp >> 2;                 // query tile of this warpgroup
+    const int t = warp >> 2;                 // query tile slot of this warpgroup
     const int r = (warp & 3) * 32 + lane;    // row within the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t scol = 128u * t, ocol = 256u + D * t;
-    const Tile T = t == 0 ? tl[0] : tl[1];
-    const int row = T.row_tile * kM + r;
-    const int nvis = visible_prefix(row, a.Nq, a.Nk, a.causal, L_b);
-    float m_run = -INFINITY, l_run = 0.f;
+    const float sl2 = a.scale_log2;
+    int sw = 0, ow = 0;
     bool ok = true;
+    for (int k = 0, idx; ok && (idx = snake_item(k, cta, grid, a.total)) >= 0; ++k) {
+      const Item it = make_item(a, idx);
+      const Tile T = t == 0 ? it.tl[0] : it.tl[1];
+      if (T.row_tile >= a.ntq) continue;
+      const int row = T.row_tile * kM + r;
+      const int nvis = visible_prefix(row, a.Nq, a.Nk, a.causal, it.L);
+      float m_run = -INFINITY, l_run = 0.f;
 
-    for (int j = 0; j < T.count; ++j) {
-      if (!mbar_wait(&bars[L::S_FULL + t], j & 1, abort_flag)) { ok = false; break; }
-      tc::fence_after();
-      const bool masked = j >= T.first_masked;
-      const int lim = nvis - j * kN;   // keys [0, lim) of this tile are visible
-      // pass 1: row max of the (masked) scores
-      float mx = -INFINITY;
-      if (!masked) {
+      for (int j = 0; j < T.count; ++j) {
+        if (!mbar_wait(&bars[L::S_FULL + t], sw & 1, abort_flag)) { ok = false; break; }
+        ++sw;
+        tc::fence_after();
+        const bool masked = j >= T.first_masked;
+        const int lim = nvis - j * kN;   // keys [0, lim) of this tile are visible
+        // pass 1: row max of the (masked) scores
+        float mx = -INFINITY;
+        if (!masked) {
 #pragma unroll
-        for (int c8 = 0; c8 < kN / 64; ++c8) {
-          float sv[64];
-          tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
-          tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
-          tc::wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = max3(mx, sv[2 * e], sv[2 * e + 1]);
-        }
-      } else {
-#pragma unroll
-        for (int c4 = 0; c4 < kN / 32; ++c4) {
-          float sv[32];
-          tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
-          tc::wait_ld();
-#pragma unroll
-          for (int e = 0; e < 32; ++e) mx = fmaxf(mx, 32 * c4 + e >= lim ? -INFINITY : sv[e]);
-        }
-      }
-      const float m_tile = mx * a.scale_log2;
-      const bool need = m_tile > m_run + kRescaleLog2;
-      if (__any_sync(0xffffffffu, need)) {
-        const float m_new = need ? fmaxf(m_run, m_tile) : m_run;
-        if (j > 0) {
-          const float f = (need && m_run != -INFINITY) ? exp2_approx(m_run - m_new) : 1.f;
-          l_run *= f;
-#pragma unroll
-          for (int c = 0; c < D / 32; ++c) {
-            float o[32];
-            tc::ld32f(tmem + lane_off + ocol + 32 * c, o);
+          for (int c8 = 0; c8 < kN / 64; ++c8) {
+            float sv[64];
+            tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
+            tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
             tc::wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) o[e] *= f;
-            tc::st32f(tmem + lane_off + ocol + 32 * c, o);
+            for (int e = 0; e < 32; ++e) mx = max3(mx, sv[2 * e], sv[2 * e + 1]);
+          }
+        } else {
+#pragma unroll
+          for (int c4 = 0; c4 < kN / 32; ++c4) {
+            float sv[32];
+            tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
+            tc::wait_ld();
+#pragma unroll
+            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, 32 * c4 + e >= lim ? -INFINITY : sv[e]);
           }
         }
-        m_run = m_new;
+        const float m_tile = mx * sl2;
+        const bool need = m_tile > m_run + kRescaleLog2;
+        if (__any_sync(0xffffffffu, need)) {
+          const float m_new = need ? fmaxf(m_run, m_tile) : m_run;
+          if (j > 0) {
+            const float f = (need && m_run != -INFINITY) ? exp2_approx(m_run - m_new) : 1.f;
+            l_run *= f;
+#pragma unroll
+            for (int c = 0; c < D / 32; ++c) {
+              float o[32];
+              tc::ld32f(tmem + lane_off + ocol + 32 * c, o);
+              tc::wait_ld();
+#pragma unroll
+              for (int e = 0; e < 32; ++e) o[e] *= f;
+              tc::st32f(tmem + lane_off + ocol + 32 * c, o);
+            }
+          }
+          m_run = m_new;
+        }
+        // pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs over the first
+        // 64 columns of S (chunk c reads S columns [64 c, 64 c + 64) and
+        // writes P columns [32 c, 32 c + 32), which were already read)
+        const float m_use = m_run == -INFINITY ? 0.f : m_run;
+        float rs = 0.f;
+        if (!masked) {
+#pragma unroll
+          for (int c8 = 0; c8 < kN / 64; ++c8) {
+            float sv[64];
+            tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
+            tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
+            tc::wait_ld();
+            uint32_t pk[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              const float x0 = fmaf(sv[2 * e], sl2, -m_use);
+              const float x1 = fmaf(sv[2 * e + 1], sl2, -m_use);
+              const bool poly0 = ((2 * e) & 7) >= 8 - kPolyPer8;
+              const bool poly1 = ((2 * e + 1) & 7) >= 8 - kPolyPer8;
+              const float p0 = poly0 ? exp2_poly(x0) : exp2_approx(x0);
+              const float p1 = poly1 ? exp2_poly(x1) : exp2_approx(x1);
+              rs += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            tc::st16(tmem + lane_off + scol + 32 * c8, pk);
+            tc::st16(tmem + lane_off + scol + 32 * c8 + 16, pk + 16);
+          }
+        } else {
+#pragma unroll
+          for (int c4 = 0; c4 < kN / 32; ++c4) {
+            float sv[32];
+            tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
+            tc::wait_ld();
+            uint32_t pk[16];
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = 32 * c4 + 2 * e;
+              const float x0 = c >= lim ? -INFINITY : sv[2 * e];
+              const float x1 = c + 1 >= lim ? -INFINITY : sv[2 * e + 1];
+              const float p0 = exp2_approx(fmaf(x0, sl2, -m_use));
+              const float p1 = exp2_approx(fmaf(x1, sl2, -m_use));
+              rs += p0 + p1;
+              pk[e] = pack_bf16x2(p0, p1);
+            }
+            tc::st16(tmem + lane_off + scol + 16 * c4, pk);
+          }
+        }
+        l_run += rs;
+        tc::wait_st();
+        tc::fence_before();
+        mbar_arrive(&bars[L::P_FULL + t]);
       }
-      // pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs over the first
-      // 64 columns of S (chunk c reads S columns [32 c, 32 c + 32) and
-      // writes P columns [16 c, 16 c + 16), which were already read)
-      const float m_use = m_run == -INFINITY ? 0.f : m_run;
-      const float sl2 = a.scale_log2;
-      float rs = 0.f;
-      if (!masked) {
-#pragma unroll
-        for (int c8 = 0; c8 < kN / 64; ++c8) {
-          float sv[64];
-          tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
-          tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
-          tc::wait_ld();
-          uint32_t pk[32];
-#pragma unroll
-          for (int e = 0; e < 32; ++e) {
-            const float x0 = fmaf(sv[2 * e], sl2, -m_use);
-            const float x1 = fmaf(sv[2 * e + 1], sl2, -m_use);
-            const bool poly0 = ((2 * e) & 7) >= 8 - kPolyPer8;
-            const bool poly1 = ((2 * e + 1) & 7) >= 8 - kPolyPer8;
-            const float p0 = poly0 ? exp2_poly(x0) : exp2_approx(x0);
-            const float p1 = poly1 ? exp2_poly(x1) : exp2_approx(x1);
-            rs += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          tc::st16(tmem + lane_off + scol + 32 * c8, pk);
-          tc::st16(tmem + lane_off + scol + 32 * c8 + 16, pk + 16);
-        }
-      } else {
-#pragma unroll
-        for (int c4 = 0; c4 < kN / 32; ++c4) {
-          float sv[32];
-          tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
-          tc::wait_ld();
-          uint32_t pk[16];
-#pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int c = 32 * c4 + 2 * e;
-            const float x0 = c >= lim ? -INFINITY : sv[2 * e];
-            const float x1 = c + 1 >= lim ? -INFINITY : sv[2 * e + 1];
-            const float p0 = exp2_approx(fmaf(x0, sl2, -m_use));
-            const float p1 = exp2_approx(fmaf(x1, sl2, -m_use));
-            rs += p0 + p1;
-            pk[e] = pack_bf16x2(p0, p1);
-          }
-          tc::st16(tmem + lane_off + scol + 16 * c4, pk);
-        }
-      }
-      l_run += rs;
-      tc::wait_st();
-      tc::fence_before();
-      mbar_arrive(&bars[L::P_FULL + t]);
-    }
+      if (!ok) break;
 
-    // ---- epilogue: O / l -> bf16 -> shared staging -> TMA store; lse
-    const bool have = ok && T.count > 0;
-    if (have && !mbar_wait(&bars[L::O_FULL + t], 0, abort_flag)) ok = false;
-    if (ok && T.row_tile < a.ntq) {
-      tc::fence_after();
+      // ---- epilogue: O / l -> bf16 straight to global; lse
+      const bool have = T.count > 0;
+      if (have) {
+        if (!mbar_wait(&bars[L::O_FULL + t], ow & 1, abort_flag)) { ok = false; break; }
+        ++ow;
+        tc::fence_after();
+      }
       const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
-      uint8_t* stage = smem + L::kQ + t * L::kTile;
+      __nv_bfloat16* orow = a.o + (((size_t)it.b * a.Hq + T.head) * a.Nq + row) * D;
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float o[32];
@@ -414,28 +475,22 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 #pragma unroll
           for (int e = 0; e < 32; ++e) o[e] = 0.f;
         }
+        if (row < a.Nq) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {   // four 16-byte chunks of 8 columns
-          const int gc = 4 * c + q;      // global 16-byte chunk index in the row
-          uint4 v;
-          v.x = pack_bf16x2((o[8 * q + 0]) * inv, (o[8 * q + 1]) * inv);
-          v.y = pack_bf16x2((o[8 * q + 2]) * inv, (o[8 * q + 3]) * inv);
-          v.z = pack_bf16x2((o[8 * q + 4]) * inv, (o[8 * q + 5]) * inv);
-          v.w = pack_bf16x2((o[8 * q + 6]) * inv, (o[8 * q + 7]) * inv);
-          *reinterpret_cast<uint4*>(stage + (gc >> 3) * L::kBox + sw128_offset(r, gc & 7)) = v;
+          for (int q = 0; q < 4; ++q) {
+            uint4 v;
+            v.x = pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+            v.y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+            v.z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+            v.w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = v;
+          }
         }
       }
+      tc::fence_before();
       if (a.lse && row < a.Nq)
-        a.lse[((size_t)b * a.Hq + T.head) * a.Nq + row] =
+        a.lse[((size_t)it.b * a.Hq + T.head) * a.Nq + row] =
             l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
-      fence_proxy_async_smem();
-      asm volatile("bar.sync %0, 128;" ::"r"(1 + t));
-      if (r == 0) {
-        for (int bx = 0; bx < kBoxes; ++bx)
-          tma_store_3d(&to, stage + bx * L::kBox, bx * 64, T.row_tile * kM, b * a.Hq + T.head);
-        bulk_commit();
-        bulk_wait_read0();
-      }
     }
   }
 
@@ -459,35 +514,36 @@ void prefill_tile_shape(int d, int* Br, int* Bc) {
 
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, float scale,
-                   const int32_t* key_lens, cudaStream_t st) {
-  CUtensorMap tq, tk, tv, to;
+                   const int32_t* key_lens, int num_sms, cudaStream_t st) {
+  CUtensorMap tq, tk, tv;
   if (make_tmap_3d_bf16(&tq, q, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
-  if (make_tmap_3d_bf16(&to, o, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tk, k, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tv, v, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
   FwdArgs a;
+  a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.key_lens = key_lens;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.causal = causal;
   a.ntq = (Nq + pf::kM - 1) / pf::kM;
   a.head_pairs = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
   a.scale_log2 = scale * kLog2e;
-  dim3 grid;
-  if (a.head_pairs) grid = dim3(a.ntq, Hq / 2, B);
-  else grid = dim3((a.ntq + 1) / 2, Hq, B);
-  if (grid.y > 65535 || grid.z > 65535) return ATTN_EUNSUPPORTED;
+  a.units = a.head_pairs ? B * (Hq / 2) : B * Hq;
+  const long long total = (long long)a.units * (a.head_pairs ? a.ntq : (a.ntq + 1) / 2);
+  if (total >= (1ll << 31)) return ATTN_EUNSUPPORTED;
+  a.total = (int)total;
+  const int grid = a.total < num_sms ? a.total : num_sms;
   if (d == 128) {
     auto kern = prefill_tc_kernel<128>;
     const int smem = pf::Smem<128>::kTotal;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return ATTN_ECUDA;
-    kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, to, a);
+    kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, a);
   } else {
     auto kern = prefill_tc_kernel<64>;
     const int smem = pf::Smem<64>::kTotal;
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
       return ATTN_ECUDA;
-    kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, to, a);
+    kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, a);
   }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
