@@ -35,6 +35,8 @@
 // the final O / l because O and l share the same reference).
 #include <cuda_bf16.h>
 
+#include <cmath>
+
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
@@ -46,8 +48,9 @@ namespace pf {
 
 constexpr int kM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kN = 128;        // keys per KV tile
-constexpr int kKS = 2;         // K ring stages
-constexpr int kVS = 2;         // V ring stages
+// K/V ring stages: d = 128 fits three K and two V tiles beside the two Q
+// tiles (224 KB); d = 64 fits three of each.
+template <int D> struct Stages { static constexpr int K = 3, V = D == 128 ? 2 : 3; };
 constexpr int kThreads = 320;
 constexpr float kRescaleLog2 = 8.0f;
 
@@ -56,6 +59,7 @@ struct Smem {
   static constexpr int kBox = 128 * 128;          // one 64-column box of a 128-row tile
   static constexpr int kTile = 128 * D * 2;       // Q, K or V tile
   static constexpr int kQ = 0;                    // Q[2]
+  static constexpr int kKS = Stages<D>::K, kVS = Stages<D>::V;
   static constexpr int kK = kQ + 2 * kTile;       // K[kKS]
   static constexpr int kV = kK + kKS * kTile;     // V[kVS]
   static constexpr int kBar = kV + kVS * kTile;
@@ -75,38 +79,17 @@ struct Smem {
   static constexpr int kTmemSlot = kBar + NUM_BARS * 8;
   static constexpr int kAbort = kTmemSlot + 16;
   static constexpr int kTotal = kAbort + 16 + 1024;   // + alignment slack
+  static_assert(kTotal <= 232448, "shared memory over the 227 KB per-CTA limit");
 };
 
 struct Tile {
   int row_tile, head, count, first_masked;
 };
 
-// Of every 8 consecutive score columns, the last kPolyPer8 take 2^x from
-// exp2_poly on the FMA pipe instead of the SFU, which is the scarcer unit:
-// one exponential per score against ~512 tensor FLOPs per score at d = 128.
-constexpr int kPolyPer8 = 3;
-
 __device__ __forceinline__ float max3(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^x for finite x <= 64 by Cody-Waite range reduction and a polynomial:
-// x = n + f with n = round(x) (the 1.5 * 2^23 shifter leaves n in the low
-// mantissa bits), f in [-0.5, 0.5]; 2^f from a degree-3 polynomial fitted
-// here for minimum maximum relative error on that interval (7.5e-5 in fp32
-// Horner form, far below the bf16 rounding of P); n is added to the
-// exponent field.  x is clamped at -126 so the exponent cannot wrap.
-__device__ __forceinline__ float exp2_poly(float x) {
-  x = fmaxf(x, -126.f);
-  const float t = x + 12582912.f;
-  const float n = t - 12582912.f;
-  const float f = x - n;
-  const float p = fmaf(fmaf(fmaf(0.0551716685295105f, f, 0.2426111400127411f), f,
-                            0.6932609677314758f),
-                       f, 0.9999280571937561f);
-  return __int_as_float(__float_as_int(p) + (__float_as_int(t) << 23));
 }
 
 }  // namespace pf
@@ -119,6 +102,8 @@ struct FwdArgs {
   int head_pairs;   // 1: tiles are heads (2p, 2p+1) at one row tile; 0: row tiles 2p, 2p+1
   int ntq;          // ceil(Nq / 128)
   int units;        // items per cost rank (head_pairs: B*Hq/2, else B*Hq)
+  int ranks;        // cost ranks (row tiles, or row-tile pairs)
+  int band;         // ranks per band (item order: band, unit, rank in band)
   int total;        // number of items
   float scale_log2;
 };
@@ -130,11 +115,24 @@ struct Item {
   int b, n, kv_row0, L;
 };
 
-// Item `idx` of the cost-sorted list: rank = idx / units walks the row tiles
-// (row pairs) from the most KV tiles to the fewest when causal.
+// Item `idx` of the ordered list.  Ranks walk the row tiles (row pairs)
+// from the most KV tiles to the fewest when causal; bands of `band` ranks
+// keep one unit's (head's) items next to each other so the CTAs that run at
+// the same time share its K/V in L2 (band = 1: plain rank-major order).
 __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx) {
   Item it;
-  const int rank = idx / a.units, unit = idx - rank * a.units;
+  const int per_band = a.units * a.band;
+  const int full = a.ranks / a.band;
+  int rank, unit;
+  if (idx < full * per_band) {
+    const int bi = idx / per_band, rem = idx - bi * per_band;
+    unit = rem / a.band;
+    rank = bi * a.band + (rem - unit * a.band);
+  } else {
+    const int lb = a.ranks - full * a.band, rem = idx - full * per_band;
+    unit = rem / lb;
+    rank = full * a.band + (rem - unit * lb);
+  }
   if (a.head_pairs) {
     const int rt = a.causal ? (a.ntq - 1 - rank) : rank;
     const int hp2 = a.Hq >> 1;
@@ -190,6 +188,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   using namespace pf;
   using L = Smem<D>;
   constexpr int kBoxes = D / 64;
+  constexpr int kKS = L::kKS, kVS = L::kVS;
   // TMEM columns: S of tile t at 128 t, O of tile t at 256 + D t
   constexpr uint32_t kIdescS = tc::idesc_bf16(kM, kN, false, false);
   constexpr uint32_t kIdescPV = tc::idesc_bf16(kM, D, false, true);
@@ -419,10 +418,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             for (int e = 0; e < 32; ++e) {
               const float x0 = fmaf(sv[2 * e], sl2, -m_use);
               const float x1 = fmaf(sv[2 * e + 1], sl2, -m_use);
-              const bool poly0 = ((2 * e) & 7) >= 8 - kPolyPer8;
-              const bool poly1 = ((2 * e + 1) & 7) >= 8 - kPolyPer8;
-              const float p0 = poly0 ? exp2_poly(x0) : exp2_approx(x0);
-              const float p1 = poly1 ? exp2_poly(x1) : exp2_approx(x1);
+              const float p0 = exp2_approx(x0);
+              const float p1 = exp2_approx(x1);
               rs += p0 + p1;
               pk[e] = pack_bf16x2(p0, p1);
             }
@@ -528,10 +525,23 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   a.head_pairs = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
   a.scale_log2 = scale * kLog2e;
   a.units = a.head_pairs ? B * (Hq / 2) : B * Hq;
-  const long long total = (long long)a.units * (a.head_pairs ? a.ntq : (a.ntq + 1) / 2);
+  a.ranks = a.head_pairs ? a.ntq : (a.ntq + 1) / 2;
+  const long long total = (long long)a.units * a.ranks;
   if (total >= (1ll << 31)) return ATTN_EUNSUPPORTED;
   a.total = (int)total;
   const int grid = a.total < num_sms ? a.total : num_sms;
+  // Band size: plain rank order while all of K/V fits comfortably in L2;
+  // otherwise enough ranks per band that the heads in flight (about
+  // grid / band) keep their K/V within ~64 MB of L2.
+  const double kv_head = 4.0 * (double)Nk * d;   // K + V bytes of one kv head
+  const double kv_all = kv_head * B * Hkv;
+  int band = 1;
+  if (kv_all > 64.0 * (1 << 20)) {
+    band = (int)ceil(grid * kv_head / (64.0 * (1 << 20)));
+    if (band > a.ranks) band = a.ranks;
+    if (band < 1) band = 1;
+  }
+  a.band = band;
   if (d == 128) {
     auto kern = prefill_tc_kernel<128>;
     const int smem = pf::Smem<128>::kTotal;
