@@ -245,10 +245,8 @@ def run_ours(args):
     kl = None if x["key_lens"] is None else torch.from_numpy(x["key_lens"]).to(device)
     O = torch.empty_like(Q[0])
     LSE = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
-    ws = None
-    if w.Nq == 1:
-        ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, 1, w.Nk, w.d),
-                         dtype=torch.uint8, device=device)
+    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d),
+                     dtype=torch.uint8, device=device)
 
     if w.rope:
         QR = torch.empty_like(Q[0])
@@ -281,7 +279,8 @@ def run_ours(args):
     ms = time_steps(step, steps, torch, dist, stream)
     clocks = sampler.stop()
     ms_step = ms / steps
-    launches_per_step = (2 if w.Nq == 1 else 1) + (2 if w.rope else 0)
+    # decode: split + combine; prefill: the scheduler-counter memset + kernel
+    launches_per_step = 2 + (2 if w.rope else 0)
     # the dominant kernel alone (differs from the step only when RoPE runs)
     ms_kernel = ms if not w.rope else time_steps(attn_only, steps, torch, dist, stream)
     if w.Nq == 1:

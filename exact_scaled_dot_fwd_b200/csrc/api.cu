@@ -130,7 +130,8 @@ const char* attn_strerror(int status) {
 
 size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   (void)Nk;
-  if (Nq != 1 || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
+  if (Nq <= 0 || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
+  if (Nq > 1) return prefill_workspace_bytes();
   const int sms = current_sms();
   if (sms <= 0) return 0;
   return decode_plan(B, Hq, Hkv, d, sms).workspace_bytes;
@@ -153,9 +154,12 @@ int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse
     return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nk, d, scale, key_lens, workspace, p, st);
   }
   if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
+  if (!workspace || workspace_bytes < prefill_workspace_bytes()) return ATTN_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
   const int sms = current_sms();
   if (sms <= 0) return ATTN_ECUDA;
-  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, sms, st);
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, workspace,
+                        sms, st);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -165,8 +169,9 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   if (rc != ATTN_OK) return rc;
   void* ws = nullptr;
   size_t ws_bytes = 0;
-  if (Nq == 1) {
-    if (!decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
+  {
+    if (Nq == 1 && !decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
+    if (Nq > 1 && !prefill_supported(d)) return ATTN_EUNSUPPORTED;
     const size_t need = attn_workspace_size(B, Hq, Hkv, Nq, Nk, d);
     if (need == 0) return ATTN_ECUDA;
     int dev = 0;

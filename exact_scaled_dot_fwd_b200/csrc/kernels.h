@@ -37,10 +37,11 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
 
 // ---- prefill (Nq > 1)
 bool prefill_supported(int d);
+size_t prefill_workspace_bytes();   // scheduler counter
 void prefill_tile_shape(int d, int* Br, int* Bc);
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, float scale,
-                   const int32_t* key_lens, int num_sms, cudaStream_t st);
+                   const int32_t* key_lens, void* workspace, int num_sms, cudaStream_t st);
 int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, const int32_t* key_lens,
                      int32_t* first, int32_t* count, cudaStream_t st);
 

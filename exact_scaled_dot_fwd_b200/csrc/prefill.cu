@@ -12,13 +12,16 @@
 // Work item = two query tiles of 128 rows that share one kv head (rows 2p,
 // 2p+1 of one head, or -- when a kv head serves an even number of query heads
 // -- the same rows of two query heads).  The kernel is persistent: one CTA
-// per SM walks the items in a snake order over a list sorted by cost (causal:
-// most KV tiles first), so every SM gets a near-equal share and the next
-// item's loads and first MMAs overlap the current item's tail.  Warp roles:
+// per SM takes items one at a time from a global counter over a list sorted
+// by cost (causal: most KV tiles first) -- greedy longest-first scheduling --
+// and the next item's loads and first MMAs overlap the current item's tail.
+// The K/V producer claims the item and hands its index to the other roles
+// through a small ring in shared memory.  Warp roles:
 //   warps 0-3  softmax for query tile 0 (one row per thread = one TMEM lane)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    tcgen05.mma issuer (one thread) and TMEM allocator
-//   warp  9    TMA producer (one thread)
+//   warp  9    K/V TMA producer and item scheduler (one thread)
+//   warp 10    Q TMA producer (one thread)
 // TMEM (512 columns): S0 | S1 | O0 | O1; P (bf16) is written over the first
 // 64 columns of its S buffer and read by the MMA straight from TMEM.
 // The MMA issue order per KV tile j is PV0(j), S0(j+1), PV1(j), S1(j+1):
@@ -27,8 +30,8 @@
 // overwrites P(j) only after PV(j) has read it, and the commit after S(j+1)
 // also covers PV(j) -- the softmax may rescale O as soon as S(j+1) is ready.
 //
-// Barrier phases run on across items; each role derives the same item
-// sequence and tile counts, so the counters stay in step.
+// Barrier phases run on across items; every role sees the same item
+// sequence and derives the same tile counts, so the counters stay in step.
 //
 // Lazy rescale: O and l are rescaled only when a row's max grows by more
 // than 8 (log2 units); otherwise the stale max is kept (P <= 2^8, exact in
@@ -51,7 +54,10 @@ constexpr int kN = 128;        // keys per KV tile
 // K/V ring stages: d = 128 fits three K and two V tiles beside the two Q
 // tiles (224 KB); d = 64 fits three of each.
 template <int D> struct Stages { static constexpr int K = 3, V = D == 128 ? 2 : 3; };
-constexpr int kThreads = 320;
+constexpr int kThreads = 352;   // 11 warps
+constexpr int kItemSlots = 4;   // depth of the shared-memory ring of work items
+// arrivals that free an item slot: MMA thread, Q producer, 256 softmax threads
+constexpr int kItemReaders = 2 + 256;
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
@@ -74,9 +80,12 @@ struct Smem {
     P_FULL = S_FULL + 2,
     O_FULL = P_FULL + 2,
     MMA_DONE = O_FULL + 2,
-    NUM_BARS = MMA_DONE + 1
+    ITEM_FULL = MMA_DONE + 1,            // [kItemSlots]
+    ITEM_EMPTY = ITEM_FULL + kItemSlots, // [kItemSlots]
+    NUM_BARS = ITEM_EMPTY + kItemSlots
   };
-  static constexpr int kTmemSlot = kBar + NUM_BARS * 8;
+  static constexpr int kItems = kBar + NUM_BARS * 8;      // int [kItemSlots]
+  static constexpr int kTmemSlot = kItems + kItemSlots * 4;
   static constexpr int kAbort = kTmemSlot + 16;
   static constexpr int kTotal = kAbort + 16 + 1024;   // + alignment slack
   static_assert(kTotal <= 232448, "shared memory over the 227 KB per-CTA limit");
@@ -95,6 +104,7 @@ __device__ __forceinline__ float max3(float a, float b, float c) {
 }  // namespace pf
 
 struct FwdArgs {
+  unsigned int* sched;   // item counter, zero at launch
   __nv_bfloat16* o;
   float* lse;
   const int32_t* key_lens;
@@ -173,12 +183,6 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx) {
   return it;
 }
 
-// k-th item of CTA c in the snake order (or -1 past the end).
-__device__ __forceinline__ int snake_item(int k, int c, int grid, int total) {
-  const int idx = k * grid + ((k & 1) ? (grid - 1 - c) : c);
-  return idx < total ? idx : -1;
-}
-
 }  // namespace pf
 
 template <int D>
@@ -201,12 +205,23 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int cta = blockIdx.x, grid = gridDim.x;
+  volatile int* items = reinterpret_cast<volatile int*>(smem + L::kItems);
+  // next item index from the ring (every reader calls it once per item);
+  // -1 ends the stream
+  auto next_item = [&](int& k) -> int {
+    const int slot = k % kItemSlots;
+    if (!mbar_wait(&bars[L::ITEM_FULL + slot], (k / kItemSlots) & 1, abort_flag)) return -1;
+    const int idx = items[slot];
+    mbar_arrive(&bars[L::ITEM_EMPTY + slot]);
+    ++k;
+    return idx;
+  };
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       uint32_t cnt = 1;
       if (i == L::P_FULL || i == L::P_FULL + 1) cnt = 128;
+      if (i >= L::ITEM_EMPTY && i < L::ITEM_EMPTY + kItemSlots) cnt = kItemReaders;
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -222,14 +237,52 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   const uint32_t tmem = *tmem_slot;
 
   if (warp == 9) {
-    // ------------------------------------------------------------ producer
+    // ------------------------------------------------- K/V producer + scheduler
     if (lane == 0) {
-      tma_prefetch_desc(&tq);
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
-      int qn[2] = {0, 0}, g = 0;
+      int g = 0, k = 0;
       bool ok = true;
-      for (int k = 0, idx; ok && (idx = snake_item(k, cta, grid, a.total)) >= 0; ++k) {
+      int idx = (int)atomicAdd(a.sched, 1u);
+      while (ok) {
+        if (idx >= a.total) idx = -1;
+        const int slot = k % kItemSlots;
+        if (!mbar_wait(&bars[L::ITEM_EMPTY + slot], ((k / kItemSlots) & 1) ^ 1, abort_flag)) break;
+        items[slot] = idx;
+        mbar_arrive(&bars[L::ITEM_FULL + slot]);
+        ++k;
+        if (idx < 0) break;
+        const Item it = make_item(a, idx);
+        // claim the next item only while issuing this item's last tile, so
+        // no CTA sits on a claimed item (greedy longest-first stays greedy);
+        // the atomic's latency hides behind the last loads
+        int nxt = -1;
+        if (it.n == 0) nxt = (int)atomicAdd(a.sched, 1u);
+        for (int j = 0; ok && j < it.n; ++j, ++g) {
+          if (j == it.n - 1) nxt = (int)atomicAdd(a.sched, 1u);
+          const int ks = g % kKS;
+          if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / kKS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kTile);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(smem + L::kK + ks * L::kTile + bx * L::kBox, &tk, bx * 64,
+                        it.kv_row0 + j * kN, &bars[L::K_FULL + ks]);
+          const int vs = g % kVS;
+          if (!mbar_wait(&bars[L::V_EMPTY + vs], ((g / kVS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kTile);
+          for (int bx = 0; bx < kBoxes; ++bx)
+            tma_load_2d(smem + L::kV + vs * L::kTile + bx * L::kBox, &tv, bx * 64,
+                        it.kv_row0 + j * kN, &bars[L::V_FULL + vs]);
+        }
+        idx = nxt;
+      }
+    }
+  } else if (warp == 10) {
+    // ------------------------------------------------------------ Q producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tq);
+      int qn[2] = {0, 0}, k = 0;
+      bool ok = true;
+      for (int idx; ok && (idx = next_item(k)) >= 0;) {
         const Item it = make_item(a, idx);
         if (it.n == 0) continue;
         for (int t = 0; t < 2 && ok; ++t) {
@@ -243,20 +296,6 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           for (int bx = 0; bx < kBoxes; ++bx)
             tma_load_3d(smem + L::kQ + t * L::kTile + bx * L::kBox, &tq, bx * 64,
                         it.tl[t].row_tile * kM, it.b * a.Hq + it.tl[t].head, &bars[L::Q_FULL + t]);
-        }
-        for (int j = 0; ok && j < it.n; ++j, ++g) {
-          const int ks = g % kKS;
-          if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / kKS) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kTile);
-          for (int bx = 0; bx < kBoxes; ++bx)
-            tma_load_2d(smem + L::kK + ks * L::kTile + bx * L::kBox, &tk, bx * 64,
-                        it.kv_row0 + j * kN, &bars[L::K_FULL + ks]);
-          const int vs = g % kVS;
-          if (!mbar_wait(&bars[L::V_EMPTY + vs], ((g / kVS) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kTile);
-          for (int bx = 0; bx < kBoxes; ++bx)
-            tma_load_2d(smem + L::kV + vs * L::kTile + bx * L::kBox, &tv, bx * 64,
-                        it.kv_row0 + j * kN, &bars[L::V_FULL + vs]);
         }
       }
     }
@@ -284,69 +323,93 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                      (acc || kk > 0) ? 1u : 0u);
         }
       };
-      int qf[2] = {0, 0}, pw[2] = {0, 0}, g = 0;
+      // Each slot's work is one stream of KV tiles across items: in the step
+      // that finishes item i for one slot, the S MMA of item i+1's first
+      // tile is issued for every slot that is done with item i, so a slot
+      // with fewer tiles moves on while the other one finishes.
+      int qf[2] = {0, 0}, pw[2] = {0, 0}, g = 0, k = 0;
       bool ok = true;
-      for (int k = 0, idx; ok && (idx = snake_item(k, cta, grid, a.total)) >= 0; ++k) {
-        const Item it = make_item(a, idx);
-        if (it.n == 0) continue;
-        const int g0 = g;
-        if (!mbar_wait(&bars[L::K_FULL + g0 % kKS], (g0 / kKS) & 1, abort_flag)) { ok = false; break; }
-        for (int t = 0; t < 2 && ok; ++t) {
-          if (it.tl[t].count == 0) continue;
-          if (!mbar_wait(&bars[L::Q_FULL + t], qf[t] & 1, abort_flag)) { ok = false; break; }
-          ++qf[t];
-          tc::fence_after();
-          issue_s(t, g0 % kKS);
-          tc::commit(&bars[L::S_FULL + t]);
-          if (it.tl[t].count == 1) tc::commit(&bars[L::Q_EMPTY + t]);
+      auto fetch = [&](Item& it) -> bool {   // next item that has KV tiles
+        for (int idx; (idx = next_item(k)) >= 0;) {
+          it = make_item(a, idx);
+          if (it.n > 0) return true;
         }
-        if (!ok) break;
-        tc::commit(&bars[L::K_EMPTY + g0 % kKS]);
-        for (int j = 0; ok && j < it.n; ++j, ++g) {
+        return false;
+      };
+      auto issue_first_s = [&](const Item& it, int t, int ks) -> bool {
+        if (!mbar_wait(&bars[L::Q_FULL + t], qf[t] & 1, abort_flag)) return false;
+        ++qf[t];
+        tc::fence_after();
+        issue_s(t, ks);
+        tc::commit(&bars[L::S_FULL + t]);
+        if (it.tl[t].count == 1) tc::commit(&bars[L::Q_EMPTY + t]);
+        return true;
+      };
+      Item cur, nxt;
+      if (fetch(cur)) {
+        ok = mbar_wait(&bars[L::K_FULL + 0], 0, abort_flag);
+        for (int t = 0; t < 2 && ok; ++t)
+          if (cur.tl[t].count > 0) ok = issue_first_s(cur, t, 0);
+        if (ok) tc::commit(&bars[L::K_EMPTY + 0]);
+        int j = 0;
+        while (ok) {
           const int vs = g % kVS, ksn = (g + 1) % kKS;
+          const bool last = j == cur.n - 1;
+          const bool more = last ? fetch(nxt) : true;
           if (!mbar_wait(&bars[L::V_FULL + vs], (g / kVS) & 1, abort_flag)) { ok = false; break; }
           bool k_next = false;
-          for (int t = 0; t < 2 && ok; ++t) {
-            const int cnt = it.tl[t].count;
-            if (j >= cnt) continue;
-            if (!mbar_wait(&bars[L::P_FULL + t], pw[t] & 1, abort_flag)) { ok = false; break; }
-            ++pw[t];
+          auto need_k = [&]() -> bool {
+            if (k_next) return true;
+            if (!mbar_wait(&bars[L::K_FULL + ksn], ((g + 1) / kKS) & 1, abort_flag)) return false;
             tc::fence_after();
-            issue_pv(t, vs, j > 0);
-            if (j + 1 < cnt) {
-              if (!k_next) {
-                if (!mbar_wait(&bars[L::K_FULL + ksn], ((g + 1) / kKS) & 1, abort_flag)) {
-                  ok = false;
-                  break;
-                }
-                tc::fence_after();
-                k_next = true;
-              }
+            k_next = true;
+            return true;
+          };
+          for (int t = 0; t < 2 && ok; ++t) {
+            const int cnt = cur.tl[t].count;
+            if (j < cnt) {
+              if (!mbar_wait(&bars[L::P_FULL + t], pw[t] & 1, abort_flag)) { ok = false; break; }
+              ++pw[t];
+              tc::fence_after();
+              issue_pv(t, vs, j > 0);
+              if (j == cnt - 1) tc::commit(&bars[L::O_FULL + t]);
+            }
+            if (j + 1 < cnt) {                                 // same item, next tile
+              if (!need_k()) { ok = false; break; }
               issue_s(t, ksn);
               tc::commit(&bars[L::S_FULL + t]);
               if (j + 2 == cnt) tc::commit(&bars[L::Q_EMPTY + t]);
-            } else {
-              tc::commit(&bars[L::O_FULL + t]);
+            } else if (last && more && nxt.tl[t].count > 0) {  // next item, first tile
+              if (!need_k() || !issue_first_s(nxt, t, ksn)) { ok = false; break; }
             }
           }
+          if (!ok) break;
           tc::commit(&bars[L::V_EMPTY + vs]);
           if (k_next) tc::commit(&bars[L::K_EMPTY + ksn]);
+          ++g;
+          if (!last) {
+            ++j;
+          } else {
+            if (!more) break;
+            cur = nxt;
+            j = 0;
+          }
         }
       }
       // every MMA of this CTA must be complete before TMEM is released
       tc::commit(&bars[L::MMA_DONE]);
       mbar_wait(&bars[L::MMA_DONE], 0, nullptr);
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
     const int t = warp >> 2;                 // query tile slot of this warpgroup
     const int r = (warp & 3) * 32 + lane;    // row within the tile = TMEM lane
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t scol = 128u * t, ocol = 256u + D * t;
     const float sl2 = a.scale_log2;
-    int sw = 0, ow = 0;
+    int sw = 0, ow = 0, k = 0;
     bool ok = true;
-    for (int k = 0, idx; ok && (idx = snake_item(k, cta, grid, a.total)) >= 0; ++k) {
+    for (int idx; ok && (idx = next_item(k)) >= 0;) {
       const Item it = make_item(a, idx);
       const Tile T = t == 0 ? it.tl[0] : it.tl[1];
       if (T.row_tile >= a.ntq) continue;
@@ -503,6 +566,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 
 bool prefill_supported(int d) { return d == 64 || d == 128; }
 
+size_t prefill_workspace_bytes() { return 256; }
+
 void prefill_tile_shape(int d, int* Br, int* Bc) {
   (void)d;
   *Br = pf::kM;
@@ -511,12 +576,13 @@ void prefill_tile_shape(int d, int* Br, int* Bc) {
 
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, float scale,
-                   const int32_t* key_lens, int num_sms, cudaStream_t st) {
+                   const int32_t* key_lens, void* workspace, int num_sms, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (make_tmap_3d_bf16(&tq, q, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tk, k, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tv, v, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
   FwdArgs a;
+  a.sched = static_cast<unsigned int*>(workspace);
   a.o = static_cast<__nv_bfloat16*>(o);
   a.lse = lse;
   a.key_lens = key_lens;
@@ -542,6 +608,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
     if (band < 1) band = 1;
   }
   a.band = band;
+  // the item counter starts every launch at zero (stream-ordered)
+  if (cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) != cudaSuccess) return ATTN_ECUDA;
   if (d == 128) {
     auto kern = prefill_tc_kernel<128>;
     const int smem = pf::Smem<128>::kTotal;

@@ -63,15 +63,16 @@ typedef enum {
 
 /* Exact attention forward.  Dispatch: Nq == 1 runs the split-KV decode kernel
  * followed by the log-sum-exp combine pass; Nq > 1 runs the tiled prefill
- * kernel (TMA + tcgen05/TMEM).
+ * kernel (TMA + tcgen05/TMEM, persistent, one CTA per SM).
  *   d: 64 or 128.  scale: finite and > 0 (usually 1/sqrt(d); "Transformer
  *   Architecture Breakdown ...", section 1.2).  causal: 0 or 1 (ignored in
  *   effect for Nq == 1, where j <= Nk - 1 always holds).
- *   lse may be NULL.  The decode path needs scratch for its partial results:
- *   this entry point uses a workspace owned by the library (allocated on
- *   first use per device, grown on demand, released at process exit); decode
- *   calls that overlap on the GPU share it and must not run concurrently --
- *   use attn_fwd_ws for concurrent streams.
+ *   lse may be NULL.  Both paths need scratch device memory (decode: its
+ *   partial results; prefill: the work-item counter of its scheduler, zeroed
+ *   in-stream before each launch): this entry point uses a workspace owned by
+ *   the library (allocated on first use per device, grown on demand, released
+ *   at process exit); calls that overlap on the GPU share it and must not run
+ *   concurrently -- use attn_fwd_ws for concurrent streams.
  * Errors: ATTN_EINVAL / EUNSUPPORTED / EALIGN before any launch; ATTN_ECUDA
  * if a launch or the workspace allocation fails. */
 ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
@@ -79,16 +80,16 @@ ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, floa
              float scale, const int32_t* key_lens, void* stream);
 
 /* attn_fwd with a caller-owned device workspace of at least
- * attn_workspace_size(...) bytes (256-byte aligned).  The prefill path uses
- * none (workspace may be NULL when Nq > 1).  The workspace must stay
- * untouched until the stream has passed this call. */
+ * attn_workspace_size(...) bytes (256-byte aligned; its contents need no
+ * initialisation).  The workspace must stay untouched until the stream has
+ * passed this call.  Returns ATTN_EWORKSPACE when it is missing or too small. */
 ATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* o,
                 float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
                 int causal, float scale, const int32_t* key_lens,
                 void* workspace, size_t workspace_bytes, void* stream);
 
 /* Bytes of workspace attn_fwd_ws needs for these sizes on the current device
- * (0 for Nq > 1). */
+ * (0 for invalid sizes). */
 ATTN_API size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 
 /* RoPE prologue ("Transformer Architecture Breakdown ...", section 3.1;

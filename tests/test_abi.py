@@ -68,10 +68,19 @@ def test_attn_fwd_rejects_bad_arguments_on_host(L):
 
 
 def test_attn_fwd_ws_rejects_missing_workspace(L):
-    # decode needs a workspace; the size query needs a device, so on a
-    # CPU-only host the call fails before any launch either way
+    # decode needs a workspace (its size query needs a device, so on a
+    # CPU-only host the call fails before any launch either way)
     rc = L.attn_fwd_ws(P, P, P, P, None, 2, 4, 1, 1, 64, 64, 0, 0.125, None, None, 0, None)
     assert rc in (4, 5)
+    # prefill needs 256 bytes for its scheduler counter
+    assert L.attn_workspace_size(1, 2, 2, 8, 8, 64) == 256
+    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0, 0.125, None, None, 0, None)
+    assert rc == 4
+    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0, 0.125, None, P, 128, None)
+    assert rc == 4
+    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0, 0.125, None,
+                       ctypes.c_void_p(0x1010), 256, None)
+    assert rc == 3
 
 
 def test_rope_rejects_bad_arguments_on_host(L):
