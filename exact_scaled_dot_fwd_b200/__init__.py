@@ -13,7 +13,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "rope_apply",
+__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_decode_static", "rope_apply",
            "prefill_tile_shape", "tile_plan", "device_status", "AttnError", "lib",
            "STATUS_NAMES"]
 
@@ -59,6 +59,10 @@ def lib():
         L.attn_strerror.restype = ctypes.c_char_p
         L.attn_abi_version.argtypes = []
         L.attn_abi_version.restype = i
+        L.attn_fwd_decode_static.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, f, vp, vp]
+        L.attn_fwd_decode_static.restype = i
+        L.attn_decode_static_max_bytes.argtypes = []
+        L.attn_decode_static_max_bytes.restype = sz
         _lib = L
     return _lib
 
@@ -158,6 +162,32 @@ def attn_fwd_ws(q, k, v, workspace, causal=False, scale=None, key_lens=None, out
                            int(bool(causal)), float(scale), _ptr(key_lens), _ptr(workspace),
                            ws_bytes, _stream(stream))
     _raise(rc, "attn_fwd_ws")
+    return (out, lse) if return_lse else out
+
+
+def attn_fwd_decode_static(q, k, v, scale=None, key_lens=None, out=None, lse=None,
+                           return_lse=True, stream=None):
+    """Decode (Nq == 1) through the entry point that allocates nothing: its
+    scratch is a fixed device array inside the library (see
+    attn_fwd_decode_static in include/attn.h).  Same result as attn_fwd."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _check_tensor(t, n, torch.bfloat16, 4)
+    B, Hq, Hkv, Nq, Nk, d = _shapes(q, k, v)
+    if Nq != 1:
+        raise ValueError("attn_fwd_decode_static takes one query row per sequence (Nq == 1)")
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if key_lens is not None:
+        _check_tensor(key_lens, "key_lens", torch.int32, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, 1), dtype=torch.float32, device=q.device)
+    rc = lib().attn_fwd_decode_static(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                                      _ptr(lse if return_lse else None), B, Hq, Hkv, Nk, d,
+                                      float(scale), _ptr(key_lens), _stream(stream))
+    _raise(rc, "attn_fwd_decode_static")
     return (out, lse) if return_lse else out
 
 

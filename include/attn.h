@@ -117,6 +117,32 @@ ATTN_API int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal,
                        const int32_t* key_lens, int32_t* first,
                        int32_t* count, void* stream);
 
+/* Decode (Nq == 1) that allocates nothing.  The pages have no counterpart:
+ * this entry point exists for callers that cannot call cudaMalloc -- code
+ * running under a fixed, preallocated memory budget, inside an allocator
+ * hook or another runtime's callback, or on latency-critical paths where
+ * cudaMalloc's implicit device synchronisation is not acceptable.
+ *   Arguments, layouts and result are those of attn_fwd with Nq = 1:
+ *   q/o bf16 [B, Hq, 1, d], k/v bf16 [B, Hkv, Nk, d], lse fp32 [B, Hq, 1] or
+ *   NULL, key_lens device int32 [B] or NULL, d 64 or 128.
+ *   The split-KV partial results live in a device array built into the
+ *   library (attn_decode_static_max_bytes() = 8 MiB), held on every GPU that
+ *   loads the library until the process exits.  Sizes whose partials do not
+ *   fit return ATTN_EWORKSPACE before any launch.
+ *   All calls share that array and it keeps the last call's contents: calls
+ *   that overlap on the GPU (other streams or threads) race and must be
+ *   serialised.  No part of it needs to start at zero.
+ *   The first call on a device looks up the array's device address with
+ *   that device current and caches it; make that first call before any
+ *   stream capture.
+ * Errors: as attn_fwd, plus ATTN_EWORKSPACE for sizes beyond the array. */
+ATTN_API int attn_fwd_decode_static(const void* q, const void* k, const void* v, void* o,
+                                    float* lse, int B, int Hq, int Hkv, int Nk, int d,
+                                    float scale, const int32_t* key_lens, void* stream);
+
+/* Size in bytes of the device array attn_fwd_decode_static works in. */
+ATTN_API size_t attn_decode_static_max_bytes(void);
+
 /* Synchronises `stream`, then returns ATTN_ETIMEOUT if any kernel of this
  * library on the current device gave up on a barrier wait since the last
  * reset, else ATTN_OK (ATTN_ECUDA if the synchronisation failed).  reset != 0
