@@ -17,6 +17,10 @@
 // unit with the two-block merge rule of the online softmax ("Transformer
 // Architecture Breakdown ...", section 4.2), generalised to n blocks.
 //
+// Head dimension 128 runs the tcgen05 split kernel of decode_tc.cu (same
+// work split and partial format); the mma.sync split kernel below serves
+// d = 64.
+//
 // Data movement.  K and V tiles of 64 keys arrive by TMA (2D tensor map over
 // the [B*Hkv*Nk, d] cache, 128-byte swizzle) into a 4-stage shared-memory ring
 // filled by a dedicated producer warp.  Consumer warps own 16 query heads
@@ -98,6 +102,8 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = a.B, Hkv = a.Hkv, U = B * Hkv;
 
+  // the combine pass may launch now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;");
   if (threadIdx.x == 0) {
     for (int s = 0; s < kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -366,7 +372,10 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
   }
 }
 
-// Combine: one CTA per (unit, 16 heads); reads the slots of the unit.
+// Combine: one CTA per (unit, kCombineThreads / D heads), one thread per
+// output element.  The log-sum-exps of the unit's slots are staged in shared
+// memory, per head lse = log2 sum_s 2^lse_s, then every (head, d) output sums
+// its slots' partials weighted by 2^(lse_s - lse) with independent loads.
 struct CombineArgs {
   const int32_t* key_lens;
   const float* part_o;
@@ -376,16 +385,20 @@ struct CombineArgs {
   int B, Hq, Hkv, Nk, G, grid;
 };
 
+constexpr int kCombineThreads = 256;
+
 template <int D>
-__global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
+__global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(CombineArgs a) {
+  extern __shared__ float cs[];          // lse_s [ns][G], then L2 [G]
+  __shared__ long long s_red[2][kCombineThreads / 32];
   __shared__ long long s_pb[2];
   __shared__ int s_len;
-  __shared__ float s_w[64][16];   // per slot weight for each of 16 heads
-  __shared__ float s_lse[16];
   const int u = blockIdx.x, b = u / a.Hkv, h = u - b * a.Hkv;
-  const int g0 = blockIdx.y * 16;
+  const int G = a.G;
+  constexpr int HB = kCombineThreads / D;            // heads of this block
+  const int g0 = blockIdx.y * HB;
+  const int gn = (G - g0) < HB ? (G - g0) : HB;
   // unit start and total key count: block-wide sums over the key lengths
-  __shared__ long long s_red[2][8];
   long long before = 0, total = 0;
   for (int bb = threadIdx.x; bb < a.B; bb += blockDim.x) {
     int len = a.key_lens ? a.key_lens[bb] : a.Nk;
@@ -413,16 +426,15 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
   __syncthreads();
   const long long p0 = s_pb[0], T = s_pb[1];
   const int len = s_len;
-  const int rows = (a.G - g0) < 16 ? (a.G - g0) : 16;
+  __nv_bfloat16* orow = a.o + ((size_t)b * a.Hq + (size_t)h * G + g0) * D;
   if (len == 0) {
-    for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
-      const int r = idx / D, c = idx - r * D;
-      a.o[(((size_t)b * a.Hq) + (size_t)h * a.G + g0 + r) * D + c] = __float2bfloat16(0.f);
-    }
-    if (a.lse && threadIdx.x < rows) a.lse[(size_t)b * a.Hq + h * a.G + g0 + threadIdx.x] = -INFINITY;
+    // o / lse may be read by earlier work in the stream only through the split
+    // kernel's inputs, so writing before the dependency wait is safe
+    for (int idx = threadIdx.x; idx < gn * D; idx += blockDim.x) orow[idx] = __float2bfloat16(0.f);
+    if (a.lse && threadIdx.x < gn) a.lse[(size_t)b * a.Hq + h * G + g0 + threadIdx.x] = -INFINITY;
     return;
   }
-  // CTAs whose ranges intersect [p0, p0 + len)
+  // CTAs whose ranges intersect [p0, p0 + len); empty ranges wrote no slot
   auto cta_of = [&](long long x) -> int {
     long long c = (x * a.grid) / T;
     while (c + 1 < a.grid && T * (c + 1) / a.grid <= x) ++c;
@@ -431,39 +443,52 @@ __global__ void __launch_bounds__(256) decode_combine_kernel(CombineArgs a) {
   };
   const int c0 = cta_of(p0), c1 = cta_of(p0 + len - 1);
   const int ns = c1 - c0 + 1;
-  // CTAs whose global range is empty (T < grid) wrote no slot: weight 0
   auto nonempty = [&](int c) -> bool { return T * c / a.grid < T * (c + 1) / a.grid; };
-  // weights: lse over slots, per head (thread r < rows handles head r)
-  if (threadIdx.x < rows) {
-    const int r = threadIdx.x;
-    float mx = -INFINITY;
-    for (int c = c0; c <= c1; ++c)
-      if (nonempty(c)) mx = fmaxf(mx, a.part_lse[((size_t)c + u) * a.G + g0 + r]);
-    float sum = 0.f;
-    for (int c = c0; c <= c1; ++c)
-      if (nonempty(c)) sum += exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - mx);
-    const float L2 = mx + __log2f(sum);
-    s_lse[r] = L2;
-    for (int c = c0; c <= c1 && c - c0 < 64; ++c)
-      s_w[c - c0][r] =
-          nonempty(c) ? exp2_approx(a.part_lse[((size_t)c + u) * a.G + g0 + r] - L2) : 0.f;
-    if (a.lse) a.lse[(size_t)b * a.Hq + h * a.G + g0 + r] = L2 * kLn2;
+  // launched as a programmatic dependent of the split kernel: everything
+  // above reads only inputs; the partials are ready after this wait
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  float* lse_s = cs;                  // [ns][HB]
+  float* L2 = cs + (size_t)ns * HB;   // [HB]
+  for (int idx = threadIdx.x; idx < ns * gn; idx += blockDim.x) {
+    const int k = idx / gn, g = idx - k * gn;
+    lse_s[k * HB + g] =
+        nonempty(c0 + k) ? a.part_lse[((size_t)(c0 + k) + u) * G + g0 + g] : -INFINITY;
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < rows * D; idx += blockDim.x) {
-    const int r = idx / D, c = idx - r * D;
-    float accv = 0.f;
-    for (int k = 0; k < ns; ++k) {
-      float w;
-      if (k < 64) {
-        w = s_w[k][r];
-      } else {
-        if (!nonempty(c0 + k)) continue;
-        w = exp2_approx(a.part_lse[((size_t)(c0 + k) + u) * a.G + g0 + r] - s_lse[r]);
-      }
-      if (w != 0.f) accv += w * a.part_o[(((size_t)(c0 + k) + u) * a.G + g0 + r) * D + c];
+  if (threadIdx.x < gn) {
+    const int g = threadIdx.x;
+    float mx = -INFINITY;
+    for (int k = 0; k < ns; ++k) mx = fmaxf(mx, lse_s[k * HB + g]);
+    float sum = 0.f;
+    for (int k = 0; k < ns; ++k) sum += exp2_approx(lse_s[k * HB + g] - mx);
+    const float l2 = mx + __log2f(sum);
+    L2[g] = l2;
+    if (a.lse) a.lse[(size_t)b * a.Hq + h * G + g0 + g] = l2 * kLn2;
+  }
+  __syncthreads();
+  for (int idx = threadIdx.x; idx < gn * D; idx += blockDim.x) {
+    const int g = idx / D, c = idx - g * D;
+    const float l2 = L2[g];
+    const float* src = a.part_o + (((size_t)c0 + u) * G + g0 + g) * D + c;
+    const size_t stride = (size_t)G * D;   // next slot
+    float acc = 0.f;
+    int k = 0;
+    for (; k + 4 <= ns; k += 4) {
+      const float w0 = exp2_approx(lse_s[(k + 0) * HB + g] - l2);
+      const float w1 = exp2_approx(lse_s[(k + 1) * HB + g] - l2);
+      const float w2 = exp2_approx(lse_s[(k + 2) * HB + g] - l2);
+      const float w3 = exp2_approx(lse_s[(k + 3) * HB + g] - l2);
+      const float x0 = w0 != 0.f ? src[(k + 0) * stride] : 0.f;
+      const float x1 = w1 != 0.f ? src[(k + 1) * stride] : 0.f;
+      const float x2 = w2 != 0.f ? src[(k + 2) * stride] : 0.f;
+      const float x3 = w3 != 0.f ? src[(k + 3) * stride] : 0.f;
+      acc += (w0 * x0 + w1 * x1) + (w2 * x2 + w3 * x3);
     }
-    a.o[(((size_t)b * a.Hq) + (size_t)h * a.G + g0 + r) * D + c] = __float2bfloat16(accv);
+    for (; k < ns; ++k) {
+      const float w = exp2_approx(lse_s[k * HB + g] - l2);
+      if (w != 0.f) acc += w * src[k * stride];
+    }
+    orow[idx] = __float2bfloat16(acc);
   }
 }
 
@@ -512,16 +537,21 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.part_o_bytes);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = p.G; a.grid = p.grid;
   a.scale_log2 = scale * kLog2e;
-  const int MT = (p.G + 15) / 16;
   int rc;
-  if (d == 128) {
-    rc = MT == 1 ? launch_decode_t<128, 1>(p, tk, tv, a, st)
-       : MT == 2 ? launch_decode_t<128, 2>(p, tk, tv, a, st)
-                 : launch_decode_t<128, 4>(p, tk, tv, a, st);
+  if (decode_tc_supported(B, Hq, Hkv, d)) {
+    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nk, scale, key_lens, a.part_o, a.part_lse,
+                                p.grid, st);
   } else {
-    rc = MT == 1 ? launch_decode_t<64, 1>(p, tk, tv, a, st)
-       : MT == 2 ? launch_decode_t<64, 2>(p, tk, tv, a, st)
-                 : launch_decode_t<64, 4>(p, tk, tv, a, st);
+    const int MT = (p.G + 15) / 16;
+    if (d == 128) {
+      rc = MT == 1 ? launch_decode_t<128, 1>(p, tk, tv, a, st)
+         : MT == 2 ? launch_decode_t<128, 2>(p, tk, tv, a, st)
+                   : launch_decode_t<128, 4>(p, tk, tv, a, st);
+    } else {
+      rc = MT == 1 ? launch_decode_t<64, 1>(p, tk, tv, a, st)
+         : MT == 2 ? launch_decode_t<64, 2>(p, tk, tv, a, st)
+                   : launch_decode_t<64, 4>(p, tk, tv, a, st);
+    }
   }
   if (rc != ATTN_OK) return rc;
   CombineArgs c;
@@ -531,9 +561,28 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   c.o = static_cast<__nv_bfloat16*>(o);
   c.lse = lse;
   c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.Nk = Nk; c.G = p.G; c.grid = p.grid;
-  dim3 cg(B * Hkv, (p.G + 15) / 16);
-  if (d == 128) decode_combine_kernel<128><<<cg, 256, 0, st>>>(c);
-  else decode_combine_kernel<64><<<cg, 256, 0, st>>>(c);
+  // shared memory: the unit's slot lse's ([slots][heads of the block], at most
+  // grid + 1 slots) + [heads of the block]
+  const int hb = kCombineThreads / d;
+  const size_t csmem = ((size_t)(p.grid + 2) * hb) * sizeof(float);
+  const dim3 cgrid(B * Hkv, (p.G + hb - 1) / hb);
+  // programmatic dependent launch: the combine grid may start while the
+  // split kernel drains; it waits for the split's results in the kernel
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = cgrid;
+  cfg.blockDim = dim3(kCombineThreads);
+  cfg.dynamicSmemBytes = csmem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (d == 128) {
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<128>, c) != cudaSuccess) return ATTN_ECUDA;
+  } else {
+    if (cudaLaunchKernelEx(&cfg, decode_combine_kernel<64>, c) != cudaSuccess) return ATTN_ECUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 

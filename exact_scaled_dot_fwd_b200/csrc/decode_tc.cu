@@ -1,0 +1,541 @@
+// decode_tc.cu -- split-KV decode (Nq == 1, d == 128) on the tcgen05 tensor
+// cores.
+//
+// Same work split and partial-result format as the mma.sync decode kernel in
+// decode.cu (balanced global key ranges per CTA, one partial per (CTA, unit)
+// segment, merged by the log-sum-exp combine pass), but the two products run
+// as tcgen05 MMAs with the roles of the operands swapped so that the 128-row
+// MMA dimension is the keys:
+//   S^T [128 keys x N heads]  = K_tile [128 x d] . Q^T      (TMEM, fp32)
+//   O^T [d x N heads]        += V_tile^T [d x 128] . P^T   (TMEM, fp32)
+// N = the unit's query heads rounded up to 16.  One softmax thread owns one
+// key (one TMEM lane of S^T) and, for O^T, one dimension of d.  The per-head
+// maximum over the tile's keys is a butterfly transpose-reduce across the
+// warp plus a four-entry exchange in shared memory; per-head running sums
+// stay per thread until the segment ends.  P^T goes to shared memory (bf16,
+// the B operand of the PV MMA).  S^T is double-buffered in TMEM, so the S MMA
+// of tile j+2 and the loads run while the softmax works on tile j.
+//
+// Warp roles: warps 0-3 softmax (TMEM lane quarters 0-3), warp 4 MMA issuer
+// and TMEM allocator, warp 5 TMA producer.
+#include <cuda_bf16.h>
+
+#include "common.cuh"
+#include "kernels.h"
+#include "tcgen05.cuh"
+
+namespace attn {
+namespace dtc {
+
+constexpr int kTile = 128;   // keys per tile
+constexpr int kD = 128;
+constexpr int kMaxB = 2048;
+constexpr float kRescaleLog2 = 8.0f;
+
+template <int N>
+struct Smem {
+  static constexpr int KS = N <= 32 ? 3 : 2;   // K ring stages
+  static constexpr int VS = 2;                 // V ring stages
+  static constexpr int kKV = kTile * kD * 2;   // one K or V tile (32 KB)
+  static constexpr int kBox = kTile * 128;     // 64-column box of a K/V tile
+  static constexpr int kQBox = N * 128;        // 64-column box of Q (N rows)
+  static constexpr int kPBox = N * 128;        // 64-key box of P^T (N rows)
+  static constexpr int kK = 0;
+  static constexpr int kV = kK + KS * kKV;
+  static constexpr int kQ = kV + VS * kKV;
+  static constexpr int kP = kQ + 2 * kQBox;    // P^T [2 buffers][2 boxes]
+  static constexpr int kScan = kP + 4 * kPBox; // int64 [kMaxB + 1]
+  static constexpr int kLens = kScan + (kMaxB + 1) * 8;
+  static constexpr int kRed = kLens + kMaxB * 4;   // float [4][64]
+  static constexpr int kMs = kRed + 4 * 64 * 4;    // float [64] running max (log2 units)
+  static constexpr int kAs = kMs + 64 * 4;         // float [64] this tile's rescale factor
+  static constexpr int kLs = kAs + 64 * 4;         // float [64] segment row sums
+  static constexpr int kBar = kLs + 64 * 4;
+  enum {
+    K_FULL = 0,
+    K_EMPTY = K_FULL + KS,
+    V_FULL = K_EMPTY + KS,
+    V_EMPTY = V_FULL + VS,
+    Q_FULL = V_EMPTY + VS,
+    Q_EMPTY = Q_FULL + 1,
+    S_FULL = Q_EMPTY + 1,    // [2]
+    P_FULL = S_FULL + 2,     // [2], 128 arrivals
+    PV_DONE = P_FULL + 2,    // [2]
+    MMA_DONE = PV_DONE + 2,
+    NUM_BARS = MMA_DONE + 1
+  };
+  static constexpr int kTmemSlot = kBar + NUM_BARS * 8;
+  static constexpr int kAbort = kTmemSlot + 16;
+  static constexpr int kTotal = kAbort + 16 + 1024;
+  static_assert(kTotal <= 232448, "shared memory over the 227 KB per-CTA limit");
+};
+
+struct Seg {
+  int u, lo, hi;
+};
+
+__device__ __forceinline__ long long unit_prefix(const long long* pb, const int* lens, int u,
+                                                 int Hkv) {
+  const int b = u / Hkv, h = u - b * Hkv;
+  return (long long)Hkv * pb[b] + (long long)h * lens[b];
+}
+
+// One butterfly step across lanes `OFF` apart: each lane keeps the half of
+// its HALF*2 values selected by its lane bit and combines it with the
+// partner's other half.
+template <int HALF, int OFF, bool SUM, int NV>
+__device__ __forceinline__ void bfly_step(float (&v)[NV], int lane) {
+  const bool up = (lane & OFF) != 0;
+#pragma unroll
+  for (int i = 0; i < HALF; ++i) {
+    const float send = up ? v[i] : v[i + HALF];
+    const float keep = up ? v[i + HALF] : v[i];
+    const float got = __shfl_xor_sync(0xffffffffu, send, OFF);
+    v[i] = SUM ? keep + got : fmaxf(keep, got);
+  }
+}
+
+// Reduce N per-lane values (one per head) over the 32 lanes of the warp.
+// Afterwards v[0 .. R) hold the results for heads lane*R + i (N >= 32,
+// R = N / 32) or head lane & 15 (N == 16, R = 1).
+template <int N, bool SUM>
+__device__ __forceinline__ void bfly_reduce(float (&v)[N], int lane) {
+  if constexpr (N == 64) {
+    bfly_step<32, 16, SUM>(v, lane);
+    bfly_step<16, 8, SUM>(v, lane);
+    bfly_step<8, 4, SUM>(v, lane);
+    bfly_step<4, 2, SUM>(v, lane);
+    bfly_step<2, 1, SUM>(v, lane);
+  } else if constexpr (N == 32) {
+    bfly_step<16, 16, SUM>(v, lane);
+    bfly_step<8, 8, SUM>(v, lane);
+    bfly_step<4, 4, SUM>(v, lane);
+    bfly_step<2, 2, SUM>(v, lane);
+    bfly_step<1, 1, SUM>(v, lane);
+  } else {
+    bfly_step<8, 8, SUM>(v, lane);
+    bfly_step<4, 4, SUM>(v, lane);
+    bfly_step<2, 2, SUM>(v, lane);
+    bfly_step<1, 1, SUM>(v, lane);
+    const float o = __shfl_xor_sync(0xffffffffu, v[0], 16);
+    v[0] = SUM ? v[0] + o : fmaxf(v[0], o);
+  }
+}
+
+// Store this warp's reduced values into red[warp][head].
+template <int N>
+__device__ __forceinline__ void put_red(float* red, int warp, int lane, const float (&v)[N]) {
+  if constexpr (N >= 32) {
+    constexpr int R = N / 32;
+#pragma unroll
+    for (int i = 0; i < R; ++i) red[warp * 64 + lane * R + i] = v[i];
+  } else {
+    if (lane < 16) red[warp * 64 + lane] = v[0];
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_ld_row(uint32_t taddr, float (&v)[N]) {
+  if constexpr (N == 16) {
+    tc::ld16f(taddr, v);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N / 32; ++c) tc::ld32f(taddr + 32 * c, v + 32 * c);
+  }
+}
+
+template <int N>
+__device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&v)[N]) {
+  if constexpr (N == 16) {
+    tc::st16f(taddr, v);
+  } else {
+#pragma unroll
+    for (int c = 0; c < N / 32; ++c) tc::st32f(taddr + 32 * c, v + 32 * c);
+  }
+}
+
+__device__ __forceinline__ bool bar_or(int id, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, 128, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id)
+      : "memory");
+  return r != 0;
+}
+
+}  // namespace dtc
+
+struct DecodeTcArgs {
+  const int32_t* key_lens;
+  float* part_o;
+  float* part_lse;
+  int B, Hq, Hkv, Nk, G, grid;
+  float scale_log2;
+};
+
+template <int N>
+__global__ void __launch_bounds__(192, 1)
+    decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
+                     const __grid_constant__ CUtensorMap tmap_k,
+                     const __grid_constant__ CUtensorMap tmap_v, DecodeTcArgs a) {
+  using namespace dtc;
+  using L = Smem<N>;
+  constexpr int KS = L::KS, VS = L::VS;
+  constexpr uint32_t kIdescS = tc::idesc_bf16(kTile, N, false, false);
+  constexpr uint32_t kIdescPV = tc::idesc_bf16(kD, N, true, false);
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
+  long long* pb = reinterpret_cast<long long*>(smem + L::kScan);
+  int* lens_s = reinterpret_cast<int*>(smem + L::kLens);
+  float* red = reinterpret_cast<float*>(smem + L::kRed);
+  float* m_s = reinterpret_cast<float*>(smem + L::kMs);
+  float* a_s = reinterpret_cast<float*>(smem + L::kAs);
+  float* l_s = reinterpret_cast<float*>(smem + L::kLs);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+
+  // the combine pass may launch now; it waits for this grid's results
+  asm volatile("griddepcontrol.launch_dependents;");
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int B = a.B, Hkv = a.Hkv, U = B * Hkv;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < L::NUM_BARS; ++i)
+      mbar_init(&bars[i], (i == L::P_FULL || i == L::P_FULL + 1) ? 128u : 1u);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 4) {
+    tc::alloc(tmem_slot, 256);
+    tc::relinquish();
+  }
+  // key lengths (clamped) and their exclusive prefix over b, by warp 5
+  if (warp == 5) {
+    long long carry = 0;
+    for (int base = 0; base < B; base += 32) {
+      const int b = base + lane;
+      int len = 0;
+      if (b < B) {
+        len = a.key_lens ? a.key_lens[b] : a.Nk;
+        len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+        lens_s[b] = len;
+      }
+      long long x = len;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const long long y = __shfl_up_sync(0xffffffffu, x, o);
+        if (lane >= o) x += y;
+      }
+      if (b < B) pb[b] = carry + x - len;
+      carry += __shfl_sync(0xffffffffu, x, 31);
+    }
+    if (lane == 0) pb[B] = carry;
+  }
+  tc::fence_before();
+  __syncthreads();
+  tc::fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const long long T = (long long)Hkv * pb[B];
+  const long long start = T * blockIdx.x / a.grid;
+  const long long end = T * (blockIdx.x + 1) / a.grid;
+  int u0 = 0;
+  if (start < end) {
+    int lo = 0, hi = U - 1;
+    while (lo < hi) {
+      const int mid = (lo + hi + 1) >> 1;
+      if (unit_prefix(pb, lens_s, mid, Hkv) <= start) lo = mid; else hi = mid - 1;
+    }
+    u0 = lo;
+  }
+  auto next_seg = [&](int& u, Seg& s) -> bool {
+    while (u < U) {
+      const long long p0 = unit_prefix(pb, lens_s, u, Hkv);
+      if (p0 >= end) return false;
+      const long long p1 = p0 + lens_s[u / Hkv];
+      const long long lo = start > p0 ? start : p0, hi = end < p1 ? end : p1;
+      const int cur = u++;
+      if (hi > lo) {
+        s.u = cur; s.lo = (int)(lo - p0); s.hi = (int)(hi - p0);
+        return true;
+      }
+    }
+    return false;
+  };
+
+  if (warp == 5) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0 && start < end) {
+      tma_prefetch_desc(&tmap_q);
+      tma_prefetch_desc(&tmap_k);
+      tma_prefetch_desc(&tmap_v);
+      int u = u0, g = 0, qn = 0;
+      Seg s;
+      bool ok = true;
+      while (ok && next_seg(u, s)) {
+        const int b = s.u / Hkv, h = s.u - b * Hkv;
+        const int n = (s.hi - s.lo + kTile - 1) / kTile;
+        if (qn > 0 && !mbar_wait(&bars[L::Q_EMPTY], (qn - 1) & 1, abort_flag)) break;
+        ++qn;
+        mbar_arrive_expect_tx(&bars[L::Q_FULL], 2 * L::kQBox);
+        for (int bx = 0; bx < 2; ++bx)
+          tma_load_2d(smem + L::kQ + bx * L::kQBox, &tmap_q, bx * 64, b * a.Hq + h * a.G,
+                      &bars[L::Q_FULL]);
+        const int row0 = s.u * a.Nk + s.lo;
+        for (int j = 0; j < n; ++j, ++g) {
+          const int ks = g % KS, vs = g % VS;
+          if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / KS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kKV);
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_2d(smem + L::kK + ks * L::kKV + bx * L::kBox, &tmap_k, bx * 64,
+                        row0 + j * kTile, &bars[L::K_FULL + ks]);
+          if (!mbar_wait(&bars[L::V_EMPTY + vs], ((g / VS) & 1) ^ 1, abort_flag)) { ok = false; break; }
+          mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kKV);
+          for (int bx = 0; bx < 2; ++bx)
+            tma_load_2d(smem + L::kV + vs * L::kKV + bx * L::kBox, &tmap_v, bx * 64,
+                        row0 + j * kTile, &bars[L::V_FULL + vs]);
+        }
+      }
+    }
+  } else if (warp == 4) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0 && start < end) {
+      const uint32_t k_base = smem_u32(smem + L::kK), v_base = smem_u32(smem + L::kV);
+      const uint32_t q_base = smem_u32(smem + L::kQ), p_base = smem_u32(smem + L::kP);
+      auto issue_s = [&](int g) {
+        const uint32_t kb = k_base + (g % KS) * L::kKV;
+#pragma unroll
+        for (int kk = 0; kk < kD / 16; ++kk) {
+          tc::mma_ss(tmem + (uint32_t)((g & 1) * N),
+                     tc::smem_desc_sw128(kb + (kk >> 2) * L::kBox + (kk & 3) * 32, 16, 1024),
+                     tc::smem_desc_sw128(q_base + (kk >> 2) * L::kQBox + (kk & 3) * 32, 16, 1024),
+                     kIdescS, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto issue_pv = [&](int g, bool acc) {
+        const uint32_t vb = v_base + (g % VS) * L::kKV;
+        const uint32_t pbuf = p_base + (g & 1) * 2 * L::kPBox;
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk) {
+          tc::mma_ss(tmem + 2u * N, tc::smem_desc_sw128(vb + kk * 16 * 128, L::kBox, 1024),
+                     tc::smem_desc_sw128(pbuf + (kk >> 2) * L::kPBox + (kk & 3) * 32, 16, 1024),
+                     kIdescPV, (acc || kk > 0) ? 1u : 0u);
+        }
+      };
+      int u = u0, g = 0, qf = 0;
+      Seg s;
+      bool ok = true;
+      while (ok && next_seg(u, s)) {
+        const int n = (s.hi - s.lo + kTile - 1) / kTile;
+        if (!mbar_wait(&bars[L::Q_FULL], qf & 1, abort_flag)) break;
+        ++qf;
+        for (int t = 0; t < 2 && t < n && ok; ++t) {
+          const int gt = g + t;
+          if (!mbar_wait(&bars[L::K_FULL + gt % KS], (gt / KS) & 1, abort_flag)) { ok = false; break; }
+          tc::fence_after();
+          issue_s(gt);
+          tc::commit(&bars[L::S_FULL + (gt & 1)]);
+          tc::commit(&bars[L::K_EMPTY + gt % KS]);
+        }
+        if (ok && n <= 2) tc::commit(&bars[L::Q_EMPTY]);
+        for (int j = 0; ok && j < n; ++j, ++g) {
+          if (!mbar_wait(&bars[L::P_FULL + (g & 1)], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait(&bars[L::V_FULL + g % VS], (g / VS) & 1, abort_flag)) { ok = false; break; }
+          tc::fence_after();
+          issue_pv(g, j > 0);
+          tc::commit(&bars[L::PV_DONE + (g & 1)]);
+          tc::commit(&bars[L::V_EMPTY + g % VS]);
+          if (j + 2 < n) {
+            const int g2 = g + 2;
+            if (!mbar_wait(&bars[L::K_FULL + g2 % KS], (g2 / KS) & 1, abort_flag)) { ok = false; break; }
+            tc::fence_after();
+            issue_s(g2);
+            tc::commit(&bars[L::S_FULL + (g2 & 1)]);
+            tc::commit(&bars[L::K_EMPTY + g2 % KS]);
+            if (j + 2 == n - 1) tc::commit(&bars[L::Q_EMPTY]);
+          }
+        }
+      }
+      tc::commit(&bars[L::MMA_DONE]);
+      mbar_wait(&bars[L::MMA_DONE], 0, nullptr);
+    }
+  } else {
+    // ------------------------------------------------------------ softmax
+    const int Lr = warp * 32 + lane;                 // key row of S^T, dimension of O^T
+    const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
+    const float sl2 = a.scale_log2;
+    uint8_t* p_smem = smem + L::kP;
+    int u = u0, g = 0;
+    Seg s;
+    bool ok = start < end;
+    while (ok && next_seg(u, s)) {
+      const int n = (s.hi - s.lo + kTile - 1) / kTile;
+      asm volatile("bar.sync 1, 128;" ::: "memory");   // previous segment done with m_s / l_s
+      if (Lr < 64) m_s[Lr] = -INFINITY;
+      float lp[N];
+#pragma unroll
+      for (int h = 0; h < N; ++h) lp[h] = 0.f;
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      for (int j = 0; j < n; ++j, ++g) {
+        const int buf = g & 1;
+        if (!mbar_wait(&bars[L::S_FULL + buf], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+        tc::fence_after();
+        float sv[N];
+        tmem_ld_row<N>(tmem + lane_off + (uint32_t)(buf * N), sv);
+        tc::wait_ld();
+        const bool valid = s.lo + j * kTile + Lr < s.hi;
+        if (!valid) {
+#pragma unroll
+          for (int h = 0; h < N; ++h) sv[h] = -INFINITY;
+        }
+        // per-head max over the tile's keys
+        {
+          float v[N];
+#pragma unroll
+          for (int h = 0; h < N; ++h) v[h] = sv[h];
+          bfly_reduce<N, false>(v, lane);
+          put_red<N>(red, warp, lane, v);
+        }
+        if (*abort_flag) { ok = false; break; }
+        asm volatile("bar.sync 1, 128;" ::: "memory");
+        bool need = false;
+        if (Lr < N) {
+          const float mt = fmaxf(fmaxf(red[Lr], red[64 + Lr]), fmaxf(red[128 + Lr], red[192 + Lr])) * sl2;
+          const float mo = m_s[Lr];
+          need = mt > mo + kRescaleLog2;
+          const float mn = need ? fmaxf(mo, mt) : mo;
+          a_s[Lr] = (need && mo != -INFINITY) ? exp2_approx(mo - mn) : 1.f;
+          m_s[Lr] = mn;
+        }
+        const bool any = bar_or(1, need);
+        float mu[N];
+#pragma unroll
+        for (int h = 0; h < N; ++h) {
+          const float m = m_s[h];
+          mu[h] = m == -INFINITY ? 0.f : m;
+        }
+        if (any) {
+          float al[N];
+#pragma unroll
+          for (int h = 0; h < N; ++h) {
+            al[h] = a_s[h];
+            lp[h] *= al[h];
+          }
+          if (j > 0) {   // O^T holds tiles < j: wait for PV of tile j-1, then rescale
+            if (!mbar_wait(&bars[L::PV_DONE + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag)) {
+              ok = false;
+              break;
+            }
+            tc::fence_after();
+            float o[N];
+            tmem_ld_row<N>(tmem + lane_off + 2u * N, o);
+            tc::wait_ld();
+#pragma unroll
+            for (int h = 0; h < N; ++h) o[h] *= al[h];
+            tmem_st_row<N>(tmem + lane_off + 2u * N, o);
+            tc::wait_st();
+          }
+        }
+        // P^T buffer `buf` was read by PV of tile g-2
+        if (g >= 2 &&
+            !mbar_wait(&bars[L::PV_DONE + buf], ((g - 2) >> 1) & 1, abort_flag)) {
+          ok = false;
+          break;
+        }
+        uint8_t* pb_ = p_smem + buf * 2 * L::kPBox + (Lr >> 6) * L::kPBox;
+        const int kc = (Lr & 63) >> 3, kb = (Lr & 7) * 2;
+#pragma unroll
+        for (int h = 0; h < N; ++h) {
+          const float p = exp2_approx(fmaf(sv[h], sl2, -mu[h]));
+          lp[h] += p;
+          const uint32_t off = (uint32_t)h * 128u + (uint32_t)((kc ^ (h & 7)) << 4) + kb;
+          *reinterpret_cast<__nv_bfloat16*>(pb_ + off) = __float2bfloat16_rn(p);
+        }
+        fence_proxy_async_smem();
+        tc::fence_before();
+        mbar_arrive(&bars[L::P_FULL + buf]);
+      }
+      if (!ok) break;
+
+      // ---- segment end: per-head sums, O^T / l, partial results
+      const int glast = g - 1;
+      if (!mbar_wait(&bars[L::PV_DONE + (glast & 1)], (glast >> 1) & 1, abort_flag)) { ok = false; break; }
+      tc::fence_after();
+      float o[N];
+      tmem_ld_row<N>(tmem + lane_off + 2u * N, o);
+      tc::wait_ld();
+      bfly_reduce<N, true>(lp, lane);
+      put_red<N>(red, warp, lane, lp);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (Lr < N) l_s[Lr] = (red[Lr] + red[64 + Lr]) + (red[128 + Lr] + red[192 + Lr]);
+      asm volatile("bar.sync 1, 128;" ::: "memory");
+      const size_t slot = (size_t)blockIdx.x + s.u;
+#pragma unroll
+      for (int h = 0; h < N; ++h) {
+        if (h < a.G) {
+          const float l = l_s[h];
+          a.part_o[(slot * a.G + h) * kD + Lr] = l > 0.f ? o[h] / l : 0.f;
+        }
+      }
+      if (Lr < a.G && Lr < N) {
+        const float l = l_s[Lr];
+        a.part_lse[slot * a.G + Lr] = l > 0.f ? m_s[Lr] + __log2f(l) : -INFINITY;
+      }
+      tc::fence_before();
+    }
+  }
+
+  tc::fence_before();
+  __syncthreads();
+  if (warp == 4) {
+    tc::fence_after();
+    tc::dealloc(tmem, 256);
+  }
+}
+
+namespace {
+template <int N>
+int launch_tc_t(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                const DecodeTcArgs& a, cudaStream_t st) {
+  auto kern = decode_tc_kernel<N>;
+  const int smem = dtc::Smem<N>::kTotal;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ECUDA;
+  kern<<<grid, 192, smem, st>>>(tq, tk, tv, a);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+}  // namespace
+
+bool decode_tc_supported(int B, int Hq, int Hkv, int d) {
+  return d == 128 && Hq / Hkv <= 64 && B <= dtc::kMaxB;
+}
+
+int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                           int Nk, float scale, const int32_t* key_lens, float* part_o,
+                           float* part_lse, int grid, cudaStream_t st) {
+  const int G = Hq / Hkv;
+  const int N = G <= 16 ? 16 : (G <= 32 ? 32 : 64);
+  CUtensorMap tq, tk, tv;
+  const uint64_t rows = (uint64_t)B * Hkv * Nk;
+  if (make_tmap_2d_bf16(&tq, q, dtc::kD, (uint64_t)B * Hq, 64, (uint32_t)N) != ATTN_OK)
+    return ATTN_ECUDA;
+  if (make_tmap_2d_bf16(&tk, k, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
+  if (make_tmap_2d_bf16(&tv, v, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
+  DecodeTcArgs a;
+  a.key_lens = key_lens;
+  a.part_o = part_o;
+  a.part_lse = part_lse;
+  a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = G; a.grid = grid;
+  a.scale_log2 = scale * kLog2e;
+  if (N == 16) return launch_tc_t<16>(grid, tq, tk, tv, a, st);
+  if (N == 32) return launch_tc_t<32>(grid, tq, tk, tv, a, st);
+  return launch_tc_t<64>(grid, tq, tk, tv, a, st);
+}
+
+}  // namespace attn

@@ -31,6 +31,12 @@ struct DecodePlan {
 };
 DecodePlan decode_plan(int B, int Hq, int Hkv, int d, int num_sms);
 bool decode_supported(int B, int Hq, int Hkv, int d);
+// tcgen05 split kernel (d == 128, up to 64 query heads per kv head); writes
+// the same partial-result format as the mma.sync split kernel.
+bool decode_tc_supported(int B, int Hq, int Hkv, int d);
+int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
+                           int Nk, float scale, const int32_t* key_lens, float* part_o,
+                           float* part_lse, int grid, cudaStream_t st);
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                   int Hkv, int Nk, int d, float scale, const int32_t* key_lens, void* workspace,
                   const DecodePlan& p, cudaStream_t st);
