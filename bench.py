@@ -40,13 +40,41 @@ METRIC = "attention fwd TFLOPS (bf16, causal) and decode GB/s; % of B200 rooflin
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
 L2_BYTES = 126 * 1024 * 1024
 
-# DRAM traffic per launch of the dominant kernels, from one ncu capture each
-# (dram__bytes_read.sum + dram__bytes_write.sum), keyed by workload; None when
-# the kernel changed after the capture.
-NCU_TRAFFIC_BYTES = {
-    "mha_prefill": None,
-    "mqa_decode": None,
+# DRAM traffic per launch of the dominant kernel, from one ncu capture each
+# (dram__bytes_read.sum + dram__bytes_write.sum; summaries in profiles/),
+# with a hash of the kernel's source files at capture time.  The figure is
+# reported only while the sources still hash the same.
+KERNEL_SOURCES = {
+    "prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
+    "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh"],
 }
+NCU_TRAFFIC = {
+    # workload: (kernel, source hash, bytes per launch)
+    "mha_prefill": ("prefill", "9389efd25a7c3dc7", 128126976 + 10136832),
+    "mqa_decode": ("decode", "33944cc49cb39b44", 324087552 + 6830592),
+}
+
+
+def source_hash(kernel):
+    import hashlib
+    m = hashlib.sha256()
+    for f in KERNEL_SOURCES[kernel]:
+        with open(os.path.join(ROOT, "exact_scaled_dot_fwd_b200", "csrc", f), "rb") as fh:
+            m.update(fh.read())
+    return m.hexdigest()[:16]
+
+
+def ncu_traffic(workload):
+    """Measured DRAM bytes per launch, or None when not captured for this
+    workload or when the kernel changed since the capture."""
+    entry = NCU_TRAFFIC.get(workload)
+    if entry is None:
+        return None
+    kernel, digest, nbytes = entry
+    try:
+        return nbytes if source_hash(kernel) == digest else None
+    except OSError:
+        return None
 
 
 def parse_args():
@@ -203,12 +231,19 @@ def time_steps(fn, steps, torch, dist, stream):
     torch.cuda.synchronize()
     if dist is not None:
         dist.barrier()
-    ms = e0.elapsed_time(e1)
-    if dist is not None:
-        t = torch.tensor([ms], dtype=torch.float64, device="cuda")
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
-    return ms
+    return reduce_max(e0.elapsed_time(e1), dist)
+
+
+def reduce_max(value, dist):
+    """Maximum of `value` over all ranks (identity without a process group).
+    The tensor lives where the backend wants it: CUDA for NCCL, CPU for gloo."""
+    if dist is None:
+        return value
+    import torch
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(value)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
 
 
 def run_ours(args):
@@ -279,8 +314,10 @@ def run_ours(args):
     ms = time_steps(step, steps, torch, dist, stream)
     clocks = sampler.stop()
     ms_step = ms / steps
-    # decode: split + combine; prefill: the scheduler-counter memset + kernel
-    launches_per_step = 2 + (2 if w.rope else 0)
+    # this library's kernels per step: decode = split + combine; prefill = the
+    # attention kernel (its counter reset is a runtime memset, not a kernel
+    # of ours); plus the two RoPE launches when the workload has RoPE
+    launches_per_step = (2 if w.Nq == 1 else 1) + (2 if w.rope else 0)
     # the dominant kernel alone (differs from the step only when RoPE runs)
     ms_kernel = ms if not w.rope else time_steps(attn_only, steps, torch, dist, stream)
     if w.Nq == 1:
@@ -289,14 +326,14 @@ def run_ours(args):
         kval = work * steps / (ms_kernel / 1e3) / 1e9
         roof = {"bound": "hbm", "achieved": kval, "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": kval / peaks["hbm_gbs"],
-                "traffic": NCU_TRAFFIC_BYTES.get(w.name), "peak_source": peak_src}
+                "traffic": ncu_traffic(w.name), "peak_source": peak_src}
     else:
         unit, work = "TFLOP/s", w.flops()
         value = world * work * steps / (ms / 1e3) / 1e12
         kval = work * steps / (ms_kernel / 1e3) / 1e12
         roof = {"bound": "tensor", "achieved": kval, "peak": peaks["bf16_tflops"],
                 "unit": "TFLOP/s", "frac": kval / peaks["bf16_tflops"],
-                "traffic": NCU_TRAFFIC_BYTES.get(w.name), "peak_source": peak_src}
+                "traffic": ncu_traffic(w.name), "peak_source": peak_src}
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -393,7 +430,7 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None):
             "l2": f"{copies} rotating KV caches ({copies * per_copy / 1e6:.0f} MB allocated)",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"],
-                         "traffic": NCU_TRAFFIC_BYTES.get(w.name), "peak_source": peak_src},
+                         "traffic": ncu_traffic(w.name), "peak_source": peak_src},
             "gpu_launches": 2 * n}
 
 

@@ -63,6 +63,8 @@ def lib():
         L.attn_fwd_decode_static.restype = i
         L.attn_decode_static_max_bytes.argtypes = []
         L.attn_decode_static_max_bytes.restype = sz
+        L.attn_debug_timeout_probe.argtypes = [ctypes.c_ulonglong, vp]
+        L.attn_debug_timeout_probe.restype = i
         _lib = L
     return _lib
 

@@ -107,6 +107,18 @@ int make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ECUDA;
 }
 
+// Failure-detection hook: one thread waits on an mbarrier that nothing ever
+// arrives on, with a short limit; the wait gives up, records ATTN_ETIMEOUT and
+// the kernel returns.  No fault, no hang.
+__global__ void timeout_probe_kernel(unsigned long long limit_ns) {
+  __shared__ uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_mbar_init();
+    mbar_wait_for(&bar, 0, nullptr, limit_ns);
+  }
+}
+
 }  // namespace attn
 
 using namespace attn;
@@ -229,6 +241,12 @@ int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal, const int32_t* 
   if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
   return launch_tile_plan(B, Nq, Nk, d, causal, key_lens, first, count,
                           static_cast<cudaStream_t>(stream));
+}
+
+int attn_debug_timeout_probe(unsigned long long limit_ns, void* stream) {
+  if (limit_ns == 0 || limit_ns > 1000000000ull) return ATTN_EINVAL;
+  timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
 int attn_device_status(void* stream, int reset) {

@@ -302,6 +302,12 @@ __global__ void __launch_bounds__(192, 1)
                         row0 + j * kTile, &bars[L::V_FULL + vs]);
         }
       }
+      // every issued load must land before the CTA may exit
+      for (int j = g - KS > 0 ? g - KS : 0; j < g; ++j)
+        mbar_wait(&bars[L::K_FULL + j % KS], (j / KS) & 1, nullptr);
+      for (int j = g - VS > 0 ? g - VS : 0; j < g; ++j)
+        mbar_wait(&bars[L::V_FULL + j % VS], (j / VS) & 1, nullptr);
+      if (qn > 0) mbar_wait(&bars[L::Q_FULL], (qn - 1) & 1, nullptr);
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer

@@ -275,6 +275,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
         idx = nxt;
       }
+      // every issued load must land before the CTA may exit (normally they
+      // have all been consumed already, and these waits return at once)
+      for (int j = g - kKS > 0 ? g - kKS : 0; j < g; ++j)
+        mbar_wait(&bars[L::K_FULL + j % kKS], (j / kKS) & 1, nullptr);
+      for (int j = g - kVS > 0 ? g - kVS : 0; j < g; ++j)
+        mbar_wait(&bars[L::V_FULL + j % kVS], (j / kVS) & 1, nullptr);
     }
   } else if (warp == 10) {
     // ------------------------------------------------------------ Q producer
@@ -298,6 +304,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
                         it.tl[t].row_tile * kM, it.b * a.Hq + it.tl[t].head, &bars[L::Q_FULL + t]);
         }
       }
+      for (int t = 0; t < 2; ++t)   // the last Q load of each slot must land before exit
+        if (qn[t] > 0) mbar_wait(&bars[L::Q_FULL + t], (qn[t] - 1) & 1, nullptr);
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer

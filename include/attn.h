@@ -149,6 +149,14 @@ ATTN_API size_t attn_decode_static_max_bytes(void);
  * clears the device status word. */
 ATTN_API int attn_device_status(void* stream, int reset);
 
+/* Failure-detection test hook: launches one tiny kernel whose single thread
+ * waits on a barrier that nothing ever completes, giving up after limit_ns
+ * (1 ns .. 1 s).  The wait's limit expires, the kernel records ATTN_ETIMEOUT
+ * in the device status word (read it with attn_device_status) and returns;
+ * nothing faults or hangs and the context stays usable.  Every barrier wait in
+ * the attention kernels takes the same path, with a 2 s limit. */
+ATTN_API int attn_debug_timeout_probe(unsigned long long limit_ns, void* stream);
+
 /* Human-readable name of a status code (static string). */
 ATTN_API const char* attn_strerror(int status);
 

@@ -105,6 +105,11 @@ def test_tile_shape_and_plan_args(L):
     assert L.attn_fwd_tile_plan(1, 8, 8, 64, 3, None, P, P, None) == 1
 
 
+def test_timeout_probe_rejects_bad_limits_on_host(L):
+    assert L.attn_debug_timeout_probe(ctypes.c_ulonglong(0), None) == 1
+    assert L.attn_debug_timeout_probe(ctypes.c_ulonglong(2_000_000_000), None) == 1
+
+
 def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(eb, "LIB_PATH", str(tmp_path / "missing.so"))
     monkeypatch.setattr(eb, "_lib", None)
