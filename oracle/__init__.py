@@ -34,14 +34,18 @@ def lib():
         L.oracle_rope.restype = None
         L.oracle_visible_prefix.argtypes = [i64, i64, i64, i32, i64]
         L.oracle_visible_prefix.restype = i64
-        L.oracle_attn_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, f64,
+        L.oracle_attn_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, i64, f64,
                                        vp, i32, f64, i32, i32, i64, i64, vp, i64, vp, vp, i32]
         L.oracle_attn_rows.restype = i32
         L.oracle_attn_online_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32,
-                                              f64, vp, i64, vp, i64, vp, vp, i32]
+                                              i64, f64, vp, i64, vp, i64, vp, vp, i32]
         L.oracle_attn_online_rows.restype = i32
         L.oracle_kv_tiles.argtypes = [i64, i64, i32, i64, i64, i64, i64, vp, vp, vp]
         L.oracle_kv_tiles.restype = None
+        L.oracle_kv_tiles_window.argtypes = [i64, i64, i32, i64, i64, i64, i64, i64, vp, vp, vp]
+        L.oracle_kv_tiles_window.restype = None
+        L.oracle_visible_range.argtypes = [i64, i64, i64, i32, i64, i64, vp, vp]
+        L.oracle_visible_range.restype = None
         _lib = L
     return _lib
 
@@ -82,11 +86,18 @@ def visible_prefix(i, Nq, Nk, causal, key_len) -> int:
     return int(lib().oracle_visible_prefix(i, Nq, Nk, int(bool(causal)), key_len))
 
 
-def kv_tiles(Nq, Nk, causal, key_len, Br, Bc, qt):
+def kv_tiles(Nq, Nk, causal, key_len, Br, Bc, qt, window=0):
     f, l, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
-    lib().oracle_kv_tiles(Nq, Nk, int(bool(causal)), key_len, Br, Bc, qt,
-                          ctypes.byref(f), ctypes.byref(l), ctypes.byref(c))
+    lib().oracle_kv_tiles_window(Nq, Nk, int(bool(causal)), key_len, window, Br, Bc, qt,
+                                 ctypes.byref(f), ctypes.byref(l), ctypes.byref(c))
     return f.value, l.value, c.value
+
+
+def visible_range(i, Nq, Nk, causal, key_len, window=0):
+    lo, hi = ctypes.c_int64(), ctypes.c_int64()
+    lib().oracle_visible_range(i, Nq, Nk, int(bool(causal)), key_len, window,
+                               ctypes.byref(lo), ctypes.byref(hi))
+    return lo.value, hi.value
 
 
 def _prep(q, k, v, key_lens, rows):
@@ -102,7 +113,7 @@ def _prep(q, k, v, key_lens, rows):
 
 
 def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
-              nthreads=None):
+              nthreads=None, window=0):
     """Naive fp64 attention for the listed flat rows (all rows if None).
 
     q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] as bf16 bit patterns.  rope_cfg: None or
@@ -115,8 +126,8 @@ def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
     lse = np.empty(nrows, np.float64)
     rc = rope_cfg or {}
     st = lib().oracle_attn_rows(
-        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale),
-        _ptr(kl), int(rope_cfg is not None), float(rc.get("base", 10000.0)),
+        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), int(window),
+        float(scale), _ptr(kl), int(rope_cfg is not None), float(rc.get("base", 10000.0)),
         int(rc.get("pairing", 0)), int(bool(rc.get("round_bf16", False))),
         int(rc.get("q_pos_offset", 0)), int(rc.get("k_pos_offset", 0)),
         _ptr(r), nrows, _ptr(o), _ptr(lse), int(nthreads or default_threads()))
@@ -125,14 +136,15 @@ def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
     return o, lse
 
 
-def attn_online_rows(q, k, v, causal, scale, block, key_lens=None, rows=None, nthreads=None):
+def attn_online_rows(q, k, v, causal, scale, block, key_lens=None, rows=None, nthreads=None,
+                     window=0):
     """Online-recurrence fp64 attention over key blocks of size `block`."""
     q, k, v, kl, r, (B, Hq, Hkv, Nq, Nk, d), nrows = _prep(q, k, v, key_lens, rows)
     o = np.empty((nrows, d), np.float64)
     lse = np.empty(nrows, np.float64)
     st = lib().oracle_attn_online_rows(
-        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), float(scale),
-        _ptr(kl), int(block), _ptr(r), nrows, _ptr(o), _ptr(lse),
+        _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), int(window),
+        float(scale), _ptr(kl), int(block), _ptr(r), nrows, _ptr(o), _ptr(lse),
         int(nthreads or default_threads()))
     if st != 0:
         raise ValueError("oracle_attn_online_rows rejected its arguments")

@@ -95,9 +95,34 @@ int64_t oracle_visible_prefix(int64_t i, int64_t Nq, int64_t Nk, int causal,
   return L < 0 ? 0 : L;
 }
 
+/* [AME] 11: with a window w > 0, key j is legal only if |p - j| < w, where
+ * p = i + (Nk - Nq) is the query's key position (the causal alignment). */
+void oracle_visible_range(int64_t i, int64_t Nq, int64_t Nk, int causal,
+                          int64_t key_len, int64_t window, int64_t* lo,
+                          int64_t* hi) {
+  int64_t h = oracle_visible_prefix(i, Nq, Nk, causal, key_len);
+  int64_t l = 0;
+  if (window > 0) {
+    const int64_t p = i + (Nk - Nq);
+    if (p - window + 1 > l) l = p - window + 1;
+    if (p + window < h) h = p + window;
+  }
+  if (h < l) h = l;
+  *lo = l;
+  *hi = h;
+}
+
 void oracle_kv_tiles(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
                      int64_t Br, int64_t Bc, int64_t qt, int64_t* first,
                      int64_t* last, int64_t* count) {
+  oracle_kv_tiles_window(Nq, Nk, causal, key_len, 0, Br, Bc, qt, first, last,
+                         count);
+}
+
+void oracle_kv_tiles_window(int64_t Nq, int64_t Nk, int causal,
+                            int64_t key_len, int64_t window, int64_t Br,
+                            int64_t Bc, int64_t qt, int64_t* first,
+                            int64_t* last, int64_t* count) {
   *first = -1; *last = -1; *count = 0;
   const int64_t i0 = qt * Br, i1 = (qt + 1) * Br < Nq ? (qt + 1) * Br : Nq;
   const int64_t ntiles = (Nk + Bc - 1) / Bc;
@@ -105,9 +130,10 @@ void oracle_kv_tiles(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
     const int64_t j0 = jt * Bc, j1 = (jt + 1) * Bc < Nk ? (jt + 1) * Bc : Nk;
     int touched = 0;
     for (int64_t i = i0; i < i1 && !touched; ++i) {
-      const int64_t vis = oracle_visible_prefix(i, Nq, Nk, causal, key_len);
+      int64_t lo, hi;
+      oracle_visible_range(i, Nq, Nk, causal, key_len, window, &lo, &hi);
       for (int64_t j = j0; j < j1; ++j)
-        if (j < vis) { touched = 1; break; }
+        if (j >= lo && j < hi) { touched = 1; break; }
     }
     if (touched) {
       if (*first < 0) *first = jt;
@@ -123,6 +149,7 @@ typedef struct {
   const uint16_t *q, *k, *v;
   int64_t B, Hq, Hkv, Nq, Nk, d;
   int causal;
+  int64_t window; /* > 0: sliding window ([AME] 11) */
   double scale;
   const int32_t* key_lens;
   int rope;
@@ -179,7 +206,10 @@ static void row_naive(job_t* J, int64_t r, double* qrow, double* krow,
   const int64_t i = r % J->Nq, h = (r / J->Nq) % J->Hq, b = r / (J->Nq * J->Hq);
   const int64_t g = h / (J->Hq / J->Hkv); /* query head -> kv head ([AME] 9) */
   const int64_t key_len = J->key_lens ? J->key_lens[b] : J->Nk;
-  const int64_t n = oracle_visible_prefix(i, J->Nq, J->Nk, J->causal, key_len);
+  int64_t lo, hi;
+  oracle_visible_range(i, J->Nq, J->Nk, J->causal, key_len, J->window, &lo,
+                       &hi);
+  const int64_t n = hi - lo;
   for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
   if (n == 0) { *lse_out = -INFINITY; return; }
 
@@ -191,17 +221,17 @@ static void row_naive(job_t* J, int64_t r, double* qrow, double* krow,
       for (int64_t c = 0; c < d; ++c) qrow[c] = round_to_bf16(qrow[c]);
   }
 
-  for (int64_t j = 0; j < n; ++j) {
+  for (int64_t j = lo; j < hi; ++j) {
     load_key(J, J->k, b, g, j, J->rope, krow);
     double dot = 0.0;
     for (int64_t c = 0; c < d; ++c) dot += qrow[c] * krow[c];
-    s[j] = J->scale * dot;
+    s[j - lo] = J->scale * dot;
   }
   /* stable softmax: p = exp(s - m) / l */
   oracle_softmax(s, n, p);
-  for (int64_t j = 0; j < n; ++j) {
+  for (int64_t j = lo; j < hi; ++j) {
     load_key(J, J->v, b, g, j, 0, krow);
-    for (int64_t c = 0; c < d; ++c) out[c] += p[j] * krow[c];
+    for (int64_t c = 0; c < d; ++c) out[c] += p[j - lo] * krow[c];
   }
   *lse_out = oracle_logsumexp(s, n);
 }
@@ -213,14 +243,17 @@ static void row_online(job_t* J, int64_t r, double* qrow, double* krow,
   const int64_t i = r % J->Nq, h = (r / J->Nq) % J->Hq, b = r / (J->Nq * J->Hq);
   const int64_t g = h / (J->Hq / J->Hkv);
   const int64_t key_len = J->key_lens ? J->key_lens[b] : J->Nk;
-  const int64_t n = oracle_visible_prefix(i, J->Nq, J->Nk, J->causal, key_len);
+  int64_t lo, hi;
+  oracle_visible_range(i, J->Nq, J->Nk, J->causal, key_len, J->window, &lo,
+                       &hi);
+  const int64_t n = hi - lo;
   const uint16_t* qsrc = J->q + r * d;
   for (int64_t c = 0; c < d; ++c) qrow[c] = bf16_bits_to_double(qsrc[c]);
 
   double m = -INFINITY, l = 0.0;
   for (int64_t c = 0; c < d; ++c) acc[c] = 0.0;
-  for (int64_t start = 0; start < n; start += J->block) {
-    const int64_t stop = start + J->block < n ? start + J->block : n;
+  for (int64_t start = lo; start < hi; start += J->block) {
+    const int64_t stop = start + J->block < hi ? start + J->block : hi;
     double bmax = -INFINITY;
     for (int64_t j = start; j < stop; ++j) {
       load_key(J, J->k, b, g, j, 0, krow);
@@ -319,7 +352,8 @@ static int run_rows(job_t* proto, int nthreads) {
 
 int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
-                     int64_t Nk, int64_t d, int causal, double scale,
+                     int64_t Nk, int64_t d, int causal, int64_t window,
+                     double scale,
                      const int32_t* key_lens, int rope, double rope_base,
                      int rope_pairing, int rope_round, int64_t q_pos_offset,
                      int64_t k_pos_offset, const int64_t* rows, int64_t nrows,
@@ -328,7 +362,8 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v;
   J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d;
-  J.causal = causal; J.scale = scale; J.key_lens = key_lens;
+  J.causal = causal; J.window = window; J.scale = scale;
+  J.key_lens = key_lens;
   J.rope = rope; J.rope_base = rope_base; J.rope_pairing = rope_pairing;
   J.rope_round = rope_round;
   J.q_pos_offset = q_pos_offset; J.k_pos_offset = k_pos_offset;
@@ -339,7 +374,8 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 int oracle_attn_online_rows(const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, int64_t B, int64_t Hq,
                             int64_t Hkv, int64_t Nq, int64_t Nk, int64_t d,
-                            int causal, double scale, const int32_t* key_lens,
+                            int causal, int64_t window, double scale,
+                            const int32_t* key_lens,
                             int64_t block, const int64_t* rows, int64_t nrows,
                             double* o, double* lse, int nthreads) {
   if (block <= 0) return -1;
@@ -347,7 +383,8 @@ int oracle_attn_online_rows(const uint16_t* q, const uint16_t* k,
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v;
   J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d;
-  J.causal = causal; J.scale = scale; J.key_lens = key_lens;
+  J.causal = causal; J.window = window; J.scale = scale;
+  J.key_lens = key_lens;
   J.block = block; J.rows = rows; J.nrows = nrows; J.o = o; J.lse = lse;
   return run_rows(&J, nthreads);
 }

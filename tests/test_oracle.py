@@ -447,3 +447,72 @@ def test_kv_tile_sets_closed_forms():
     # bottom-right alignment with Nq < Nk shifts the diagonal right by Nk - Nq
     assert oracle.kv_tiles(128, 1024, True, 1024, 128, 128, 0) == (0, 7, 8)
     assert oracle.visible_prefix(0, 128, 1024, True, 1024) == 897
+
+
+# -------------------------------------------------------- sliding window ----
+
+def window_mask(Nq, Nk, w, causal):
+    """The pages' sliding-window legality ('Attention mechanisms ...', section
+    11: abs(i - j) < w, plus j <= i when causal), written with np.ogrid as on
+    the page, with query positions bottom-right aligned when Nq < Nk."""
+    i, j = np.ogrid[:Nq, :Nk]
+    p = i + (Nk - Nq)
+    allowed = np.abs(p - j) < w
+    if causal:
+        allowed &= (j <= p)
+    return allowed
+
+
+@pytest.mark.parametrize("Nq,Nk,w,causal", [(40, 40, 5, True), (40, 40, 5, False),
+                                            (16, 50, 7, True), (33, 33, 1, True),
+                                            (33, 33, 100, False)])
+def test_window_matches_library_sdpa(Nq, Nk, w, causal):
+    B, H, d = 2, 2, 16
+    q = synth.normal_bf16((B, H, Nq, d), 201)
+    k = synth.normal_bf16((B, H, Nk, d), 202)
+    v = synth.normal_bf16((B, H, Nk, d), 203)
+    o, lse = oracle.attn_rows(q, k, v, causal, 0.25, window=w)
+    m = torch.from_numpy(window_mask(Nq, Nk, w, causal))
+    O = F.scaled_dot_product_attention(f64(q), f64(k), f64(v), attn_mask=m, scale=0.25)
+    S = (torch.matmul(f64(q), f64(k).transpose(-1, -2)) * 0.25).masked_fill(~m, -math.inf)
+    L = scipy.special.logsumexp(S.numpy(), axis=-1).reshape(-1)
+    ok = np.broadcast_to(m.numpy().any(-1), (B, H, Nq)).reshape(-1)
+    assert np.max(np.abs(o[ok] - O.numpy().reshape(-1, d)[ok])) < 1e-13
+    assert np.max(np.abs(lse[ok] - L[ok])) < 1e-12
+
+
+def test_window_counts_closed_form():
+    N, d, w = 60, 8, 9
+    zero = np.zeros((1, 1, N, d), np.uint16)
+    k = synth.normal_bf16((1, 1, N, d), 211)
+    _, lse = oracle.attn_rows(zero, k, k, True, 1.0, window=w)
+    for i in range(N):
+        assert round(math.exp(lse[i])) == min(i + 1, w)
+    _, lse = oracle.attn_rows(zero, k, k, False, 1.0, window=w)
+    for i in range(N):
+        assert round(math.exp(lse[i])) == min(i + w, N) - max(0, i - w + 1)
+
+
+def test_window_online_equals_naive():
+    B, H, N, d = 1, 2, 70, 16
+    q = synth.normal_bf16((B, H, N, d), 221)
+    k = synth.normal_bf16((B, H, N, d), 222)
+    v = synth.normal_bf16((B, H, N, d), 223)
+    for w in (1, 3, 17, 70):
+        o1, l1 = oracle.attn_rows(q, k, v, True, 0.25, window=w)
+        for block in (1, 4, 16):
+            o2, l2 = oracle.attn_online_rows(q, k, v, True, 0.25, block, window=w)
+            assert np.max(np.abs(o1 - o2)) < 1e-13 and np.max(np.abs(l1 - l2)) < 1e-13
+
+
+def test_window_tile_sets_closed_forms():
+    Br = Bc = 128
+    for kk in (1, 2, 3):
+        w = 128 * kk
+        for qt in range(8):
+            first = max(0, qt - kk)
+            assert oracle.kv_tiles(1024, 1024, True, 1024, Br, Bc, qt, window=w) == \
+                (first, qt, qt - first + 1)
+    # a window of one key: each row sees only itself
+    for i in (0, 5, 127, 128):
+        assert oracle.visible_range(i, 256, 256, True, 256, 1) == (i, i + 1)
