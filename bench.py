@@ -15,7 +15,8 @@ collective on the data path).
 The JSON line also carries: the roofline of the dominant kernel, the
 end-to-end figure through the public API with host buffers, the oracle timed
 on host cores (rank 0, N=1, bounded sample), SM clocks sampled during the
-timed region, and the decode workload (MQA over a ragged KV cache) in GB/s.
+timed region, the decode workload (MQA over a ragged KV cache) in GB/s, and
+the sliding-window prefill workload in useful TFLOP/s.
 """
 from __future__ import annotations
 
@@ -85,6 +86,7 @@ def parse_args():
     p.add_argument("--config", default="mha_prefill", choices=sorted(synth.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-decode", action="store_true")
+    p.add_argument("--no-window", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -184,7 +186,8 @@ def oracle_sample(w, seconds, seed=12345, rows_per_batch=None):
             i = int(r % w.Nq)
             b = int(r // (w.Nq * w.Hq))
             L = w.Nk if kl is None else int(kl[b])
-            f += 4.0 * w.d * oracle.visible_prefix(i, w.Nq, w.Nk, w.causal, L)
+            lo, hi = oracle.visible_range(i, w.Nq, w.Nk, w.causal, L, w.window)
+            f += 4.0 * w.d * (hi - lo)
         return f
 
     rope = (dict(base=synth.ROPE_BASE, pairing=0, q_pos_offset=0, k_pos_offset=0)
@@ -195,7 +198,7 @@ def oracle_sample(w, seconds, seed=12345, rows_per_batch=None):
         rows = np.sort(rng.integers(0, total_rows, size=n)).astype(np.int64)
         t0 = time.perf_counter()
         oracle.attn_rows(x["q"], x["k"], x["v"], w.causal, w.scale, key_lens=kl, rows=rows,
-                         rope_cfg=rope, nthreads=threads)
+                         rope_cfg=rope, nthreads=threads, window=w.window)
         dt = time.perf_counter() - t0
         used_f += flops(rows)
         used_t += dt
@@ -291,7 +294,7 @@ def run_ours(args):
         c = i % copies
         q, k = (QR, KR) if w.rope else (Q[c], K[c])
         eb.attn_fwd_ws(q, k, V[c], ws, causal=w.causal, scale=w.scale, key_lens=kl,
-                       out=O, lse=LSE)
+                       out=O, lse=LSE, window=w.window)
 
     def step(i):
         # one pass of the whole path: the RoPE prologue (when the workload has
@@ -341,6 +344,7 @@ def run_ours(args):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
                    "Nk": w.Nk, "d": w.d, "causal": w.causal, "rope": w.rope,
                    "key_lens": list(w.key_lens) if w.key_lens else None,
+                   "window": w.window,
                    "l2": f"{copies} rotating input copies ({copies * per_copy / 1e6:.0f} MB > "
                          f"126 MB L2)",
                    "parallelism": f"replicas x{world} (independent batch per GPU)"},
@@ -378,6 +382,9 @@ def run_ours(args):
     # ---- decode workload (HBM-bound half of the metric), same run
     if not args.no_decode and w.Nq != 1 and rank == 0 and world == 1:
         line["decode"] = run_decode(torch, eb, device, stream, peaks, peak_src)
+    # ---- sliding-window prefill, same run
+    if not args.no_window and w.name != "long_window" and rank == 0 and world == 1:
+        line["window"] = run_window(torch, eb, device, stream, peaks, peak_src)
 
     # ---- oracle on host cores (rank 0, N=1 only)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -434,6 +441,37 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None):
             "gpu_launches": 2 * n}
 
 
+def run_window(torch, eb, device, stream, peaks, peak_src, steps=None):
+    """The sliding-window prefill workload (inputs larger than L2, one copy)."""
+    w = synth.WORKLOADS["long_window"]
+    x = synth.make_inputs(w)
+    q, k, v = (to_dev(x[n], torch, device) for n in ("q", "k", "v"))
+    O = torch.empty_like(q)
+    LSE = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
+    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d),
+                     dtype=torch.uint8, device=device)
+
+    def step(i):
+        eb.attn_fwd_ws(q, k, v, ws, causal=w.causal, scale=w.scale, out=O, lse=LSE,
+                       window=w.window)
+
+    for i in range(3):
+        step(i)
+    probe = time_steps(step, 3, torch, None, stream) / 3
+    n = steps or max(10, int(1000.0 / max(probe, 1e-3)))
+    ms = time_steps(step, n, torch, None, stream)
+    tf = w.flops() * n / (ms / 1e3) / 1e12
+    mb = (x["q"].nbytes + x["k"].nbytes + x["v"].nbytes) / 1e6
+    return {"metric": "useful TFLOP/s (4 d per visible (row, key) pair)", "value": tf,
+            "unit": "TFLOP/s", "workload": w.name, "window": w.window, "steps": n,
+            "ms_per_step": ms / n, "flops_per_step": w.flops(),
+            "l2": f"inputs {mb:.0f} MB > 126 MB L2",
+            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
+                         "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
+                         "traffic": ncu_traffic(w.name), "peak_source": peak_src},
+            "gpu_launches": n}
+
+
 # -------------------------------------------------------------- reference ---
 
 def run_reference(args):
@@ -456,7 +494,7 @@ def run_reference(args):
 
     def one(rows):
         oracle.attn_rows(x["q"], x["k"], x["v"], w.causal, w.scale, key_lens=kl, rows=rows,
-                         rope_cfg=rope, nthreads=threads)
+                         rope_cfg=rope, nthreads=threads, window=w.window)
 
     def flops(rows):
         f = 0.0
@@ -464,7 +502,8 @@ def run_reference(args):
             i = int(r % w.Nq)
             b = int(r // (w.Nq * w.Hq))
             L = w.Nk if kl is None else int(kl[b])
-            f += 4.0 * w.d * oracle.visible_prefix(i, w.Nq, w.Nk, w.causal, L)
+            lo, hi = oracle.visible_range(i, w.Nq, w.Nk, w.causal, L, w.window)
+            f += 4.0 * w.d * (hi - lo)
         return f
 
     steps = args.steps or 5
@@ -489,7 +528,7 @@ def run_reference(args):
             "ms_per_step": 1e3 * t_total / steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
-                       "Nk": w.Nk, "d": w.d, "causal": w.causal},
+                       "Nk": w.Nk, "d": w.d, "causal": w.causal, "window": w.window},
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,

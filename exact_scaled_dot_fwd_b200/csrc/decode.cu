@@ -76,6 +76,7 @@ struct DecodeArgs {
   float* part_o;
   float* part_lse;
   int B, Hq, Hkv, Nk, G, grid;
+  int kv_lo;        // first key of every unit (sliding window), 0 without one
   float scale_log2;
 };
 
@@ -121,6 +122,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
       if (b < B) {
         len = a.key_lens ? a.key_lens[b] : a.Nk;
         len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+        len = len > a.kv_lo ? len - a.kv_lo : 0;   // keys [kv_lo, L)
         lens_s[b] = len;
       }
       long long x = len;
@@ -180,7 +182,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
           uint8_t* kt = smem + L::kRing + st * L::kStageBytes;
           uint8_t* vt = kt + L::kTileBytes;
           mbar_arrive_expect_tx(&full[st], L::kStageBytes);
-          const int row = s.u * a.Nk + t;
+          const int row = s.u * a.Nk + a.kv_lo + t;
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx) {
             tma_load_2d(kt + bx * (kTileKeys * 128), &tmap_k, bx * 64, row, &full[st]);
@@ -383,6 +385,7 @@ struct CombineArgs {
   __nv_bfloat16* o;
   float* lse;
   int B, Hq, Hkv, Nk, G, grid;
+  int kv_lo;
 };
 
 constexpr int kCombineThreads = 256;
@@ -403,6 +406,7 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
   for (int bb = threadIdx.x; bb < a.B; bb += blockDim.x) {
     int len = a.key_lens ? a.key_lens[bb] : a.Nk;
     len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+    len = len > a.kv_lo ? len - a.kv_lo : 0;
     total += len;
     if (bb < b) before += len;
     if (bb == b) s_len = len;
@@ -524,8 +528,8 @@ bool decode_supported(int B, int Hq, int Hkv, int d) {
 }
 
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nk, int d, float scale, const int32_t* key_lens, void* workspace,
-                  const DecodePlan& p, cudaStream_t st) {
+                  int Hkv, int Nk, int d, int kv_lo, float scale, const int32_t* key_lens,
+                  void* workspace, const DecodePlan& p, cudaStream_t st) {
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)B * Hkv * Nk;
   if (make_tmap_2d_bf16(&tk, k, d, rows, 64, kTileKeys) != ATTN_OK) return ATTN_ECUDA;
@@ -536,11 +540,12 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.part_o_bytes);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = p.G; a.grid = p.grid;
+  a.kv_lo = kv_lo;
   a.scale_log2 = scale * kLog2e;
   int rc;
   if (decode_tc_supported(B, Hq, Hkv, d)) {
-    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nk, scale, key_lens, a.part_o, a.part_lse,
-                                p.grid, st);
+    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nk, kv_lo, scale, key_lens, a.part_o,
+                                a.part_lse, p.grid, st);
   } else {
     const int MT = (p.G + 15) / 16;
     if (d == 128) {
@@ -561,6 +566,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   c.o = static_cast<__nv_bfloat16*>(o);
   c.lse = lse;
   c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.Nk = Nk; c.G = p.G; c.grid = p.grid;
+  c.kv_lo = kv_lo;
   // shared memory: the unit's slot lse's ([slots][heads of the block], at most
   // grid + 1 slots) + [heads of the block]
   const int hb = kCombineThreads / d;

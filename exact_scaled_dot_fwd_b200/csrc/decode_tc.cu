@@ -174,6 +174,7 @@ struct DecodeTcArgs {
   float* part_o;
   float* part_lse;
   int B, Hq, Hkv, Nk, G, grid;
+  int kv_lo;        // first key of every unit (sliding window), 0 without one
   float scale_log2;
 };
 
@@ -224,6 +225,7 @@ __global__ void __launch_bounds__(192, 1)
       if (b < B) {
         len = a.key_lens ? a.key_lens[b] : a.Nk;
         len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
+        len = len > a.kv_lo ? len - a.kv_lo : 0;   // keys [kv_lo, L)
         lens_s[b] = len;
       }
       long long x = len;
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(192, 1)
         for (int bx = 0; bx < 2; ++bx)
           tma_load_2d(smem + L::kQ + bx * L::kQBox, &tmap_q, bx * 64, b * a.Hq + h * a.G,
                       &bars[L::Q_FULL]);
-        const int row0 = s.u * a.Nk + s.lo;
+        const int row0 = s.u * a.Nk + a.kv_lo + s.lo;
         for (int j = 0; j < n; ++j, ++g) {
           const int ks = g % KS, vs = g % VS;
           if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / KS) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -523,8 +525,8 @@ bool decode_tc_supported(int B, int Hq, int Hkv, int d) {
 }
 
 int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                           int Nk, float scale, const int32_t* key_lens, float* part_o,
-                           float* part_lse, int grid, cudaStream_t st) {
+                           int Nk, int kv_lo, float scale, const int32_t* key_lens,
+                           float* part_o, float* part_lse, int grid, cudaStream_t st) {
   const int G = Hq / Hkv;
   const int N = G <= 16 ? 16 : (G <= 32 ? 32 : 64);
   CUtensorMap tq, tk, tv;
@@ -538,6 +540,7 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   a.part_o = part_o;
   a.part_lse = part_lse;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = G; a.grid = grid;
+  a.kv_lo = kv_lo;
   a.scale_log2 = scale * kLog2e;
   if (N == 16) return launch_tc_t<16>(grid, tq, tk, tv, a, st);
   if (N == 32) return launch_tc_t<32>(grid, tq, tk, tv, a, st);

@@ -35,21 +35,23 @@ bool decode_supported(int B, int Hq, int Hkv, int d);
 // the same partial-result format as the mma.sync split kernel.
 bool decode_tc_supported(int B, int Hq, int Hkv, int d);
 int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                           int Nk, float scale, const int32_t* key_lens, float* part_o,
-                           float* part_lse, int grid, cudaStream_t st);
+                           int Nk, int kv_lo, float scale, const int32_t* key_lens,
+                           float* part_o, float* part_lse, int grid, cudaStream_t st);
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nk, int d, float scale, const int32_t* key_lens, void* workspace,
-                  const DecodePlan& p, cudaStream_t st);
+                  int Hkv, int Nk, int d, int kv_lo, float scale, const int32_t* key_lens,
+                  void* workspace, const DecodePlan& p, cudaStream_t st);
+// Decode reads keys [kv_lo, min(key_lens[b], Nk)) of every sequence; kv_lo is
+// Nk - window (at least 0) under a sliding window of `window` keys, else 0.
 
 // ---- prefill (Nq > 1)
 bool prefill_supported(int d);
 size_t prefill_workspace_bytes();   // scheduler counter
 void prefill_tile_shape(int d, int* Br, int* Bc);
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                   int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                   int Hkv, int Nq, int Nk, int d, int causal, int window, float scale,
                    const int32_t* key_lens, void* workspace, int num_sms, cudaStream_t st);
-int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, const int32_t* key_lens,
-                     int32_t* first, int32_t* count, cudaStream_t st);
+int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window,
+                     const int32_t* key_lens, int32_t* first, int32_t* count, cudaStream_t st);
 
 // ---- RoPE
 int launch_rope(const void* x_in, void* x_out, int B, int H, int N, int d, float base,

@@ -36,6 +36,12 @@
 // Lazy rescale: O and l are rescaled only when a row's max grows by more
 // than 8 (log2 units); otherwise the stale max is kept (P <= 2^8, exact in
 // the final O / l because O and l share the same reference).
+//
+// Sliding window ("Attention mechanisms ...", section 11): a query tile
+// visits the contiguous KV-tile range that covers its rows' windows.  When
+// the two tiles of an item start at different KV tiles, both walk the union
+// of their ranges (one or two extra tiles per item, fully masked for the
+// tile they do not belong to), so the slots stay on one KV stream.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -92,7 +98,8 @@ struct Smem {
 };
 
 struct Tile {
-  int row_tile, head, count, first_masked;
+  int row_tile, head, count;
+  int um_begin, um_end;   // KV tiles (absolute index) that need no element mask
 };
 
 __device__ __forceinline__ float max3(float a, float b, float c) {
@@ -109,6 +116,7 @@ struct FwdArgs {
   float* lse;
   const int32_t* key_lens;
   int B, Hq, Hkv, Nq, Nk, causal;
+  int window;       // sliding window in keys, 0 = none
   int head_pairs;   // 1: tiles are heads (2p, 2p+1) at one row tile; 0: row tiles 2p, 2p+1
   int ntq;          // ceil(Nq / 128)
   int units;        // items per cost rank (head_pairs: B*Hq/2, else B*Hq)
@@ -122,14 +130,17 @@ namespace pf {
 
 struct Item {
   Tile tl[2];       // tl[0] has the fewer KV tiles
-  int b, n, kv_row0, L;
+  int b, n, L;
+  int kv_begin;     // KV tile of step 0 (both slots)
+  int kv_row0;      // cache row of KV tile kv_begin
 };
 
-// Item `idx` of the ordered list.  Ranks walk the row tiles (row pairs)
+// Item `idx` of the ordered list (window: the sliding window, 0 = none;
+// callers pass a compile-time 0 when the launch has no window).  Ranks walk the row tiles (row pairs)
 // from the most KV tiles to the fewest when causal; bands of `band` ranks
 // keep one unit's (head's) items next to each other so the CTAs that run at
 // the same time share its K/V in L2 (band = 1: plain rank-major order).
-__device__ __forceinline__ Item make_item(const FwdArgs& a, int idx) {
+__device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window) {
   Item it;
   const int per_band = a.units * a.band;
   const int full = a.ranks / a.band;
@@ -161,16 +172,27 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx) {
     it.tl[0].head = it.tl[1].head = h;
   }
   it.L = clamp_len(a.key_lens ? a.key_lens[it.b] : a.Nk, a.Nk);
+  int begin[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
-    if (it.tl[t].row_tile < a.ntq) {
-      const KvRange r = kv_tile_range(it.tl[t].row_tile, kM, kN, a.Nq, a.Nk, a.causal, it.L);
-      it.tl[t].count = r.count;
-      it.tl[t].first_masked = r.first_masked;
-    } else {
-      it.tl[t].count = 0;
-      it.tl[t].first_masked = 0;
-    }
+    KvRange r;
+    r.begin = r.count = r.um_begin = r.um_end = 0;
+    if (it.tl[t].row_tile < a.ntq)
+      r = kv_tile_range(it.tl[t].row_tile, kM, kN, a.Nq, a.Nk, a.causal, it.L, window);
+    begin[t] = r.begin;
+    it.tl[t].count = r.count;
+    it.tl[t].um_begin = r.um_begin;
+    it.tl[t].um_end = r.um_end;
+  }
+  it.kv_begin = 0;
+  if (it.tl[0].count > 0 && it.tl[1].count > 0 && begin[0] != begin[1]) {
+    // different first tiles (sliding window): both walk the union
+    const int b0 = begin[0] < begin[1] ? begin[0] : begin[1];
+    const int e0 = begin[0] + it.tl[0].count, e1 = begin[1] + it.tl[1].count;
+    it.kv_begin = b0;
+    it.tl[0].count = it.tl[1].count = (e0 > e1 ? e0 : e1) - b0;
+  } else {
+    it.kv_begin = it.tl[0].count > 0 ? begin[0] : begin[1];
   }
   if (it.tl[0].count > it.tl[1].count) {
     const Tile x = it.tl[0];
@@ -179,19 +201,20 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx) {
   }
   it.n = it.tl[1].count;
   const int hk = it.tl[1].head / (a.Hq / a.Hkv);
-  it.kv_row0 = (it.b * a.Hkv + hk) * a.Nk;
+  it.kv_row0 = (it.b * a.Hkv + hk) * a.Nk + it.kv_begin * kN;
   return it;
 }
 
 }  // namespace pf
 
-template <int D>
+template <int D, bool kWindow>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, FwdArgs a) {
   using namespace pf;
   using L = Smem<D>;
   constexpr int kBoxes = D / 64;
+  const int window = kWindow ? a.window : 0;
   constexpr int kKS = L::kKS, kVS = L::kVS;
   // TMEM columns: S of tile t at 128 t, O of tile t at 256 + D t
   constexpr uint32_t kIdescS = tc::idesc_bf16(kM, kN, false, false);
@@ -252,7 +275,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         mbar_arrive(&bars[L::ITEM_FULL + slot]);
         ++k;
         if (idx < 0) break;
-        const Item it = make_item(a, idx);
+        const Item it = make_item(a, idx, window);
         // claim the next item only while issuing this item's last tile, so
         // no CTA sits on a claimed item (greedy longest-first stays greedy);
         // the atomic's latency hides behind the last loads
@@ -289,7 +312,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       int qn[2] = {0, 0}, k = 0;
       bool ok = true;
       for (int idx; ok && (idx = next_item(k)) >= 0;) {
-        const Item it = make_item(a, idx);
+        const Item it = make_item(a, idx, window);
         if (it.n == 0) continue;
         for (int t = 0; t < 2 && ok; ++t) {
           if (it.tl[t].count == 0) continue;
@@ -337,27 +360,31 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       // with fewer tiles moves on while the other one finishes.
       int qf[2] = {0, 0}, pw[2] = {0, 0}, g = 0, k = 0;
       bool ok = true;
-      auto fetch = [&](Item& it) -> bool {   // next item that has KV tiles
+      struct Counts { int c[2], n; };   // all the issuer needs of an item
+      auto fetch = [&](Counts& it) -> bool {   // next item that has KV tiles
         for (int idx; (idx = next_item(k)) >= 0;) {
-          it = make_item(a, idx);
+          const Item full = make_item(a, idx, window);
+          it.c[0] = full.tl[0].count;
+          it.c[1] = full.tl[1].count;
+          it.n = full.n;
           if (it.n > 0) return true;
         }
         return false;
       };
-      auto issue_first_s = [&](const Item& it, int t, int ks) -> bool {
+      auto issue_first_s = [&](const Counts& it, int t, int ks) -> bool {
         if (!mbar_wait(&bars[L::Q_FULL + t], qf[t] & 1, abort_flag)) return false;
         ++qf[t];
         tc::fence_after();
         issue_s(t, ks);
         tc::commit(&bars[L::S_FULL + t]);
-        if (it.tl[t].count == 1) tc::commit(&bars[L::Q_EMPTY + t]);
+        if (it.c[t] == 1) tc::commit(&bars[L::Q_EMPTY + t]);
         return true;
       };
-      Item cur, nxt;
+      Counts cur, nxt;
       if (fetch(cur)) {
         ok = mbar_wait(&bars[L::K_FULL + 0], 0, abort_flag);
         for (int t = 0; t < 2 && ok; ++t)
-          if (cur.tl[t].count > 0) ok = issue_first_s(cur, t, 0);
+          if (cur.c[t] > 0) ok = issue_first_s(cur, t, 0);
         if (ok) tc::commit(&bars[L::K_EMPTY + 0]);
         int j = 0;
         while (ok) {
@@ -374,7 +401,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             return true;
           };
           for (int t = 0; t < 2 && ok; ++t) {
-            const int cnt = cur.tl[t].count;
+            const int cnt = cur.c[t];
             if (j < cnt) {
               if (!mbar_wait(&bars[L::P_FULL + t], pw[t] & 1, abort_flag)) { ok = false; break; }
               ++pw[t];
@@ -387,7 +414,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
               issue_s(t, ksn);
               tc::commit(&bars[L::S_FULL + t]);
               if (j + 2 == cnt) tc::commit(&bars[L::Q_EMPTY + t]);
-            } else if (last && more && nxt.tl[t].count > 0) {  // next item, first tile
+            } else if (last && more && nxt.c[t] > 0) {  // next item, first tile
               if (!need_k() || !issue_first_s(nxt, t, ksn)) { ok = false; break; }
             }
           }
@@ -418,19 +445,22 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     int sw = 0, ow = 0, k = 0;
     bool ok = true;
     for (int idx; ok && (idx = next_item(k)) >= 0;) {
-      const Item it = make_item(a, idx);
+      const Item it = make_item(a, idx, window);
       const Tile T = t == 0 ? it.tl[0] : it.tl[1];
       if (T.row_tile >= a.ntq) continue;
       const int row = T.row_tile * kM + r;
-      const int nvis = visible_prefix(row, a.Nq, a.Nk, a.causal, it.L);
+      int vlo, vhi;   // this row's visible keys [vlo, vhi)
+      visible_range(row, a.Nq, a.Nk, a.causal, it.L, window, &vlo, &vhi);
       float m_run = -INFINITY, l_run = 0.f;
 
       for (int j = 0; j < T.count; ++j) {
         if (!mbar_wait(&bars[L::S_FULL + t], sw & 1, abort_flag)) { ok = false; break; }
         ++sw;
         tc::fence_after();
-        const bool masked = j >= T.first_masked;
-        const int lim = nvis - j * kN;   // keys [0, lim) of this tile are visible
+        const int kt = it.kv_begin + j;   // KV tile index
+        const bool masked = kWindow ? (kt < T.um_begin || kt >= T.um_end) : j >= T.um_end;
+        const int lim = vhi - kt * kN;    // keys [base, lim) of this tile are visible
+        const int base = vlo - kt * kN;
         // pass 1: row max of the (masked) scores
         float mx = -INFINITY;
         if (!masked) {
@@ -450,7 +480,10 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
             tc::wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = fmaxf(mx, 32 * c4 + e >= lim ? -INFINITY : sv[e]);
+            for (int e = 0; e < 32; ++e) {
+              const int c = 32 * c4 + e;
+              mx = fmaxf(mx, (c >= lim || (kWindow && c < base)) ? -INFINITY : sv[e]);
+            }
           }
         }
         const float m_tile = mx * sl2;
@@ -507,8 +540,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
 #pragma unroll
             for (int e = 0; e < 16; ++e) {
               const int c = 32 * c4 + 2 * e;
-              const float x0 = c >= lim ? -INFINITY : sv[2 * e];
-              const float x1 = c + 1 >= lim ? -INFINITY : sv[2 * e + 1];
+              const float x0 = (c >= lim || (kWindow && c < base)) ? -INFINITY : sv[2 * e];
+              const float x1 = (c + 1 >= lim || (kWindow && c + 1 < base)) ? -INFINITY : sv[2 * e + 1];
               const float p0 = exp2_approx(fmaf(x0, sl2, -m_use));
               const float p1 = exp2_approx(fmaf(x1, sl2, -m_use));
               rs += p0 + p1;
@@ -583,7 +616,7 @@ void prefill_tile_shape(int d, int* Br, int* Bc) {
 }
 
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                   int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                   int Hkv, int Nq, int Nk, int d, int causal, int window, float scale,
                    const int32_t* key_lens, void* workspace, int num_sms, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (make_tmap_3d_bf16(&tq, q, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
@@ -595,6 +628,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   a.lse = lse;
   a.key_lens = key_lens;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.causal = causal;
+  a.window = window;
   a.ntq = (Nq + pf::kM - 1) / pf::kM;
   a.head_pairs = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
   a.scale_log2 = scale * kLog2e;
@@ -618,42 +652,39 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   a.band = band;
   // the item counter starts every launch at zero (stream-ordered)
   if (cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) != cudaSuccess) return ATTN_ECUDA;
-  if (d == 128) {
-    auto kern = prefill_tc_kernel<128>;
-    const int smem = pf::Smem<128>::kTotal;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return ATTN_ECUDA;
-    kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, a);
-  } else {
-    auto kern = prefill_tc_kernel<64>;
-    const int smem = pf::Smem<64>::kTotal;
-    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
-      return ATTN_ECUDA;
-    kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, a);
-  }
+  // a window shifts each tile's first visible key: a separate instantiation
+  // keeps that arithmetic out of the unwindowed kernel
+  const bool win = window > 0;
+  auto kern = d == 128 ? (win ? prefill_tc_kernel<128, true> : prefill_tc_kernel<128, false>)
+                       : (win ? prefill_tc_kernel<64, true> : prefill_tc_kernel<64, false>);
+  const int smem = d == 128 ? pf::Smem<128>::kTotal : pf::Smem<64>::kTotal;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
+    return ATTN_ECUDA;
+  kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
-__global__ void tile_plan_kernel(const int32_t* key_lens, int B, int Nq, int Nk, int causal, int Br,
-                                 int Bc, int nqt, int32_t* first, int32_t* count) {
+__global__ void tile_plan_kernel(const int32_t* key_lens, int B, int Nq, int Nk, int causal,
+                                 int window, int Br, int Bc, int nqt, int32_t* first,
+                                 int32_t* count) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * nqt) return;
   const int b = idx / nqt, qt = idx - b * nqt;
   const int L_b = clamp_len(key_lens ? key_lens[b] : Nk, Nk);
-  const KvRange r = kv_tile_range(qt, Br, Bc, Nq, Nk, causal, L_b);
-  first[idx] = r.count > 0 ? 0 : -1;
+  const KvRange r = kv_tile_range(qt, Br, Bc, Nq, Nk, causal, L_b, window);
+  first[idx] = r.count > 0 ? r.begin : -1;
   count[idx] = r.count;
 }
 
-int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, const int32_t* key_lens,
-                     int32_t* first, int32_t* count, cudaStream_t st) {
+int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window,
+                     const int32_t* key_lens, int32_t* first, int32_t* count, cudaStream_t st) {
   int Br, Bc;
   prefill_tile_shape(d, &Br, &Bc);
   const int nqt = (Nq + Br - 1) / Br;
   const int n = B * nqt;
   if (n == 0) return ATTN_OK;
-  tile_plan_kernel<<<(n + 255) / 256, 256, 0, st>>>(key_lens, B, Nq, Nk, causal, Br, Bc, nqt, first,
-                                                    count);
+  tile_plan_kernel<<<(n + 255) / 256, 256, 0, st>>>(key_lens, B, Nq, Nk, causal, window, Br, Bc,
+                                                    nqt, first, count);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 

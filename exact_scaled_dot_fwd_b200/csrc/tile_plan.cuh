@@ -1,13 +1,14 @@
-// tile_plan.cuh -- which KV tiles a query tile visits, and which of them need
-// element-wise masking.  Used by the prefill kernel and by the tile-plan debug
-// entry point, so both report the same set.
+// tile_plan.cuh -- which keys a query row sees, which KV tiles a query tile
+// visits, and which of them need element-wise masking.  Used by the prefill
+// kernel and by the tile-plan debug entry point, so both report the same set.
 //
-// Key j is visible to query row i iff j < L and (not causal or
-// j <= i + (Nk - Nq)), L = clamp(key_len, 0, Nk).  The visible keys of a row
-// form a prefix whose length grows with i, so a query tile with rows
-// [i0, i1) visits KV tiles 0 .. ceil(n(i1 - 1) / Bc) - 1 (n = prefix length)
-// and every tile at or beyond floor(n(i0) / Bc) holds a masked element for
-// some row.  Tiles wholly past every row's prefix are skipped.
+// Query row i sits at key position p = i + (Nk - Nq) (bottom-right alignment).
+// Key j is visible iff j < L (L = clamp(key_len, 0, Nk)), and, when causal,
+// j <= p, and, with a sliding window w > 0 ("Attention mechanisms ...",
+// section 11), |p - j| < w.  The visible keys of a row form a range
+// [lo, hi) whose ends never decrease with i, and the rows that see any key
+// form one contiguous block, so a query tile's KV tiles are a contiguous
+// range computable in closed form.
 #pragma once
 
 namespace attn {
@@ -16,7 +17,7 @@ __host__ __device__ __forceinline__ int clamp_len(int key_len, int Nk) {
   return key_len < 0 ? 0 : (key_len > Nk ? Nk : key_len);
 }
 
-// Number of visible keys (the prefix length) of query row i.
+// Number of visible keys (the prefix length) of query row i without a window.
 __host__ __device__ __forceinline__ int visible_prefix(int i, int Nq, int Nk, int causal, int L) {
   int n = L;
   if (causal) {
@@ -26,21 +27,71 @@ __host__ __device__ __forceinline__ int visible_prefix(int i, int Nq, int Nk, in
   return n;
 }
 
+// Visible keys [lo, hi) of query row i (hi <= lo: none).
+__host__ __device__ __forceinline__ void visible_range(int i, int Nq, int Nk, int causal, int L,
+                                                       int window, int* lo, int* hi) {
+  int h = visible_prefix(i, Nq, Nk, causal, L);
+  int l = 0;
+  if (window > 0) {
+    const long long p = (long long)i + (Nk - Nq);
+    if (p - window + 1 > l) l = (int)(p - window + 1);
+    if (p + window < h) h = p + window < 0 ? 0 : (int)(p + window);
+  }
+  *lo = l;
+  *hi = h > l ? h : l;
+}
+
 struct KvRange {
-  int count;        // tiles 0 .. count-1 are visited
-  int first_masked; // tiles >= first_masked need the element mask
+  int begin;       // first KV tile visited
+  int count;       // tiles begin .. begin+count-1 are visited
+  int um_begin;    // tiles in [um_begin, um_end) need no element mask
+  int um_end;
 };
 
 __host__ __device__ __forceinline__ KvRange kv_tile_range(int qt, int Br, int Bc, int Nq, int Nk,
-                                                          int causal, int L) {
+                                                          int causal, int L, int window) {
+  KvRange r;
+  r.begin = 0;
+  r.count = 0;
+  r.um_begin = 0;
+  r.um_end = 0;
   const int i0 = qt * Br;
   int i1 = i0 + Br;
   if (i1 > Nq) i1 = Nq;
-  KvRange r;
-  const int nmax = visible_prefix(i1 - 1, Nq, Nk, causal, L);
-  const int nmin = visible_prefix(i0, Nq, Nk, causal, L);
-  r.count = (nmax + Bc - 1) / Bc;
-  r.first_masked = nmin / Bc;
+  if (window <= 0) {
+    // prefix ranges: tiles 0 .. ceil(n_max / Bc) - 1, unmasked below n_min / Bc
+    const int nmax = visible_prefix(i1 - 1, Nq, Nk, causal, L);
+    const int nmin = visible_prefix(i0, Nq, Nk, causal, L);
+    r.count = (nmax + Bc - 1) / Bc;
+    r.um_end = nmin / Bc;
+    return r;
+  }
+  if (i1 <= i0 || L <= 0) return r;
+  // rows that see at least one key: positions p in [p_min, p_max]
+  const long long off = (long long)Nk - Nq;
+  long long p_min = causal ? 0 : (window > 0 ? 1 - (long long)window : (long long)i0 + off);
+  long long p_max = window > 0 ? (long long)L + window - 2 : (long long)i1 - 1 + off;
+  long long pa = (long long)i0 + off, pb = (long long)i1 - 1 + off;
+  if (pa < p_min) pa = p_min;
+  if (pb > p_max) pb = p_max;
+  if (pa > pb) return r;
+  int lo_a, hi_a, lo_b, hi_b;
+  visible_range((int)(pa - off), Nq, Nk, causal, L, window, &lo_a, &hi_a);
+  visible_range((int)(pb - off), Nq, Nk, causal, L, window, &lo_b, &hi_b);
+  const int S = lo_a, E = hi_b;   // union of the rows' ranges
+  if (E <= S) return r;
+  r.begin = S / Bc;
+  r.count = (E + Bc - 1) / Bc - r.begin;
+  // element masks are needed unless a tile lies inside every row's range
+  int lo_first, hi_first, lo_last, hi_last;
+  visible_range(i0, Nq, Nk, causal, L, window, &lo_first, &hi_first);
+  visible_range(i1 - 1, Nq, Nk, causal, L, window, &lo_last, &hi_last);
+  const int um_b = (lo_last + Bc - 1) / Bc;   // first tile at or after every row's lo
+  const int um_e = hi_first / Bc;             // tiles ending at or before every row's hi
+  if (hi_first > lo_last && um_e > um_b) {
+    r.um_begin = um_b;
+    r.um_end = um_e;
+  }
   return r;
 }
 

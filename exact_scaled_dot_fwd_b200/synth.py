@@ -60,6 +60,7 @@ class Workload:
     rope: bool = False
     key_lens: tuple | None = None   # (lo, hi) inclusive uniform range
     note: str = ""
+    window: int = 0                 # sliding window in keys (0 = none)
 
     @property
     def scale(self) -> float:
@@ -70,7 +71,15 @@ class Workload:
         return 1000 * self.number
 
     def flops(self) -> float:
-        """Formula FLOPs: 4*B*Hq*Nq*Nk*d, halved for causal."""
+        """Formula FLOPs: 4*B*Hq*Nq*Nk*d, halved for causal.  With a causal
+        sliding window over Nq == Nk keys (no padding): 4*B*Hq*d times the
+        number of (row, key) pairs inside the window, sum_i min(i + 1, w)."""
+        if self.window:
+            if not (self.causal and self.Nq == self.Nk and self.key_lens is None):
+                raise NotImplementedError("window FLOPs: causal, Nq == Nk, no padding")
+            n, w = self.Nq, min(self.window, self.Nq)
+            pairs = w * (w + 1) // 2 + (n - w) * w
+            return 4.0 * self.B * self.Hq * self.d * pairs
         f = 4.0 * self.B * self.Hq * self.Nq * self.Nk * self.d
         return f / 2 if self.causal else f
 
@@ -87,6 +96,10 @@ WORKLOADS = {
     "long_causal": Workload("long_causal", 5, 1, 32, 32, 32768, 32768, 128, True),
     "cross_padded": Workload("cross_padded", 6, 8, 16, 16, 1024, 4096, 64, False,
                              key_lens=(2048, 4096)),
+    # long causal context under a sliding window of 4096 keys (the pages give
+    # the rule but no size; 4096 is a common choice)
+    "long_window": Workload("long_window", 7, 1, 32, 32, 32768, 32768, 128, True,
+                            window=4096),
 }
 
 ROPE_BASE = 10000.0

@@ -88,6 +88,24 @@ ATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* o,
                 int causal, float scale, const int32_t* key_lens,
                 void* workspace, size_t workspace_bytes, void* stream);
 
+/* Sliding-window attention ("Attention mechanisms ...", section 11): as
+ * attn_fwd_ws, with key j visible to query row i only if, in addition to the
+ * rules above, |p - j| < window, where p = i + (Nk - Nq) is the row's key
+ * position (bottom-right alignment, as for the causal mask).  window = 0
+ * means no window (identical to attn_fwd_ws); window < 0 is ATTN_EINVAL.
+ * With causal = 1 a row sees the last `window` positions up to and including
+ * its own; with causal = 0 it also sees window - 1 positions after it.
+ *   Prefill (Nq > 1) visits only the KV tiles that hold visible keys
+ *   (attn_fwd_tile_plan_window reports them).  Decode (Nq == 1) reads keys
+ *   [max(0, Nk - window), key_lens[b]) of each sequence.
+ *   Workspace: attn_workspace_size(...) bytes, as for attn_fwd_ws.
+ * Errors: as attn_fwd_ws. */
+ATTN_API int attn_fwd_window(const void* q, const void* k, const void* v, void* o,
+                             float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
+                             int causal, int window, float scale,
+                             const int32_t* key_lens, void* workspace,
+                             size_t workspace_bytes, void* stream);
+
 /* Bytes of workspace attn_fwd_ws needs for these sizes on the current device
  * (0 for invalid sizes). */
 ATTN_API size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
@@ -116,6 +134,13 @@ ATTN_API int attn_prefill_tile_shape(int d, int* Br, int* Bc);
 ATTN_API int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal,
                        const int32_t* key_lens, int32_t* first,
                        int32_t* count, void* stream);
+
+/* attn_fwd_tile_plan under a sliding window of `window` keys (0 = none):
+ * first = the first KV tile a query tile visits, count = how many in a row
+ * (the range covers every visible key of the tile's rows and nothing else). */
+ATTN_API int attn_fwd_tile_plan_window(int B, int Nq, int Nk, int d, int causal,
+                                       int window, const int32_t* key_lens,
+                                       int32_t* first, int32_t* count, void* stream);
 
 /* Decode (Nq == 1) that allocates nothing.  The pages have no counterpart:
  * this entry point exists for callers that cannot call cudaMalloc -- code

@@ -12,6 +12,21 @@ TOL_O_MEAN = 2e-3
 TOL_LSE = 1e-3
 
 
+def rand_inputs(B, Hq, Hkv, Nq, Nk, d, seed, key_lens=None, std=1.0):
+    """Seeded bf16 q/k/v; keys at or beyond key_lens[b] hold a large finite
+    sentinel (they must get zero weight)."""
+    x = {"q": synth.normal_bf16((B, Hq, Nq, d), seed, std),
+         "k": synth.normal_bf16((B, Hkv, Nk, d), seed + 1, std),
+         "v": synth.normal_bf16((B, Hkv, Nk, d), seed + 2),
+         "key_lens": None if key_lens is None else np.asarray(key_lens, np.int32)}
+    if key_lens is not None:
+        sent = synth.bf16_bits_from_f32(np.array([synth.PAD_SENTINEL], np.float32))[0]
+        for b, L in enumerate(key_lens):
+            x["k"][b, :, L:] = sent
+            x["v"][b, :, L:] = sent
+    return x
+
+
 def to_dev(x, torch):
     """uint16 bf16 bits (numpy) -> CUDA bf16 tensor, bit-exact."""
     t = torch.from_numpy(np.ascontiguousarray(x).view(np.int16)).view(torch.bfloat16)
@@ -25,7 +40,7 @@ def from_dev(t):
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
 
 
-def run_gpu(inputs, causal, scale, rope=None):
+def run_gpu(inputs, causal, scale, rope=None, window=0):
     """Attention through the C ABI; returns (o float64 [B,Hq,Nq,d], lse float64)."""
     import torch
     import exact_scaled_dot_fwd_b200 as eb
@@ -37,7 +52,7 @@ def run_gpu(inputs, causal, scale, rope=None):
                           pairing=rope["pairing"])
         k = eb.rope_apply(k, base=rope["base"], pos_offset=rope.get("k_pos_offset", 0),
                           pairing=rope["pairing"])
-    o, lse = eb.attn_fwd(q, k, v, causal=causal, scale=scale, key_lens=kl_t)
+    o, lse = eb.attn_fwd(q, k, v, causal=causal, scale=scale, key_lens=kl_t, window=window)
     torch.cuda.synchronize()
     assert eb.device_status() == 0
     return from_dev(o), lse.cpu().numpy().astype(np.float64)
@@ -65,14 +80,14 @@ def compare(o_gpu_rows, lse_gpu_rows, o_ref, lse_ref, what=""):
     return res
 
 
-def check_workload(inputs, shape, causal, scale, rows=None, rope=None, what=""):
+def check_workload(inputs, shape, causal, scale, rows=None, rope=None, what="", window=0):
     """Run GPU + oracle on the same inputs; rows = flat row ids or None (all)."""
     B, Hq, Nq, d = shape
-    o, lse = run_gpu(inputs, causal, scale, rope=rope)
+    o, lse = run_gpu(inputs, causal, scale, rope=rope, window=window)
     o = o.reshape(-1, d)
     lse = lse.reshape(-1)
     o_ref, lse_ref = oracle.attn_rows(inputs["q"], inputs["k"], inputs["v"], causal, scale,
                                       key_lens=inputs.get("key_lens"), rows=rows,
-                                      rope_cfg=rope)
+                                      rope_cfg=rope, window=window)
     sel = slice(None) if rows is None else rows
     return compare(o[sel], lse[sel], o_ref, lse_ref, what)

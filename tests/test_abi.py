@@ -115,3 +115,19 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
     monkeypatch.setattr(eb, "_lib", None)
     with pytest.raises(OSError):
         eb.lib()
+
+
+def test_window_entry_points_reject_bad_arguments_on_host(L):
+    w = L.attn_fwd_window
+    # negative window
+    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, -1, 0.125, None, P, 256, None) == 1
+    # the checks shared with attn_fwd_ws come first
+    assert w(None, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, 16, 0.125, None, P, 256, None) == 1
+    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 96, 1, 16, 0.125, None, P, 256, None) == 2
+    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, 16, 0.125, None, None, 0, None) == 4
+    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, 16, 0.125, None,
+             ctypes.c_void_p(0x1010), 256, None) == 3
+    t = L.attn_fwd_tile_plan_window
+    assert t(1, 8, 8, 64, 1, -1, None, P, P, None) == 1
+    assert t(1, 8, 8, 64, 1, 16, None, None, P, None) == 1
+    assert t(1, 8, 8, 96, 1, 16, None, P, P, None) == 2

@@ -10,7 +10,7 @@ import pytest
 import oracle
 from exact_scaled_dot_fwd_b200 import synth
 
-from parity import check_workload, compare, from_dev, run_gpu, to_dev
+from parity import check_workload, compare, from_dev, rand_inputs, run_gpu, to_dev
 
 pytestmark = pytest.mark.gpu
 
@@ -21,19 +21,6 @@ def torch():
     from exact_scaled_dot_fwd_b200 import build
     build.build()
     return t
-
-
-def rand_inputs(B, Hq, Hkv, Nq, Nk, d, seed, key_lens=None, std=1.0):
-    x = {"q": synth.normal_bf16((B, Hq, Nq, d), seed, std),
-         "k": synth.normal_bf16((B, Hkv, Nk, d), seed + 1, std),
-         "v": synth.normal_bf16((B, Hkv, Nk, d), seed + 2),
-         "key_lens": None if key_lens is None else np.asarray(key_lens, np.int32)}
-    if key_lens is not None:
-        sent = synth.bf16_bits_from_f32(np.array([synth.PAD_SENTINEL], np.float32))[0]
-        for b, L in enumerate(key_lens):
-            x["k"][b, :, L:] = sent
-            x["v"][b, :, L:] = sent
-    return x
 
 
 # ------------------------------------------------------ named workloads -----
