@@ -34,11 +34,12 @@ def lib():
         L.oracle_rope.restype = None
         L.oracle_visible_prefix.argtypes = [i64, i64, i64, i32, i64]
         L.oracle_visible_prefix.restype = i64
-        L.oracle_attn_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, i64, f64,
-                                       vp, i32, f64, i32, i32, i64, i64, vp, i64, vp, vp, i32]
+        L.oracle_attn_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32, i64, i32,
+                                       f64, vp, i32, f64, i32, i32, i64, i64, vp, i64, vp, vp,
+                                       i32]
         L.oracle_attn_rows.restype = i32
         L.oracle_attn_online_rows.argtypes = [vp, vp, vp, i64, i64, i64, i64, i64, i64, i32,
-                                              i64, f64, vp, i64, vp, i64, vp, vp, i32]
+                                              i64, i32, f64, vp, i64, vp, i64, vp, vp, i32]
         L.oracle_attn_online_rows.restype = i32
         L.oracle_kv_tiles.argtypes = [i64, i64, i32, i64, i64, i64, i64, vp, vp, vp]
         L.oracle_kv_tiles.restype = None
@@ -46,6 +47,13 @@ def lib():
         L.oracle_kv_tiles_window.restype = None
         L.oracle_visible_range.argtypes = [i64, i64, i64, i32, i64, i64, vp, vp]
         L.oracle_visible_range.restype = None
+        L.oracle_visible_range_ex.argtypes = [i64, i64, i64, i32, i64, i64, i32, vp, vp]
+        L.oracle_visible_range_ex.restype = None
+        L.oracle_query_position.argtypes = [i64, i64, i64, i64, i32]
+        L.oracle_query_position.restype = i64
+        L.oracle_kv_tiles_ex.argtypes = [i64, i64, i32, i64, i64, i32, i64, i64, i64, vp, vp,
+                                         vp]
+        L.oracle_kv_tiles_ex.restype = None
         _lib = L
     return _lib
 
@@ -86,17 +94,29 @@ def visible_prefix(i, Nq, Nk, causal, key_len) -> int:
     return int(lib().oracle_visible_prefix(i, Nq, Nk, int(bool(causal)), key_len))
 
 
-def kv_tiles(Nq, Nk, causal, key_len, Br, Bc, qt, window=0):
+def kv_tiles(Nq, Nk, causal, key_len, Br, Bc, qt, window=0, align=0):
     f, l, c = ctypes.c_int64(), ctypes.c_int64(), ctypes.c_int64()
-    lib().oracle_kv_tiles_window(Nq, Nk, int(bool(causal)), key_len, window, Br, Bc, qt,
-                                 ctypes.byref(f), ctypes.byref(l), ctypes.byref(c))
+    if align:
+        lib().oracle_kv_tiles_ex(Nq, Nk, int(bool(causal)), key_len, window, int(align), Br, Bc,
+                                 qt, ctypes.byref(f), ctypes.byref(l), ctypes.byref(c))
+    else:
+        lib().oracle_kv_tiles_window(Nq, Nk, int(bool(causal)), key_len, window, Br, Bc, qt,
+                                     ctypes.byref(f), ctypes.byref(l), ctypes.byref(c))
     return f.value, l.value, c.value
 
 
-def visible_range(i, Nq, Nk, causal, key_len, window=0):
+def query_position(i, Nq, Nk, key_len, align=0) -> int:
+    return int(lib().oracle_query_position(i, Nq, Nk, key_len, int(align)))
+
+
+def visible_range(i, Nq, Nk, causal, key_len, window=0, align=0):
     lo, hi = ctypes.c_int64(), ctypes.c_int64()
-    lib().oracle_visible_range(i, Nq, Nk, int(bool(causal)), key_len, window,
-                               ctypes.byref(lo), ctypes.byref(hi))
+    if align:
+        lib().oracle_visible_range_ex(i, Nq, Nk, int(bool(causal)), key_len, window, int(align),
+                                      ctypes.byref(lo), ctypes.byref(hi))
+    else:
+        lib().oracle_visible_range(i, Nq, Nk, int(bool(causal)), key_len, window,
+                                   ctypes.byref(lo), ctypes.byref(hi))
     return lo.value, hi.value
 
 
@@ -113,13 +133,15 @@ def _prep(q, k, v, key_lens, rows):
 
 
 def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
-              nthreads=None, window=0):
+              nthreads=None, window=0, align=0):
     """Naive fp64 attention for the listed flat rows (all rows if None).
 
     q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] as bf16 bit patterns.  rope_cfg: None or
     dict(base=, pairing=, q_pos_offset=, k_pos_offset=, round_bf16=) -- round_bf16
     rounds the rotated rows to bf16 (a RoPE pass with bf16 output feeding the
-    attention).  Returns (o [n,d], lse [n]).
+    attention).  window: sliding window (0 = none).  align: 0 puts query row i
+    at key position i + Nk - Nq, 1 at i + key_lens[b] - Nq.
+    Returns (o [n,d], lse [n]).
     """
     q, k, v, kl, r, (B, Hq, Hkv, Nq, Nk, d), nrows = _prep(q, k, v, key_lens, rows)
     o = np.empty((nrows, d), np.float64)
@@ -127,7 +149,8 @@ def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
     rc = rope_cfg or {}
     st = lib().oracle_attn_rows(
         _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), int(window),
-        float(scale), _ptr(kl), int(rope_cfg is not None), float(rc.get("base", 10000.0)),
+        int(align), float(scale), _ptr(kl), int(rope_cfg is not None),
+        float(rc.get("base", 10000.0)),
         int(rc.get("pairing", 0)), int(bool(rc.get("round_bf16", False))),
         int(rc.get("q_pos_offset", 0)), int(rc.get("k_pos_offset", 0)),
         _ptr(r), nrows, _ptr(o), _ptr(lse), int(nthreads or default_threads()))
@@ -137,14 +160,14 @@ def attn_rows(q, k, v, causal, scale, key_lens=None, rows=None, rope_cfg=None,
 
 
 def attn_online_rows(q, k, v, causal, scale, block, key_lens=None, rows=None, nthreads=None,
-                     window=0):
+                     window=0, align=0):
     """Online-recurrence fp64 attention over key blocks of size `block`."""
     q, k, v, kl, r, (B, Hq, Hkv, Nq, Nk, d), nrows = _prep(q, k, v, key_lens, rows)
     o = np.empty((nrows, d), np.float64)
     lse = np.empty(nrows, np.float64)
     st = lib().oracle_attn_online_rows(
         _ptr(q), _ptr(k), _ptr(v), B, Hq, Hkv, Nq, Nk, d, int(bool(causal)), int(window),
-        float(scale), _ptr(kl), int(block), _ptr(r), nrows, _ptr(o), _ptr(lse),
+        int(align), float(scale), _ptr(kl), int(block), _ptr(r), nrows, _ptr(o), _ptr(lse),
         int(nthreads or default_threads()))
     if st != 0:
         raise ValueError("oracle_attn_online_rows rejected its arguments")

@@ -95,15 +95,27 @@ int64_t oracle_visible_prefix(int64_t i, int64_t Nq, int64_t Nk, int causal,
   return L < 0 ? 0 : L;
 }
 
+/* Key position of query row i.  align 0: the Nq rows are the last Nq
+ * positions of the Nk keys, p = i + (Nk - Nq).  align 1: they are the last
+ * Nq positions of the sequence's own L = key_len keys, p = i + (L - Nq)
+ * ([CIA] self-test 5: t new tokens after a cache of `len` keys see the
+ * cache and a lower triangle among themselves, per sequence). */
+int64_t oracle_query_position(int64_t i, int64_t Nq, int64_t Nk,
+                              int64_t key_len, int align) {
+  const int64_t L = key_len < 0 ? 0 : (key_len > Nk ? Nk : key_len);
+  return i + ((align ? L : Nk) - Nq);
+}
+
 /* [AME] 11: with a window w > 0, key j is legal only if |p - j| < w, where
- * p = i + (Nk - Nq) is the query's key position (the causal alignment). */
-void oracle_visible_range(int64_t i, int64_t Nq, int64_t Nk, int causal,
-                          int64_t key_len, int64_t window, int64_t* lo,
-                          int64_t* hi) {
-  int64_t h = oracle_visible_prefix(i, Nq, Nk, causal, key_len);
-  int64_t l = 0;
+ * p is the query's key position; causal adds j <= p; key_len adds j < L. */
+void oracle_visible_range_ex(int64_t i, int64_t Nq, int64_t Nk, int causal,
+                             int64_t key_len, int64_t window, int align,
+                             int64_t* lo, int64_t* hi) {
+  const int64_t L = key_len < 0 ? 0 : (key_len > Nk ? Nk : key_len);
+  const int64_t p = oracle_query_position(i, Nq, Nk, key_len, align);
+  int64_t h = L, l = 0;
+  if (causal && p + 1 < h) h = p + 1;
   if (window > 0) {
-    const int64_t p = i + (Nk - Nq);
     if (p - window + 1 > l) l = p - window + 1;
     if (p + window < h) h = p + window;
   }
@@ -112,17 +124,31 @@ void oracle_visible_range(int64_t i, int64_t Nq, int64_t Nk, int causal,
   *hi = h;
 }
 
+void oracle_visible_range(int64_t i, int64_t Nq, int64_t Nk, int causal,
+                          int64_t key_len, int64_t window, int64_t* lo,
+                          int64_t* hi) {
+  oracle_visible_range_ex(i, Nq, Nk, causal, key_len, window, 0, lo, hi);
+}
+
 void oracle_kv_tiles(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
                      int64_t Br, int64_t Bc, int64_t qt, int64_t* first,
                      int64_t* last, int64_t* count) {
-  oracle_kv_tiles_window(Nq, Nk, causal, key_len, 0, Br, Bc, qt, first, last,
-                         count);
+  oracle_kv_tiles_ex(Nq, Nk, causal, key_len, 0, 0, Br, Bc, qt, first, last,
+                     count);
 }
 
 void oracle_kv_tiles_window(int64_t Nq, int64_t Nk, int causal,
                             int64_t key_len, int64_t window, int64_t Br,
                             int64_t Bc, int64_t qt, int64_t* first,
                             int64_t* last, int64_t* count) {
+  oracle_kv_tiles_ex(Nq, Nk, causal, key_len, window, 0, Br, Bc, qt, first,
+                     last, count);
+}
+
+void oracle_kv_tiles_ex(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
+                        int64_t window, int align, int64_t Br, int64_t Bc,
+                        int64_t qt, int64_t* first, int64_t* last,
+                        int64_t* count) {
   *first = -1; *last = -1; *count = 0;
   const int64_t i0 = qt * Br, i1 = (qt + 1) * Br < Nq ? (qt + 1) * Br : Nq;
   const int64_t ntiles = (Nk + Bc - 1) / Bc;
@@ -131,7 +157,8 @@ void oracle_kv_tiles_window(int64_t Nq, int64_t Nk, int causal,
     int touched = 0;
     for (int64_t i = i0; i < i1 && !touched; ++i) {
       int64_t lo, hi;
-      oracle_visible_range(i, Nq, Nk, causal, key_len, window, &lo, &hi);
+      oracle_visible_range_ex(i, Nq, Nk, causal, key_len, window, align, &lo,
+                              &hi);
       for (int64_t j = j0; j < j1; ++j)
         if (j >= lo && j < hi) { touched = 1; break; }
     }
@@ -150,6 +177,7 @@ typedef struct {
   int64_t B, Hq, Hkv, Nq, Nk, d;
   int causal;
   int64_t window; /* > 0: sliding window ([AME] 11) */
+  int align;      /* query positions: 0 end of Nk, 1 end of key_lens[b] */
   double scale;
   const int32_t* key_lens;
   int rope;
@@ -207,8 +235,8 @@ static void row_naive(job_t* J, int64_t r, double* qrow, double* krow,
   const int64_t g = h / (J->Hq / J->Hkv); /* query head -> kv head ([AME] 9) */
   const int64_t key_len = J->key_lens ? J->key_lens[b] : J->Nk;
   int64_t lo, hi;
-  oracle_visible_range(i, J->Nq, J->Nk, J->causal, key_len, J->window, &lo,
-                       &hi);
+  oracle_visible_range_ex(i, J->Nq, J->Nk, J->causal, key_len, J->window,
+                          J->align, &lo, &hi);
   const int64_t n = hi - lo;
   for (int64_t c = 0; c < d; ++c) out[c] = 0.0;
   if (n == 0) { *lse_out = -INFINITY; return; }
@@ -244,8 +272,8 @@ static void row_online(job_t* J, int64_t r, double* qrow, double* krow,
   const int64_t g = h / (J->Hq / J->Hkv);
   const int64_t key_len = J->key_lens ? J->key_lens[b] : J->Nk;
   int64_t lo, hi;
-  oracle_visible_range(i, J->Nq, J->Nk, J->causal, key_len, J->window, &lo,
-                       &hi);
+  oracle_visible_range_ex(i, J->Nq, J->Nk, J->causal, key_len, J->window,
+                          J->align, &lo, &hi);
   const int64_t n = hi - lo;
   const uint16_t* qsrc = J->q + r * d;
   for (int64_t c = 0; c < d; ++c) qrow[c] = bf16_bits_to_double(qsrc[c]);
@@ -353,7 +381,7 @@ static int run_rows(job_t* proto, int nthreads) {
 int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                      int64_t Nk, int64_t d, int causal, int64_t window,
-                     double scale,
+                     int align, double scale,
                      const int32_t* key_lens, int rope, double rope_base,
                      int rope_pairing, int rope_round, int64_t q_pos_offset,
                      int64_t k_pos_offset, const int64_t* rows, int64_t nrows,
@@ -362,7 +390,7 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v;
   J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d;
-  J.causal = causal; J.window = window; J.scale = scale;
+  J.causal = causal; J.window = window; J.align = align; J.scale = scale;
   J.key_lens = key_lens;
   J.rope = rope; J.rope_base = rope_base; J.rope_pairing = rope_pairing;
   J.rope_round = rope_round;
@@ -374,8 +402,8 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 int oracle_attn_online_rows(const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, int64_t B, int64_t Hq,
                             int64_t Hkv, int64_t Nq, int64_t Nk, int64_t d,
-                            int causal, int64_t window, double scale,
-                            const int32_t* key_lens,
+                            int causal, int64_t window, int align,
+                            double scale, const int32_t* key_lens,
                             int64_t block, const int64_t* rows, int64_t nrows,
                             double* o, double* lse, int nthreads) {
   if (block <= 0) return -1;
@@ -383,7 +411,7 @@ int oracle_attn_online_rows(const uint16_t* q, const uint16_t* k,
   memset(&J, 0, sizeof J);
   J.q = q; J.k = k; J.v = v;
   J.B = B; J.Hq = Hq; J.Hkv = Hkv; J.Nq = Nq; J.Nk = Nk; J.d = d;
-  J.causal = causal; J.window = window; J.scale = scale;
+  J.causal = causal; J.window = window; J.align = align; J.scale = scale;
   J.key_lens = key_lens;
   J.block = block; J.rows = rows; J.nrows = nrows; J.o = o; J.lse = lse;
   return run_rows(&J, nthreads);

@@ -52,16 +52,29 @@ void oracle_rope(const uint16_t* x, double* out, int64_t B, int64_t H,
 int64_t oracle_visible_prefix(int64_t i, int64_t Nq, int64_t Nk, int causal,
                               int64_t key_len);
 
-/* Visible keys of query row i as a range [lo, hi): the prefix above, cut by
- * a sliding window when window > 0 ([AME] 11: |p - j| < w, p = i + Nk - Nq,
- * the query's key position under the causal alignment). */
+/* Key position p of query row i.  align 0: p = i + (Nk - Nq) (the Nq rows
+ * end at key Nk - 1).  align 1: p = i + (L - Nq), L = key_len clamped to
+ * [0, Nk] (the rows are the newest Nq tokens of each sequence, [CIA]
+ * self-test 5). */
+int64_t oracle_query_position(int64_t i, int64_t Nq, int64_t Nk,
+                              int64_t key_len, int align);
+
+/* Visible keys of query row i as a range [lo, hi) (hi == lo: none):
+ * j < L; causal adds j <= p; a sliding window w > 0 adds |p - j| < w
+ * ([AME] 11); p from oracle_query_position. */
+void oracle_visible_range_ex(int64_t i, int64_t Nq, int64_t Nk, int causal,
+                             int64_t key_len, int64_t window, int align,
+                             int64_t* lo, int64_t* hi);
+
+/* oracle_visible_range_ex with align 0. */
 void oracle_visible_range(int64_t i, int64_t Nq, int64_t Nk, int causal,
                           int64_t key_len, int64_t window, int64_t* lo,
                           int64_t* hi);
 
 /* Definition of the result ([AME] 3, 5, 9; [CIA] 3.2, 3.4):
  *   g = h / (Hq / Hkv);  s_j = scale * <q_i, k_j> for visible j (the range
- *   of oracle_visible_range; window <= 0 means no window);
+ *   of oracle_visible_range_ex; window <= 0 means no window, align picks
+ *   the query positions);
  *   m = max s; p_j = exp(s_j - m); l = sum p; O_i = sum p_j v_j / l;
  *   lse_i = m + log(l).  No visible key: O_i = 0, lse_i = -inf.
  * Layout: q [B,Hq,Nq,d], k/v [B,Hkv,Nk,d] row-major bf16 bits.
@@ -76,7 +89,7 @@ void oracle_visible_range(int64_t i, int64_t Nq, int64_t Nk, int causal,
 int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
                      int64_t B, int64_t Hq, int64_t Hkv, int64_t Nq,
                      int64_t Nk, int64_t d, int causal, int64_t window,
-                     double scale, const int32_t* key_lens, int rope,
+                     int align, double scale, const int32_t* key_lens, int rope,
                      double rope_base,
                      int rope_pairing, int rope_round, int64_t q_pos_offset,
                      int64_t k_pos_offset, const int64_t* rows, int64_t nrows,
@@ -89,8 +102,9 @@ int oracle_attn_rows(const uint16_t* q, const uint16_t* k, const uint16_t* v,
 int oracle_attn_online_rows(const uint16_t* q, const uint16_t* k,
                             const uint16_t* v, int64_t B, int64_t Hq,
                             int64_t Hkv, int64_t Nq, int64_t Nk, int64_t d,
-                            int causal, int64_t window, double scale,
-                            const int32_t* key_lens, int64_t block, const int64_t* rows, int64_t nrows,
+                            int causal, int64_t window, int align,
+                            double scale, const int32_t* key_lens,
+                            int64_t block, const int64_t* rows, int64_t nrows,
                             double* o, double* lse, int nthreads);
 
 /* Which KV tiles a query tile touches, by brute force over the visibility
@@ -107,6 +121,13 @@ void oracle_kv_tiles_window(int64_t Nq, int64_t Nk, int causal,
                             int64_t key_len, int64_t window, int64_t Br,
                             int64_t Bc, int64_t qt, int64_t* first,
                             int64_t* last, int64_t* count);
+
+/* Same with a sliding window and a query alignment (see
+ * oracle_query_position). */
+void oracle_kv_tiles_ex(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
+                        int64_t window, int align, int64_t Br, int64_t Bc,
+                        int64_t qt, int64_t* first, int64_t* last,
+                        int64_t* count);
 
 #ifdef __cplusplus
 }

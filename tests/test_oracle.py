@@ -516,3 +516,75 @@ def test_window_tile_sets_closed_forms():
     # a window of one key: each row sees only itself
     for i in (0, 5, 127, 128):
         assert oracle.visible_range(i, 256, 256, True, 256, 1) == (i, i + 1)
+
+
+# ------------------------------------------- multi-token decode alignment ----
+
+def multi_token_mask(lens, t, Nk):
+    """The pages' speculative-decode mask ('Coding interview (14)', self-test
+    5), per sequence: t new tokens after a cache of len keys see the whole
+    cache and a lower triangle among themselves, [ones(t, len) | tril(t, t)];
+    the row is padded with invisible columns up to Nk."""
+    rows = []
+    for n in lens:
+        m = np.concatenate([np.ones((t, n), bool), np.tril(np.ones((t, t), bool))], axis=1)
+        rows.append(np.concatenate([m, np.zeros((t, Nk - n - t), bool)], axis=1))
+    return np.stack(rows)[:, None]          # [B, 1, t, Nk]
+
+
+@pytest.mark.parametrize("t", [1, 2, 4, 7])
+def test_multi_token_decode_matches_page_mask(t):
+    """align = 1 places each sequence's t query rows at the end of its own
+    key_lens[b] keys (cache + new tokens)."""
+    B, Hq, Hkv, d, Nk = 4, 4, 2, 16, 40
+    lens = [0, 5, 20, Nk - t]               # cache lengths before the new tokens
+    key_lens = np.array([n + t for n in lens], np.int32)
+    q = synth.normal_bf16((B, Hq, t, d), 301)
+    k = synth.normal_bf16((B, Hkv, Nk, d), 302)
+    v = synth.normal_bf16((B, Hkv, Nk, d), 303)
+    o, lse = oracle.attn_rows(q, k, v, True, 0.25, key_lens=key_lens, align=1)
+    m = torch.from_numpy(multi_token_mask(lens, t, Nk))
+    kr = f64(k).repeat_interleave(Hq // Hkv, dim=1)
+    vr = f64(v).repeat_interleave(Hq // Hkv, dim=1)
+    O = F.scaled_dot_product_attention(f64(q), kr, vr, attn_mask=m, scale=0.25)
+    S = (torch.matmul(f64(q), kr.transpose(-1, -2)) * 0.25).masked_fill(~m, -math.inf)
+    L = scipy.special.logsumexp(S.numpy(), axis=-1).reshape(-1)
+    assert np.max(np.abs(o - O.numpy().reshape(-1, d))) < 1e-13
+    assert np.max(np.abs(lse - L)) < 1e-12
+    # the online recurrence agrees under the same alignment
+    o2, l2 = oracle.attn_online_rows(q, k, v, True, 0.25, 3, key_lens=key_lens, align=1)
+    assert np.max(np.abs(o - o2)) < 1e-13 and np.max(np.abs(lse - l2)) < 1e-13
+
+
+def test_alignment_special_cases():
+    B, H, Nq, Nk, d = 2, 2, 6, 30, 8
+    q = synth.normal_bf16((B, H, Nq, d), 311)
+    k = synth.normal_bf16((B, H, Nk, d), 312)
+    v = synth.normal_bf16((B, H, Nk, d), 313)
+    # full-length sequences: both alignments put the rows at the end of Nk
+    full = np.array([Nk, Nk], np.int32)
+    a0 = oracle.attn_rows(q, k, v, True, 0.3, key_lens=full)
+    a1 = oracle.attn_rows(q, k, v, True, 0.3, key_lens=full, align=1)
+    assert np.array_equal(a0[0], a1[0]) and np.array_equal(a0[1], a1[1])
+    # one new token: causal changes nothing, it sees its whole sequence
+    q1 = q[:, :, :1]
+    kl = np.array([17, 30], np.int32)
+    c1 = oracle.attn_rows(q1, k, v, True, 0.3, key_lens=kl, align=1)
+    c0 = oracle.attn_rows(q1, k, v, False, 0.3, key_lens=kl, align=1)
+    assert np.array_equal(c1[0], c0[0]) and np.array_equal(c1[1], c0[1])
+    # closed forms: row i of a sequence of L keys sees L - Nq + i + 1 keys
+    # (causal), and its window ends at its own position
+    for L in (6, 9, 30):
+        for i in range(Nq):
+            assert oracle.query_position(i, Nq, Nk, L, 1) == L - Nq + i
+            assert oracle.visible_range(i, Nq, Nk, True, L, 0, 1) == (0, L - Nq + i + 1)
+            p = L - Nq + i
+            assert oracle.visible_range(i, Nq, Nk, True, L, 4, 1) == (max(0, p - 3), p + 1)
+    # fewer keys than query rows: the leading rows see nothing when causal
+    assert oracle.visible_range(0, Nq, Nk, True, 3, 0, 1) == (0, 0)
+    assert oracle.visible_range(Nq - 1, Nq, Nk, True, 3, 0, 1) == (0, 3)
+    # decode under a window over a ragged cache reads its last w keys
+    assert oracle.visible_range(0, 1, 1000, False, 700, 64, 1) == (636, 700)
+    # tile sets follow each sequence's own length
+    assert oracle.kv_tiles(8, 4096, True, 1000, 128, 128, 0, align=1) == (0, 7, 8)
+    assert oracle.kv_tiles(8, 4096, True, 1000, 128, 128, 0, window=300, align=1) == (5, 7, 3)
