@@ -186,7 +186,7 @@ def oracle_sample(w, seconds, seed=12345, rows_per_batch=None):
             i = int(r % w.Nq)
             b = int(r // (w.Nq * w.Hq))
             L = w.Nk if kl is None else int(kl[b])
-            lo, hi = oracle.visible_range(i, w.Nq, w.Nk, w.causal, L, w.window)
+            lo, hi = oracle.visible_range(i, w.Nq, w.Nk, w.causal, L, w.window, w.align)
             f += 4.0 * w.d * (hi - lo)
         return f
 
@@ -198,7 +198,7 @@ def oracle_sample(w, seconds, seed=12345, rows_per_batch=None):
         rows = np.sort(rng.integers(0, total_rows, size=n)).astype(np.int64)
         t0 = time.perf_counter()
         oracle.attn_rows(x["q"], x["k"], x["v"], w.causal, w.scale, key_lens=kl, rows=rows,
-                         rope_cfg=rope, nthreads=threads, window=w.window)
+                         rope_cfg=rope, nthreads=threads, window=w.window, align=w.align)
         dt = time.perf_counter() - t0
         used_f += flops(rows)
         used_t += dt
@@ -214,9 +214,19 @@ def to_dev(bits, torch, device):
     return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).to(device)
 
 
+def memory_bound(w):
+    """Decode-shaped workloads (at most 64 query rows per kv head) are judged
+    on HBM bytes; the rest on tensor FLOPs."""
+    return w.Nq * (w.Hq // w.Hkv) <= 64
+
+
 def decode_bytes(w, key_lens):
-    kv = float(np.clip(key_lens, 0, w.Nk).sum()) * w.Hkv * w.d * 2 * 2
-    return kv + w.B * w.Hq * w.d * 2 * 2 + w.B * w.Hq * 4
+    """Algorithmic bytes of a decode step: K and V of every valid key once
+    per kv head, plus Q, O (bf16) and lse (fp32).  No window here."""
+    assert w.window == 0
+    kl = np.full(w.B, w.Nk) if key_lens is None else np.clip(key_lens, 0, w.Nk)
+    kv = float(kl.sum()) * w.Hkv * w.d * 2 * 2
+    return kv + w.B * w.Hq * w.Nq * (w.d * 2 * 2 + 4)
 
 
 def time_steps(fn, steps, torch, dist, stream):
@@ -294,7 +304,7 @@ def run_ours(args):
         c = i % copies
         q, k = (QR, KR) if w.rope else (Q[c], K[c])
         eb.attn_fwd_ws(q, k, V[c], ws, causal=w.causal, scale=w.scale, key_lens=kl,
-                       out=O, lse=LSE, window=w.window)
+                       out=O, lse=LSE, window=w.window, align=w.align)
 
     def step(i):
         # one pass of the whole path: the RoPE prologue (when the workload has
@@ -320,10 +330,10 @@ def run_ours(args):
     # this library's kernels per step: decode = split + combine; prefill = the
     # attention kernel (its counter reset is a runtime memset, not a kernel
     # of ours); plus the two RoPE launches when the workload has RoPE
-    launches_per_step = (2 if w.Nq == 1 else 1) + (2 if w.rope else 0)
+    launches_per_step = (2 if memory_bound(w) else 1) + (2 if w.rope else 0)
     # the dominant kernel alone (differs from the step only when RoPE runs)
     ms_kernel = ms if not w.rope else time_steps(attn_only, steps, torch, dist, stream)
-    if w.Nq == 1:
+    if memory_bound(w):
         unit, work = "GB/s", decode_bytes(w, x["key_lens"])
         value = world * work * steps / (ms / 1e3) / 1e9
         kval = work * steps / (ms_kernel / 1e3) / 1e9
@@ -344,7 +354,7 @@ def run_ours(args):
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
                    "Nk": w.Nk, "d": w.d, "causal": w.causal, "rope": w.rope,
                    "key_lens": list(w.key_lens) if w.key_lens else None,
-                   "window": w.window,
+                   "window": w.window, "align": w.align,
                    "l2": f"{copies} rotating input copies ({copies * per_copy / 1e6:.0f} MB > "
                          f"126 MB L2)",
                    "parallelism": f"replicas x{world} (independent batch per GPU)"},
@@ -380,8 +390,10 @@ def run_ours(args):
                        "d2h_bytes_per_step": d2h, "steps": e_steps}
 
     # ---- decode workload (HBM-bound half of the metric), same run
-    if not args.no_decode and w.Nq != 1 and rank == 0 and world == 1:
+    if not args.no_decode and not memory_bound(w) and rank == 0 and world == 1:
         line["decode"] = run_decode(torch, eb, device, stream, peaks, peak_src)
+        line["multi_token_decode"] = run_decode(torch, eb, device, stream, peaks, peak_src,
+                                                name="spec_decode")
     # ---- sliding-window prefill, same run
     if not args.no_window and w.name != "long_window" and rank == 0 and world == 1:
         line["window"] = run_window(torch, eb, device, stream, peaks, peak_src)
@@ -407,8 +419,8 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None):
-    w = synth.WORKLOADS["mqa_decode"]
+def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa_decode"):
+    w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
     per_copy = x["k"].nbytes + x["v"].nbytes
     copies = 2
@@ -417,13 +429,13 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None):
     V = [to_dev(x["v"], torch, device) for _ in range(copies)]
     kl = torch.from_numpy(x["key_lens"]).to(device)
     O = torch.empty_like(Q)
-    LSE = torch.empty((w.B, w.Hq, 1), dtype=torch.float32, device=device)
-    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, 1, w.Nk, w.d), dtype=torch.uint8,
-                     device=device)
+    LSE = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
+    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d),
+                     dtype=torch.uint8, device=device)
 
     def step(i):
-        eb.attn_fwd_ws(Q, K[i % copies], V[i % copies], ws, scale=w.scale, key_lens=kl, out=O,
-                       lse=LSE)
+        eb.attn_fwd_ws(Q, K[i % copies], V[i % copies], ws, causal=w.causal, scale=w.scale,
+                       key_lens=kl, out=O, lse=LSE, window=w.window, align=w.align)
 
     for i in range(5):
         step(i)
@@ -494,7 +506,7 @@ def run_reference(args):
 
     def one(rows):
         oracle.attn_rows(x["q"], x["k"], x["v"], w.causal, w.scale, key_lens=kl, rows=rows,
-                         rope_cfg=rope, nthreads=threads, window=w.window)
+                         rope_cfg=rope, nthreads=threads, window=w.window, align=w.align)
 
     def flops(rows):
         f = 0.0
@@ -502,7 +514,7 @@ def run_reference(args):
             i = int(r % w.Nq)
             b = int(r // (w.Nq * w.Hq))
             L = w.Nk if kl is None else int(kl[b])
-            lo, hi = oracle.visible_range(i, w.Nq, w.Nk, w.causal, L, w.window)
+            lo, hi = oracle.visible_range(i, w.Nq, w.Nk, w.causal, L, w.window, w.align)
             f += 4.0 * w.d * (hi - lo)
         return f
 
@@ -516,7 +528,7 @@ def run_reference(args):
         one(rows)
         t_total += time.perf_counter() - t0
         f_total += flops(rows)
-    if w.Nq == 1:
+    if memory_bound(w):
         unit = "GB/s"
         value = (f_total / (4.0 * w.d)) * w.d * 4 / t_total / 1e9
     else:
@@ -528,7 +540,8 @@ def run_reference(args):
             "ms_per_step": 1e3 * t_total / steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
-                       "Nk": w.Nk, "d": w.d, "causal": w.causal, "window": w.window},
+                       "Nk": w.Nk, "d": w.d, "causal": w.causal, "window": w.window,
+                       "align": w.align},
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                              "sample": sample},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,

@@ -48,6 +48,8 @@ def lib():
         L.attn_fwd_window.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, f, vp, vp, sz,
                                       vp]
         L.attn_fwd_window.restype = i
+        L.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp, vp, sz, vp]
+        L.attn_fwd_ex.restype = i
         L.attn_workspace_size.argtypes = [i, i, i, i, i, i]
         L.attn_workspace_size.restype = sz
         L.rope_apply.argtypes = [vp, vp, i, i, i, i, f, i, i, vp]
@@ -58,6 +60,8 @@ def lib():
         L.attn_fwd_tile_plan.restype = i
         L.attn_fwd_tile_plan_window.argtypes = [i, i, i, i, i, i, vp, vp, vp, vp]
         L.attn_fwd_tile_plan_window.restype = i
+        L.attn_fwd_tile_plan_ex.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp]
+        L.attn_fwd_tile_plan_ex.restype = i
         L.attn_device_status.argtypes = [vp, i]
         L.attn_device_status.restype = i
         L.attn_strerror.argtypes = [i]
@@ -118,22 +122,25 @@ def _shapes(q, k, v):
 
 
 def attn_fwd(q, k, v, causal=False, scale=None, key_lens=None, out=None, lse=None,
-             return_lse=True, stream=None, window=0):
+             return_lse=True, stream=None, window=0, align=0):
     """O = softmax(Q K^T * scale + M) V on the GPU.
 
     q: bf16 [B, Hq, Nq, d]; k, v: bf16 [B, Hkv, Nk, d]; key_lens: int32 [B]
-    (device) or None; window: sliding window in keys (0 = none).  Returns
-    (o, lse) (lse fp32 [B, Hq, Nq], natural log) or o alone when return_lse is
-    False.  Without a window the library's own workspace is used; with one, a
-    workspace tensor is allocated here and passed to attn_fwd_window.
+    (device) or None; window: sliding window in keys (0 = none); align: 0
+    puts query row i at key position i + Nk - Nq, 1 at i + key_lens[b] - Nq
+    (multi-token decode over ragged caches).  Returns (o, lse) (lse fp32
+    [B, Hq, Nq], natural log) or o alone when return_lse is False.  Plain
+    calls use the library's own workspace; with a window or align = 1 a
+    workspace tensor is allocated here and passed to attn_fwd_ex.
     """
-    if window:
+    if window or align:
         B, Hq, Hkv, Nq, Nk, d = _shapes(q, k, v)
         torch = _torch()
         ws = torch.empty(max(attn_workspace_size(B, Hq, Hkv, Nq, Nk, d), 256),
                          dtype=torch.uint8, device=q.device)
         return attn_fwd_ws(q, k, v, ws, causal=causal, scale=scale, key_lens=key_lens, out=out,
-                           lse=lse, return_lse=return_lse, stream=stream, window=window)
+                           lse=lse, return_lse=return_lse, stream=stream, window=window,
+                           align=align)
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_tensor(t, n, torch.bfloat16, 4)
@@ -158,9 +165,9 @@ def attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) -> int:
 
 
 def attn_fwd_ws(q, k, v, workspace, causal=False, scale=None, key_lens=None, out=None,
-                lse=None, return_lse=True, stream=None, window=0):
-    """attn_fwd with a caller-owned workspace (uint8 CUDA tensor); window > 0
-    calls attn_fwd_window."""
+                lse=None, return_lse=True, stream=None, window=0, align=0):
+    """attn_fwd with a caller-owned workspace (uint8 CUDA tensor); a window or
+    align = 1 calls attn_fwd_ex."""
     torch = _torch()
     for t, n in ((q, "q"), (k, "k"), (v, "v")):
         _check_tensor(t, n, torch.bfloat16, 4)
@@ -174,12 +181,12 @@ def attn_fwd_ws(q, k, v, workspace, causal=False, scale=None, key_lens=None, out
     if return_lse and lse is None:
         lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
     ws_bytes = 0 if workspace is None else workspace.numel() * workspace.element_size()
-    if window:
-        rc = lib().attn_fwd_window(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
-                                   _ptr(lse if return_lse else None), B, Hq, Hkv, Nq, Nk, d,
-                                   int(bool(causal)), int(window), float(scale), _ptr(key_lens),
-                                   _ptr(workspace), ws_bytes, _stream(stream))
-        _raise(rc, "attn_fwd_window")
+    if window or align:
+        rc = lib().attn_fwd_ex(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
+                               _ptr(lse if return_lse else None), B, Hq, Hkv, Nq, Nk, d,
+                               int(bool(causal)), int(window), int(align), float(scale),
+                               _ptr(key_lens), _ptr(workspace), ws_bytes, _stream(stream))
+        _raise(rc, "attn_fwd_ex")
     else:
         rc = lib().attn_fwd_ws(_ptr(q), _ptr(k), _ptr(v), _ptr(out),
                                _ptr(lse if return_lse else None), B, Hq, Hkv, Nq, Nk, d,
@@ -235,7 +242,8 @@ def prefill_tile_shape(d):
     return br.value, bc.value
 
 
-def tile_plan(B, Nq, Nk, d, causal, key_lens=None, device="cuda", stream=None, window=0):
+def tile_plan(B, Nq, Nk, d, causal, key_lens=None, device="cuda", stream=None, window=0,
+              align=0):
     """(first, count) int32 [B, nqt] tensors: the KV tiles the prefill kernel
     visits for each (b, query tile), optionally under a sliding window."""
     torch = _torch()
@@ -243,10 +251,9 @@ def tile_plan(B, Nq, Nk, d, causal, key_lens=None, device="cuda", stream=None, w
     nqt = -(-Nq // br)
     first = torch.empty((B, nqt), dtype=torch.int32, device=device)
     count = torch.empty((B, nqt), dtype=torch.int32, device=device)
-    rc = lib().attn_fwd_tile_plan_window(B, Nq, Nk, d, int(bool(causal)), int(window),
-                                         _ptr(key_lens), _ptr(first), _ptr(count),
-                                         _stream(stream))
-    _raise(rc, "attn_fwd_tile_plan_window")
+    rc = lib().attn_fwd_tile_plan_ex(B, Nq, Nk, d, int(bool(causal)), int(window), int(align),
+                                     _ptr(key_lens), _ptr(first), _ptr(count), _stream(stream))
+    _raise(rc, "attn_fwd_tile_plan_ex")
     return first, count
 
 

@@ -143,47 +143,56 @@ const char* attn_strerror(int status) {
 size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   (void)Nk;
   if (Nq <= 0 || B <= 0 || Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return 0;
-  if (Nq > 1) return prefill_workspace_bytes();
+  // the decode kernels take every call with at most 64 query rows per kv head
+  if (!decode_supported(B, Hq, Hkv, Nq, d)) return prefill_workspace_bytes();
   const int sms = current_sms();
   if (sms <= 0) return 0;
-  return decode_plan(B, Hq, Hkv, d, sms).workspace_bytes;
+  return decode_plan(B, Hq, Hkv, Nq, d, sms).workspace_bytes;
 }
 
-int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
-                    int Hq, int Hkv, int Nq, int Nk, int d, int causal, int window, float scale,
-                    const int32_t* key_lens, void* workspace, size_t workspace_bytes,
-                    void* stream) {
+int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
+                int Hkv, int Nq, int Nk, int d, int causal, int window, int align, float scale,
+                const int32_t* key_lens, void* workspace, size_t workspace_bytes, void* stream) {
   int rc = check_common(q, k, v, o, B, Hq, Hkv, Nq, Nk, d, causal, scale);
   if (rc != ATTN_OK) return rc;
-  if (window < 0) return ATTN_EINVAL;
+  if (window < 0 || (align != 0 && align != 1)) return ATTN_EINVAL;
   if (lse && !aligned16(lse)) return ATTN_EALIGN;
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (Nq == 1) {
-    if (!decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
+  if (decode_supported(B, Hq, Hkv, Nq, d)) {
     const int sms = current_sms();
     if (sms <= 0) return ATTN_ECUDA;
-    const DecodePlan p = decode_plan(B, Hq, Hkv, d, sms);
+    const DecodePlan p = decode_plan(B, Hq, Hkv, Nq, d, sms);
     if (!workspace || workspace_bytes < p.workspace_bytes) return ATTN_EWORKSPACE;
     if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
-    // the single query row sits at position Nk - 1: its window starts at Nk - window
-    const int kv_lo = (window > 0 && window < Nk) ? Nk - window : 0;
-    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nk, d, kv_lo, scale, key_lens, workspace, p,
-                         st);
+    DecodeMask mk;
+    mk.causal = causal;
+    mk.window = window;
+    mk.align = align;
+    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, mk, scale, key_lens, workspace,
+                         p, st);
   }
   if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
   if (!workspace || workspace_bytes < prefill_workspace_bytes()) return ATTN_EWORKSPACE;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
   const int sms = current_sms();
   if (sms <= 0) return ATTN_ECUDA;
-  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, window, scale, key_lens,
-                        workspace, sms, st);
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, window, align, scale,
+                        key_lens, workspace, sms, st);
+}
+
+int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                    int Hq, int Hkv, int Nq, int Nk, int d, int causal, int window, float scale,
+                    const int32_t* key_lens, void* workspace, size_t workspace_bytes,
+                    void* stream) {
+  return attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, window, 0, scale, key_lens,
+                     workspace, workspace_bytes, stream);
 }
 
 int attn_fwd_ws(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                 int Hkv, int Nq, int Nk, int d, int causal, float scale, const int32_t* key_lens,
                 void* workspace, size_t workspace_bytes, void* stream) {
-  return attn_fwd_window(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, 0, scale, key_lens,
-                         workspace, workspace_bytes, stream);
+  return attn_fwd_ex(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, 0, 0, scale, key_lens,
+                     workspace, workspace_bytes, stream);
 }
 
 int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
@@ -194,8 +203,7 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
   void* ws = nullptr;
   size_t ws_bytes = 0;
   {
-    if (Nq == 1 && !decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
-    if (Nq > 1 && !prefill_supported(d)) return ATTN_EUNSUPPORTED;
+    if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
     const size_t need = attn_workspace_size(B, Hq, Hkv, Nq, Nk, d);
     if (need == 0) return ATTN_ECUDA;
     int dev = 0;
@@ -246,15 +254,22 @@ int attn_prefill_tile_shape(int d, int* Br, int* Bc) {
   return ATTN_OK;
 }
 
+int attn_fwd_tile_plan_ex(int B, int Nq, int Nk, int d, int causal, int window, int align,
+                          const int32_t* key_lens, int32_t* first, int32_t* count,
+                          void* stream) {
+  if (!first || !count) return ATTN_EINVAL;
+  if (B <= 0 || Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1) || window < 0 ||
+      (align != 0 && align != 1))
+    return ATTN_EINVAL;
+  if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
+  return launch_tile_plan(B, Nq, Nk, d, causal, window, align, key_lens, first, count,
+                          static_cast<cudaStream_t>(stream));
+}
+
 int attn_fwd_tile_plan_window(int B, int Nq, int Nk, int d, int causal, int window,
                               const int32_t* key_lens, int32_t* first, int32_t* count,
                               void* stream) {
-  if (!first || !count) return ATTN_EINVAL;
-  if (B <= 0 || Nq <= 0 || Nk <= 0 || (causal != 0 && causal != 1) || window < 0)
-    return ATTN_EINVAL;
-  if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
-  return launch_tile_plan(B, Nq, Nk, d, causal, window, key_lens, first, count,
-                          static_cast<cudaStream_t>(stream));
+  return attn_fwd_tile_plan_ex(B, Nq, Nk, d, causal, window, 0, key_lens, first, count, stream);
 }
 
 int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal, const int32_t* key_lens,

@@ -1,4 +1,5 @@
-// decode.cu -- split-KV decode (Nq == 1) and its log-sum-exp combine pass.
+// decode.cu -- split-KV decode (one or a few query rows per sequence) and its
+// log-sum-exp combine pass.
 //
 // One new query token per sequence reads the whole KV cache of its sequence
 // ("Coding interview (14): attention from scratch", section 3.6: the newest
@@ -6,6 +7,10 @@
 // Architecture Deconstructed ...", KV cache section: decode is a
 // bandwidth-bound matrix-vector product).  All Hq/Hkv query heads that share
 // a kv head are processed together, so every K/V byte is read from HBM once.
+// Multi-token decode (Nq new tokens per sequence, e.g. verifying a draft;
+// "Coding interview (14)", self-test 5) processes the R = (Hq/Hkv) * Nq rows
+// of a kv head together the same way; the causal mask among the new tokens
+// (and a sliding window, if any) is applied per (key, row).
 //
 // Work split.  Unit u = (b, kv head h) owns len_u = clamp(key_lens[b], 0, Nk)
 // keys.  The units' keys are laid end to end (T keys in total) and CTA c of a
@@ -32,6 +37,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "tile_plan.cuh"
 
 namespace attn {
 
@@ -50,7 +56,8 @@ struct DecodeSmem {
   static constexpr int kBars = kRing + kStages * kStageBytes;   // full[S], empty[S]
   static constexpr int kScan = kBars + 2 * kStages * 8;          // int64 [kMaxScanB + 1]
   static constexpr int kLens = kScan + (kMaxScanB + 1) * 8;      // int [kMaxScanB]
-  static constexpr int kMbuf = kLens + kMaxScanB * 4;             // float [4 kq][4 mt][16]
+  static constexpr int kLo = kLens + kMaxScanB * 4;               // int [kMaxScanB]
+  static constexpr int kMbuf = kLo + kMaxScanB * 4;               // float [4 kq][4 mt][16]
   static constexpr int kLbuf = kMbuf + 4 * 4 * 16 * 4;           // float [4 mt][16]
   static constexpr int kObuf = kLbuf + 4 * 16 * 4;               // float [4 mt][16][D]
   static constexpr int kAbort = kObuf + 4 * 16 * D * 4;
@@ -76,7 +83,8 @@ struct DecodeArgs {
   float* part_o;
   float* part_lse;
   int B, Hq, Hkv, Nk, G, grid;
-  int kv_lo;        // first key of every unit (sliding window), 0 without one
+  int Nq, R;                 // query rows per sequence, rows per unit (G * Nq)
+  int causal, window, align;
   float scale_log2;
 };
 
@@ -99,6 +107,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
   float* obuf = reinterpret_cast<float*>(smem + L::kObuf);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
   int* lens_s = reinterpret_cast<int*>(smem + L::kLens);
+  int* lo_s = reinterpret_cast<int*>(smem + L::kLo);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int B = a.B, Hkv = a.Hkv, U = B * Hkv;
@@ -120,10 +129,11 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
       const int b = base + lane;
       int len = 0;
       if (b < B) {
-        len = a.key_lens ? a.key_lens[b] : a.Nk;
-        len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
-        len = len > a.kv_lo ? len - a.kv_lo : 0;   // keys [kv_lo, L)
-        lens_s[b] = len;
+        const int Lb = clamp_len(a.key_lens ? a.key_lens[b] : a.Nk, a.Nk);
+        int lo;
+        len = decode_key_range(Lb, query_offset(a.Nq, a.Nk, Lb, a.align), a.window, &lo);
+        lens_s[b] = len;   // keys [lo, L) of every unit of sequence b
+        lo_s[b] = lo;
       }
       long long x = len;
 #pragma unroll
@@ -182,7 +192,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
           uint8_t* kt = smem + L::kRing + st * L::kStageBytes;
           uint8_t* vt = kt + L::kTileBytes;
           mbar_arrive_expect_tx(&full[st], L::kStageBytes);
-          const int row = s.u * a.Nk + a.kv_lo + t;
+          const int row = s.u * a.Nk + lo_s[s.u / Hkv] + t;
 #pragma unroll
           for (int bx = 0; bx < kBoxes; ++bx) {
             tma_load_2d(kt + bx * (kTileKeys * 128), &tmap_k, bx * 64, row, &full[st]);
@@ -206,22 +216,28 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
   bool alive = start < end;
   while (alive && next_seg(u, s)) {
     const int b = s.u / Hkv, h = s.u - b * Hkv;
-    // Q fragments for heads mt*16 .. mt*16+15 of this unit's group
+    // Q fragments for rows mt*16 .. mt*16+15 of this unit (row r = head
+    // (r / Nq) of the group, token r % Nq; the unit's rows are contiguous)
     uint32_t qa[D / 16][4];
+    const int r0 = mt * 16 + g, r1 = r0 + 8;
     {
-      const int r0 = mt * 16 + g, r1 = r0 + 8;
-      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(
-          a.q + ((size_t)b * a.Hq + (size_t)h * a.G + r0) * D);
-      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(
-          a.q + ((size_t)b * a.Hq + (size_t)h * a.G + r1) * D);
+      const size_t qrow = ((size_t)b * a.Hq + (size_t)h * a.G) * a.Nq;
+      const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + (qrow + r0) * D);
+      const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + (qrow + r1) * D);
 #pragma unroll
       for (int ks = 0; ks < D / 16; ++ks) {
-        qa[ks][0] = r0 < a.G ? q0[ks * 8 + t4] : 0u;
-        qa[ks][1] = r1 < a.G ? q1[ks * 8 + t4] : 0u;
-        qa[ks][2] = r0 < a.G ? q0[ks * 8 + 4 + t4] : 0u;
-        qa[ks][3] = r1 < a.G ? q1[ks * 8 + 4 + t4] : 0u;
+        qa[ks][0] = r0 < a.R ? q0[ks * 8 + t4] : 0u;
+        qa[ks][1] = r1 < a.R ? q1[ks * 8 + t4] : 0u;
+        qa[ks][2] = r0 < a.R ? q0[ks * 8 + 4 + t4] : 0u;
+        qa[ks][3] = r1 < a.R ? q1[ks * 8 + 4 + t4] : 0u;
       }
     }
+    // positions of this thread's two rows; key index of segment position 0
+    const int Lb = clamp_len(a.key_lens ? a.key_lens[b] : a.Nk, a.Nk);
+    const int off = query_offset(a.Nq, a.Nk, Lb, a.align);
+    const int pos0 = off + r0 % a.Nq, pos1 = off + r1 % a.Nq;
+    const int key_base = lo_s[b];
+    const bool row_masks = a.Nq > 1 || a.window > 0;
     float m[2] = {-INFINITY, -INFINITY}, l[2] = {0.f, 0.f};
     float acc[D / 8][4];
 #pragma unroll
@@ -255,7 +271,13 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int key = kfirst + n * 8 + 2 * t4 + (e & 1);
-          const float v = key < s.hi ? sc[n][e] * a.scale_log2 : -INFINITY;
+          bool vis = key < s.hi;
+          if (row_masks) {   // causal among the new tokens, sliding window
+            const int dlt = (e >> 1 ? pos1 : pos0) - (key_base + key);
+            vis = vis && (!a.causal || dlt >= 0) &&
+                  (a.window <= 0 || (dlt < a.window && dlt > -a.window));
+          }
+          const float v = vis ? sc[n][e] * a.scale_log2 : -INFINITY;
           sc[n][e] = v;
           mx[e >> 1] = fmaxf(mx[e >> 1], v);
         }
@@ -355,18 +377,18 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
     const size_t slot = (size_t)blockIdx.x + s.u;
     for (int idx = threadIdx.x; idx < MT * 16 * D; idx += kConsumerThreads) {
       const int row = idx / D, c = idx - row * D;   // row = mt*16 + r
-      if (row < a.G) {
+      if (row < a.R) {
         const float lv = lbuf[row];
-        a.part_o[(slot * a.G + row) * D + c] = lv > 0.f ? obuf[idx] / lv : 0.f;
+        a.part_o[(slot * a.R + row) * D + c] = lv > 0.f ? obuf[idx] / lv : 0.f;
       }
     }
     if (kq == 0 && t4 == 0) {
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int row = mt * 16 + g + 8 * r;
-        if (row < a.G) {
+        if (row < a.R) {
           const float lv = lbuf[row];
-          a.part_lse[slot * a.G + row] = lv > 0.f ? M[r] + __log2f(lv) : -INFINITY;
+          a.part_lse[slot * a.R + row] = lv > 0.f ? M[r] + __log2f(lv) : -INFINITY;
         }
       }
     }
@@ -374,10 +396,11 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
   }
 }
 
-// Combine: one CTA per (unit, kCombineThreads / D heads), one thread per
+// Combine: one CTA per (unit, kCombineThreads / D rows), one thread per
 // output element.  The log-sum-exps of the unit's slots are staged in shared
-// memory, per head lse = log2 sum_s 2^lse_s, then every (head, d) output sums
+// memory, per row lse = log2 sum_s 2^lse_s, then every (row, d) output sums
 // its slots' partials weighted by 2^(lse_s - lse) with independent loads.
+// A row no slot saw a key for (masked everywhere) gets O = 0, lse = -inf.
 struct CombineArgs {
   const int32_t* key_lens;
   const float* part_o;
@@ -385,7 +408,8 @@ struct CombineArgs {
   __nv_bfloat16* o;
   float* lse;
   int B, Hq, Hkv, Nk, G, grid;
-  int kv_lo;
+  int Nq, R;
+  int window, align;
 };
 
 constexpr int kCombineThreads = 256;
@@ -397,16 +421,16 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
   __shared__ long long s_pb[2];
   __shared__ int s_len;
   const int u = blockIdx.x, b = u / a.Hkv, h = u - b * a.Hkv;
-  const int G = a.G;
-  constexpr int HB = kCombineThreads / D;            // heads of this block
+  const int G = a.R;                                 // rows of a unit
+  constexpr int HB = kCombineThreads / D;            // rows of this block
   const int g0 = blockIdx.y * HB;
   const int gn = (G - g0) < HB ? (G - g0) : HB;
   // unit start and total key count: block-wide sums over the key lengths
   long long before = 0, total = 0;
   for (int bb = threadIdx.x; bb < a.B; bb += blockDim.x) {
-    int len = a.key_lens ? a.key_lens[bb] : a.Nk;
-    len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
-    len = len > a.kv_lo ? len - a.kv_lo : 0;
+    const int Lb = clamp_len(a.key_lens ? a.key_lens[bb] : a.Nk, a.Nk);
+    int lo;
+    const int len = decode_key_range(Lb, query_offset(a.Nq, a.Nk, Lb, a.align), a.window, &lo);
     total += len;
     if (bb < b) before += len;
     if (bb == b) s_len = len;
@@ -430,12 +454,14 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
   __syncthreads();
   const long long p0 = s_pb[0], T = s_pb[1];
   const int len = s_len;
-  __nv_bfloat16* orow = a.o + ((size_t)b * a.Hq + (size_t)h * G + g0) * D;
+  // the unit's rows are contiguous in o and lse
+  const size_t row0 = ((size_t)b * a.Hq + (size_t)h * a.G) * a.Nq + g0;
+  __nv_bfloat16* orow = a.o + row0 * D;
   if (len == 0) {
     // o / lse may be read by earlier work in the stream only through the split
     // kernel's inputs, so writing before the dependency wait is safe
     for (int idx = threadIdx.x; idx < gn * D; idx += blockDim.x) orow[idx] = __float2bfloat16(0.f);
-    if (a.lse && threadIdx.x < gn) a.lse[(size_t)b * a.Hq + h * G + g0 + threadIdx.x] = -INFINITY;
+    if (a.lse && threadIdx.x < gn) a.lse[row0 + threadIdx.x] = -INFINITY;
     return;
   }
   // CTAs whose ranges intersect [p0, p0 + len); empty ranges wrote no slot
@@ -463,16 +489,23 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
     const int g = threadIdx.x;
     float mx = -INFINITY;
     for (int k = 0; k < ns; ++k) mx = fmaxf(mx, lse_s[k * HB + g]);
-    float sum = 0.f;
-    for (int k = 0; k < ns; ++k) sum += exp2_approx(lse_s[k * HB + g] - mx);
-    const float l2 = mx + __log2f(sum);
+    float l2 = -INFINITY;   // no slot saw a visible key for this row
+    if (mx != -INFINITY) {
+      float sum = 0.f;
+      for (int k = 0; k < ns; ++k) sum += exp2_approx(lse_s[k * HB + g] - mx);
+      l2 = mx + __log2f(sum);
+    }
     L2[g] = l2;
-    if (a.lse) a.lse[(size_t)b * a.Hq + h * G + g0 + g] = l2 * kLn2;
+    if (a.lse) a.lse[row0 + g] = l2 == -INFINITY ? -INFINITY : l2 * kLn2;
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < gn * D; idx += blockDim.x) {
     const int g = idx / D, c = idx - g * D;
     const float l2 = L2[g];
+    if (l2 == -INFINITY) {
+      orow[idx] = __float2bfloat16(0.f);
+      continue;
+    }
     const float* src = a.part_o + (((size_t)c0 + u) * G + g0 + g) * D + c;
     const size_t stride = (size_t)G * D;   // next slot
     float acc = 0.f;
@@ -511,25 +544,27 @@ int launch_decode_t(const DecodePlan& p, const CUtensorMap& tk, const CUtensorMa
 }
 }  // namespace
 
-DecodePlan decode_plan(int B, int Hq, int Hkv, int d, int num_sms) {
+DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int d, int num_sms) {
   DecodePlan p;
   p.grid = num_sms;   // one CTA per SM (the ring takes most of shared memory)
   p.G = Hq / Hkv;
+  p.R = p.G * Nq;
   p.slots = (size_t)p.grid + (size_t)B * Hkv;
-  p.part_o_bytes = ((p.slots * p.G * d * sizeof(float)) + 255) & ~size_t(255);
-  p.part_lse_bytes = ((p.slots * p.G * sizeof(float)) + 255) & ~size_t(255);
+  p.part_o_bytes = ((p.slots * p.R * d * sizeof(float)) + 255) & ~size_t(255);
+  p.part_lse_bytes = ((p.slots * p.R * sizeof(float)) + 255) & ~size_t(255);
   p.workspace_bytes = p.part_o_bytes + p.part_lse_bytes;
   return p;
 }
 
-bool decode_supported(int B, int Hq, int Hkv, int d) {
-  const int G = Hq / Hkv;
-  return (d == 64 || d == 128) && G >= 1 && G <= 64 && B <= kMaxScanB;
+bool decode_supported(int B, int Hq, int Hkv, int Nq, int d) {
+  const long long R = (long long)(Hq / Hkv) * Nq;
+  return (d == 64 || d == 128) && Nq >= 1 && R >= 1 && R <= 64 && B <= kMaxScanB;
 }
 
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nk, int d, int kv_lo, float scale, const int32_t* key_lens,
-                  void* workspace, const DecodePlan& p, cudaStream_t st) {
+                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, float scale,
+                  const int32_t* key_lens, void* workspace, const DecodePlan& p,
+                  cudaStream_t st) {
   CUtensorMap tk, tv;
   const uint64_t rows = (uint64_t)B * Hkv * Nk;
   if (make_tmap_2d_bf16(&tk, k, d, rows, 64, kTileKeys) != ATTN_OK) return ATTN_ECUDA;
@@ -540,14 +575,15 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   a.part_o = static_cast<float*>(workspace);
   a.part_lse = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + p.part_o_bytes);
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = p.G; a.grid = p.grid;
-  a.kv_lo = kv_lo;
+  a.Nq = Nq; a.R = p.R;
+  a.causal = mk.causal; a.window = mk.window; a.align = mk.align;
   a.scale_log2 = scale * kLog2e;
   int rc;
-  if (decode_tc_supported(B, Hq, Hkv, d)) {
-    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nk, kv_lo, scale, key_lens, a.part_o,
+  if (decode_tc_supported(B, Hq, Hkv, Nq, d)) {
+    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nq, Nk, mk, scale, key_lens, a.part_o,
                                 a.part_lse, p.grid, st);
   } else {
-    const int MT = (p.G + 15) / 16;
+    const int MT = (p.R + 15) / 16;
     if (d == 128) {
       rc = MT == 1 ? launch_decode_t<128, 1>(p, tk, tv, a, st)
          : MT == 2 ? launch_decode_t<128, 2>(p, tk, tv, a, st)
@@ -566,12 +602,13 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   c.o = static_cast<__nv_bfloat16*>(o);
   c.lse = lse;
   c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.Nk = Nk; c.G = p.G; c.grid = p.grid;
-  c.kv_lo = kv_lo;
+  c.Nq = Nq; c.R = p.R;
+  c.window = mk.window; c.align = mk.align;
   // shared memory: the unit's slot lse's ([slots][heads of the block], at most
   // grid + 1 slots) + [heads of the block]
   const int hb = kCombineThreads / d;
   const size_t csmem = ((size_t)(p.grid + 2) * hb) * sizeof(float);
-  const dim3 cgrid(B * Hkv, (p.G + hb - 1) / hb);
+  const dim3 cgrid(B * Hkv, (p.R + hb - 1) / hb);
   // programmatic dependent launch: the combine grid may start while the
   // split kernel drains; it waits for the split's results in the kernel
   cudaLaunchConfig_t cfg = {};

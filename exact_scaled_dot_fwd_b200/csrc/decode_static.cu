@@ -73,20 +73,20 @@ int attn_fwd_decode_static(const void* q, const void* k, const void* v, void* o,
   if (d != 64 && d != 128) return ATTN_EUNSUPPORTED;
   if ((long long)B * Hq >= (1ll << 31) || (long long)B * Hkv * Nk >= (1ll << 31))
     return ATTN_EUNSUPPORTED;
-  if (!decode_supported(B, Hq, Hkv, d)) return ATTN_EUNSUPPORTED;
+  if (!decode_supported(B, Hq, Hkv, 1, d)) return ATTN_EUNSUPPORTED;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o)) return ATTN_EALIGN;
   if (lse && !aligned16(lse)) return ATTN_EALIGN;
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return ATTN_ECUDA;
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0)
     return ATTN_ECUDA;
-  const DecodePlan p = decode_plan(B, Hq, Hkv, d, sms);
+  const DecodePlan p = decode_plan(B, Hq, Hkv, 1, d, sms);
   if (p.workspace_bytes > kDecodeStaticScratchBytes) return ATTN_EWORKSPACE;
   void* scratch = nullptr;
   const int rc = scratch_address(&scratch);
   if (rc != ATTN_OK) return rc;
-  return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nk, d, 0, scale, key_lens, scratch, p,
-                       static_cast<cudaStream_t>(stream));
+  return launch_decode(q, k, v, o, lse, B, Hq, Hkv, 1, Nk, d, DecodeMask(), scale, key_lens,
+                       scratch, p, static_cast<cudaStream_t>(stream));
 }
 
 }  // extern "C"

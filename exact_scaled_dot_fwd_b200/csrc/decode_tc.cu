@@ -1,5 +1,5 @@
-// decode_tc.cu -- split-KV decode (Nq == 1, d == 128) on the tcgen05 tensor
-// cores.
+// decode_tc.cu -- split-KV decode (one or a few query rows per sequence,
+// d == 128) on the tcgen05 tensor cores.
 //
 // Same work split and partial-result format as the mma.sync decode kernel in
 // decode.cu (balanced global key ranges per CTA, one partial per (CTA, unit)
@@ -8,7 +8,10 @@
 // MMA dimension is the keys:
 //   S^T [128 keys x N heads]  = K_tile [128 x d] . Q^T      (TMEM, fp32)
 //   O^T [d x N heads]        += V_tile^T [d x 128] . P^T   (TMEM, fp32)
-// N = the unit's query heads rounded up to 16.  One softmax thread owns one
+// N = the unit's query rows rounded up to 16: its G = Hq / Hkv query heads
+// times the Nq query rows of each (multi-token decode: Nq new tokens verified
+// at once; "Coding interview (14)", self-test 5), R = G * Nq <= 64; these rows
+// are contiguous in q, o and lse.  One softmax thread owns one
 // key (one TMEM lane of S^T) and, for O^T, one dimension of d.  The per-head
 // maximum over the tile's keys is a butterfly transpose-reduce across the
 // warp plus a four-entry exchange in shared memory; per-head running sums
@@ -23,6 +26,7 @@
 #include "common.cuh"
 #include "kernels.h"
 #include "tcgen05.cuh"
+#include "tile_plan.cuh"
 
 namespace attn {
 namespace dtc {
@@ -45,8 +49,9 @@ struct Smem {
   static constexpr int kQ = kV + VS * kKV;
   static constexpr int kP = kQ + 2 * kQBox;    // P^T [2 buffers][2 boxes]
   static constexpr int kScan = kP + 4 * kPBox; // int64 [kMaxB + 1]
-  static constexpr int kLens = kScan + (kMaxB + 1) * 8;
-  static constexpr int kRed = kLens + kMaxB * 4;   // float [4][64]
+  static constexpr int kLens = kScan + (kMaxB + 1) * 8;   // int [kMaxB] keys per unit
+  static constexpr int kLo = kLens + kMaxB * 4;            // int [kMaxB] first key
+  static constexpr int kRed = kLo + kMaxB * 4;     // float [4][64]
   static constexpr int kMs = kRed + 4 * 64 * 4;    // float [64] running max (log2 units)
   static constexpr int kAs = kMs + 64 * 4;         // float [64] this tile's rescale factor
   static constexpr int kLs = kAs + 64 * 4;         // float [64] segment row sums
@@ -174,7 +179,8 @@ struct DecodeTcArgs {
   float* part_o;
   float* part_lse;
   int B, Hq, Hkv, Nk, G, grid;
-  int kv_lo;        // first key of every unit (sliding window), 0 without one
+  int Nq, R;                 // query rows per sequence, rows per unit (G * Nq)
+  int causal, window, align;
   float scale_log2;
 };
 
@@ -194,6 +200,7 @@ __global__ void __launch_bounds__(192, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   long long* pb = reinterpret_cast<long long*>(smem + L::kScan);
   int* lens_s = reinterpret_cast<int*>(smem + L::kLens);
+  int* lo_s = reinterpret_cast<int*>(smem + L::kLo);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
   float* m_s = reinterpret_cast<float*>(smem + L::kMs);
   float* a_s = reinterpret_cast<float*>(smem + L::kAs);
@@ -223,10 +230,11 @@ __global__ void __launch_bounds__(192, 1)
       const int b = base + lane;
       int len = 0;
       if (b < B) {
-        len = a.key_lens ? a.key_lens[b] : a.Nk;
-        len = len < 0 ? 0 : (len > a.Nk ? a.Nk : len);
-        len = len > a.kv_lo ? len - a.kv_lo : 0;   // keys [kv_lo, L)
-        lens_s[b] = len;
+        const int Lb = clamp_len(a.key_lens ? a.key_lens[b] : a.Nk, a.Nk);
+        int lo;
+        len = decode_key_range(Lb, query_offset(a.Nq, a.Nk, Lb, a.align), a.window, &lo);
+        lens_s[b] = len;   // keys [lo, L) of every unit of sequence b
+        lo_s[b] = lo;
       }
       long long x = len;
 #pragma unroll
@@ -287,9 +295,9 @@ __global__ void __launch_bounds__(192, 1)
         ++qn;
         mbar_arrive_expect_tx(&bars[L::Q_FULL], 2 * L::kQBox);
         for (int bx = 0; bx < 2; ++bx)
-          tma_load_2d(smem + L::kQ + bx * L::kQBox, &tmap_q, bx * 64, b * a.Hq + h * a.G,
-                      &bars[L::Q_FULL]);
-        const int row0 = s.u * a.Nk + a.kv_lo + s.lo;
+          tma_load_2d(smem + L::kQ + bx * L::kQBox, &tmap_q, bx * 64,
+                      (b * a.Hq + h * a.G) * a.Nq, &bars[L::Q_FULL]);
+        const int row0 = s.u * a.Nk + lo_s[b] + s.lo;
         for (int j = 0; j < n; ++j, ++g) {
           const int ks = g % KS, vs = g % VS;
           if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / KS) & 1) ^ 1, abort_flag)) { ok = false; break; }
@@ -384,6 +392,11 @@ __global__ void __launch_bounds__(192, 1)
     bool ok = start < end;
     while (ok && next_seg(u, s)) {
       const int n = (s.hi - s.lo + kTile - 1) / kTile;
+      // key index of segment position 0, and the rows' position offset
+      const int sb = s.u / a.Hkv;
+      const int Lb = clamp_len(a.key_lens ? a.key_lens[sb] : a.Nk, a.Nk);
+      const int off = query_offset(a.Nq, a.Nk, Lb, a.align);
+      const int key0 = lo_s[sb] + s.lo;
       asm volatile("bar.sync 1, 128;" ::: "memory");   // previous segment done with m_s / l_s
       if (Lr < 64) m_s[Lr] = -INFINITY;
       float lp[N];
@@ -401,6 +414,32 @@ __global__ void __launch_bounds__(192, 1)
         if (!valid) {
 #pragma unroll
           for (int h = 0; h < N; ++h) sv[h] = -INFINITY;
+        }
+        // rows (tokens) that do not see every key of this tile: causal keys
+        // past row 0's position, window keys before the last row's window
+        const int kfirst = key0 + j * kTile;
+        const int klast = kfirst + kTile - 1;
+        const bool tile_mask =
+            (a.causal && klast > off) ||
+            (a.window > 0 && ((long long)kfirst < (long long)off + a.Nq - a.window ||
+                              (!a.causal && (long long)klast >= (long long)off + a.window)));
+        if (tile_mask) {
+          // this key is visible to the rows whose token index t satisfies
+          // t >= key - off (causal) and |off + t - key| < window
+          const int key = kfirst + Lr;
+          int tlo = a.causal ? key - off : -(1 << 30);
+          int thi = 1 << 30;
+          if (a.window > 0) {
+            const int wlo = key - off - a.window + 1;
+            tlo = tlo > wlo ? tlo : wlo;
+            thi = key - off + a.window - 1;
+          }
+          int t = 0;
+#pragma unroll
+          for (int h = 0; h < N; ++h) {
+            if (t < tlo || t > thi) sv[h] = -INFINITY;
+            t = t + 1 == a.Nq ? 0 : t + 1;
+          }
         }
         // per-head max over the tile's keys
         {
@@ -486,14 +525,14 @@ __global__ void __launch_bounds__(192, 1)
       const size_t slot = (size_t)blockIdx.x + s.u;
 #pragma unroll
       for (int h = 0; h < N; ++h) {
-        if (h < a.G) {
+        if (h < a.R) {
           const float l = l_s[h];
-          a.part_o[(slot * a.G + h) * kD + Lr] = l > 0.f ? o[h] / l : 0.f;
+          a.part_o[(slot * a.R + h) * kD + Lr] = l > 0.f ? o[h] / l : 0.f;
         }
       }
-      if (Lr < a.G && Lr < N) {
+      if (Lr < a.R && Lr < N) {
         const float l = l_s[Lr];
-        a.part_lse[slot * a.G + Lr] = l > 0.f ? m_s[Lr] + __log2f(l) : -INFINITY;
+        a.part_lse[slot * a.R + Lr] = l > 0.f ? m_s[Lr] + __log2f(l) : -INFINITY;
       }
       tc::fence_before();
     }
@@ -520,18 +559,19 @@ int launch_tc_t(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CU
 }
 }  // namespace
 
-bool decode_tc_supported(int B, int Hq, int Hkv, int d) {
-  return d == 128 && Hq / Hkv <= 64 && B <= dtc::kMaxB;
+bool decode_tc_supported(int B, int Hq, int Hkv, int Nq, int d) {
+  return d == 128 && (Hq / Hkv) * Nq <= 64 && B <= dtc::kMaxB;
 }
 
 int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                           int Nk, int kv_lo, float scale, const int32_t* key_lens,
-                           float* part_o, float* part_lse, int grid, cudaStream_t st) {
-  const int G = Hq / Hkv;
-  const int N = G <= 16 ? 16 : (G <= 32 ? 32 : 64);
+                           int Nq, int Nk, const DecodeMask& mk, float scale,
+                           const int32_t* key_lens, float* part_o, float* part_lse, int grid,
+                           cudaStream_t st) {
+  const int G = Hq / Hkv, R = G * Nq;
+  const int N = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
   CUtensorMap tq, tk, tv;
   const uint64_t rows = (uint64_t)B * Hkv * Nk;
-  if (make_tmap_2d_bf16(&tq, q, dtc::kD, (uint64_t)B * Hq, 64, (uint32_t)N) != ATTN_OK)
+  if (make_tmap_2d_bf16(&tq, q, dtc::kD, (uint64_t)B * Hq * Nq, 64, (uint32_t)N) != ATTN_OK)
     return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tk, k, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tv, v, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
@@ -540,7 +580,8 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   a.part_o = part_o;
   a.part_lse = part_lse;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = G; a.grid = grid;
-  a.kv_lo = kv_lo;
+  a.Nq = Nq; a.R = R;
+  a.causal = mk.causal; a.window = mk.window; a.align = mk.align;
   a.scale_log2 = scale * kLog2e;
   if (N == 16) return launch_tc_t<16>(grid, tq, tk, tv, a, st);
   if (N == 32) return launch_tc_t<32>(grid, tq, tk, tv, a, st);

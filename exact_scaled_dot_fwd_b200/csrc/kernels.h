@@ -22,35 +22,43 @@ int make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_
 int make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                       uint64_t mats, uint32_t box_cols, uint32_t box_rows);
 
-// ---- decode (Nq == 1)
+// ---- decode (R = (Hq / Hkv) * Nq <= 64 query rows per kv head)
 struct DecodePlan {
   int grid = 0;          // CTAs of the split kernel (one wave)
   int G = 0;             // query heads per kv head
+  int R = 0;             // query rows per kv head (G * Nq)
   size_t slots = 0;      // partial-result slots (grid + B*Hkv)
   size_t part_o_bytes = 0, part_lse_bytes = 0, workspace_bytes = 0;
 };
-DecodePlan decode_plan(int B, int Hq, int Hkv, int d, int num_sms);
-bool decode_supported(int B, int Hq, int Hkv, int d);
-// tcgen05 split kernel (d == 128, up to 64 query heads per kv head); writes
+// Mask of a decode call: causal among the Nq rows, sliding window, query
+// alignment (0: rows end at key Nk - 1; 1: at key key_lens[b] - 1).
+struct DecodeMask {
+  int causal = 0, window = 0, align = 0;
+};
+DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int d, int num_sms);
+bool decode_supported(int B, int Hq, int Hkv, int Nq, int d);
+// tcgen05 split kernel (d == 128, up to 64 query rows per kv head); writes
 // the same partial-result format as the mma.sync split kernel.
-bool decode_tc_supported(int B, int Hq, int Hkv, int d);
+bool decode_tc_supported(int B, int Hq, int Hkv, int Nq, int d);
 int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                           int Nk, int kv_lo, float scale, const int32_t* key_lens,
-                           float* part_o, float* part_lse, int grid, cudaStream_t st);
+                           int Nq, int Nk, const DecodeMask& mk, float scale,
+                           const int32_t* key_lens, float* part_o, float* part_lse, int grid,
+                           cudaStream_t st);
+// Each sequence's units read keys [lo, L) (decode_key_range in tile_plan.cuh).
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nk, int d, int kv_lo, float scale, const int32_t* key_lens,
-                  void* workspace, const DecodePlan& p, cudaStream_t st);
-// Decode reads keys [kv_lo, min(key_lens[b], Nk)) of every sequence; kv_lo is
-// Nk - window (at least 0) under a sliding window of `window` keys, else 0.
+                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, float scale,
+                  const int32_t* key_lens, void* workspace, const DecodePlan& p,
+                  cudaStream_t st);
 
 // ---- prefill (Nq > 1)
 bool prefill_supported(int d);
 size_t prefill_workspace_bytes();   // scheduler counter
 void prefill_tile_shape(int d, int* Br, int* Bc);
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                   int Hkv, int Nq, int Nk, int d, int causal, int window, float scale,
-                   const int32_t* key_lens, void* workspace, int num_sms, cudaStream_t st);
-int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window,
+                   int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
+                   float scale, const int32_t* key_lens, void* workspace, int num_sms,
+                   cudaStream_t st);
+int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window, int align,
                      const int32_t* key_lens, int32_t* first, int32_t* count, cudaStream_t st);
 
 // ---- RoPE

@@ -117,6 +117,7 @@ struct FwdArgs {
   const int32_t* key_lens;
   int B, Hq, Hkv, Nq, Nk, causal;
   int window;       // sliding window in keys, 0 = none
+  int align;        // query positions: 0 end at key Nk - 1, 1 at key key_lens[b] - 1
   int head_pairs;   // 1: tiles are heads (2p, 2p+1) at one row tile; 0: row tiles 2p, 2p+1
   int ntq;          // ceil(Nq / 128)
   int units;        // items per cost rank (head_pairs: B*Hq/2, else B*Hq)
@@ -131,6 +132,7 @@ namespace pf {
 struct Item {
   Tile tl[2];       // tl[0] has the fewer KV tiles
   int b, n, L;
+  int off;          // key position of query row i is i + off
   int kv_begin;     // KV tile of step 0 (both slots)
   int kv_row0;      // cache row of KV tile kv_begin
 };
@@ -172,13 +174,14 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window)
     it.tl[0].head = it.tl[1].head = h;
   }
   it.L = clamp_len(a.key_lens ? a.key_lens[it.b] : a.Nk, a.Nk);
+  it.off = query_offset(a.Nq, a.Nk, it.L, a.align);
   int begin[2];
 #pragma unroll
   for (int t = 0; t < 2; ++t) {
     KvRange r;
     r.begin = r.count = r.um_begin = r.um_end = 0;
     if (it.tl[t].row_tile < a.ntq)
-      r = kv_tile_range(it.tl[t].row_tile, kM, kN, a.Nq, a.Nk, a.causal, it.L, window);
+      r = kv_tile_range(it.tl[t].row_tile, kM, kN, a.Nq, it.off, a.causal, it.L, window);
     begin[t] = r.begin;
     it.tl[t].count = r.count;
     it.tl[t].um_begin = r.um_begin;
@@ -450,7 +453,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       if (T.row_tile >= a.ntq) continue;
       const int row = T.row_tile * kM + r;
       int vlo, vhi;   // this row's visible keys [vlo, vhi)
-      visible_range(row, a.Nq, a.Nk, a.causal, it.L, window, &vlo, &vhi);
+      visible_range(row, it.off, a.causal, it.L, window, &vlo, &vhi);
       float m_run = -INFINITY, l_run = 0.f;
 
       for (int j = 0; j < T.count; ++j) {
@@ -616,8 +619,9 @@ void prefill_tile_shape(int d, int* Br, int* Bc) {
 }
 
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                   int Hkv, int Nq, int Nk, int d, int causal, int window, float scale,
-                   const int32_t* key_lens, void* workspace, int num_sms, cudaStream_t st) {
+                   int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
+                   float scale, const int32_t* key_lens, void* workspace, int num_sms,
+                   cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (make_tmap_3d_bf16(&tq, q, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tk, k, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
@@ -629,6 +633,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   a.key_lens = key_lens;
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.causal = causal;
   a.window = window;
+  a.align = align;
   a.ntq = (Nq + pf::kM - 1) / pf::kM;
   a.head_pairs = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
   a.scale_log2 = scale * kLog2e;
@@ -665,26 +670,27 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
 }
 
 __global__ void tile_plan_kernel(const int32_t* key_lens, int B, int Nq, int Nk, int causal,
-                                 int window, int Br, int Bc, int nqt, int32_t* first,
+                                 int window, int align, int Br, int Bc, int nqt, int32_t* first,
                                  int32_t* count) {
   const int idx = blockIdx.x * blockDim.x + threadIdx.x;
   if (idx >= B * nqt) return;
   const int b = idx / nqt, qt = idx - b * nqt;
   const int L_b = clamp_len(key_lens ? key_lens[b] : Nk, Nk);
-  const KvRange r = kv_tile_range(qt, Br, Bc, Nq, Nk, causal, L_b, window);
+  const KvRange r =
+      kv_tile_range(qt, Br, Bc, Nq, query_offset(Nq, Nk, L_b, align), causal, L_b, window);
   first[idx] = r.count > 0 ? r.begin : -1;
   count[idx] = r.count;
 }
 
-int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window,
+int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window, int align,
                      const int32_t* key_lens, int32_t* first, int32_t* count, cudaStream_t st) {
   int Br, Bc;
   prefill_tile_shape(d, &Br, &Bc);
   const int nqt = (Nq + Br - 1) / Br;
   const int n = B * nqt;
   if (n == 0) return ATTN_OK;
-  tile_plan_kernel<<<(n + 255) / 256, 256, 0, st>>>(key_lens, B, Nq, Nk, causal, window, Br, Bc,
-                                                    nqt, first, count);
+  tile_plan_kernel<<<(n + 255) / 256, 256, 0, st>>>(key_lens, B, Nq, Nk, causal, window, align,
+                                                    Br, Bc, nqt, first, count);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 

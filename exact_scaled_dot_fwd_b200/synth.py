@@ -61,6 +61,7 @@ class Workload:
     key_lens: tuple | None = None   # (lo, hi) inclusive uniform range
     note: str = ""
     window: int = 0                 # sliding window in keys (0 = none)
+    align: int = 0                  # 1: query rows are each sequence's newest Nq tokens
 
     @property
     def scale(self) -> float:
@@ -100,6 +101,10 @@ WORKLOADS = {
     # the rule but no size; 4096 is a common choice)
     "long_window": Workload("long_window", 7, 1, 32, 32, 32768, 32768, 128, True,
                             window=4096),
+    # multi-token decode (draft verification): 4 new tokens per sequence after
+    # a ragged cache, GQA 32/8; key_lens count cache + new tokens
+    "spec_decode": Workload("spec_decode", 8, 16, 32, 8, 4, 16384, 128, True,
+                            key_lens=(1028, 16384), align=1),
 }
 
 ROPE_BASE = 10000.0

@@ -61,9 +61,11 @@ typedef enum {
   ATTN_ETIMEOUT = 6       /* a kernel gave up waiting on a barrier (device status) */
 } attn_status;
 
-/* Exact attention forward.  Dispatch: Nq == 1 runs the split-KV decode kernel
- * followed by the log-sum-exp combine pass; Nq > 1 runs the tiled prefill
- * kernel (TMA + tcgen05/TMEM, persistent, one CTA per SM).
+/* Exact attention forward.  Dispatch: calls with at most 64 query rows per kv
+ * head ((Hq / Hkv) * Nq <= 64: single-token decode, multi-token decode) run
+ * the split-KV decode kernel followed by the log-sum-exp combine pass; all
+ * others run the tiled prefill kernel (TMA + tcgen05/TMEM, persistent, one
+ * CTA per SM).
  *   d: 64 or 128.  scale: finite and > 0 (usually 1/sqrt(d); "Transformer
  *   Architecture Breakdown ...", section 1.2).  causal: 0 or 1 (ignored in
  *   effect for Nq == 1, where j <= Nk - 1 always holds).
@@ -88,18 +90,35 @@ ATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* o,
                 int causal, float scale, const int32_t* key_lens,
                 void* workspace, size_t workspace_bytes, void* stream);
 
-/* Sliding-window attention ("Attention mechanisms ...", section 11): as
- * attn_fwd_ws, with key j visible to query row i only if, in addition to the
- * rules above, |p - j| < window, where p = i + (Nk - Nq) is the row's key
- * position (bottom-right alignment, as for the causal mask).  window = 0
- * means no window (identical to attn_fwd_ws); window < 0 is ATTN_EINVAL.
- * With causal = 1 a row sees the last `window` positions up to and including
- * its own; with causal = 0 it also sees window - 1 positions after it.
- *   Prefill (Nq > 1) visits only the KV tiles that hold visible keys
- *   (attn_fwd_tile_plan_window reports them).  Decode (Nq == 1) reads keys
- *   [max(0, Nk - window), key_lens[b]) of each sequence.
+/* Query alignment (the `align` argument of attn_fwd_ex). */
+#define ATTN_ALIGN_NK 0      /* row i at key position p = i + (Nk - Nq) */
+#define ATTN_ALIGN_KEYLEN 1  /* row i at p = i + (L - Nq), L = clamp(key_lens[b], 0, Nk) */
+
+/* The general entry point: attn_fwd_ws plus a sliding window and a choice of
+ * query positions.
+ *   Query row i of batch b sits at key position p (align, above).  Key j is
+ *   visible iff j < L, and (causal) j <= p, and (window > 0) |p - j| < window
+ *   ("Attention mechanisms ...", section 11).  window = 0: no window;
+ *   window < 0, or align not 0/1: ATTN_EINVAL.  With causal = 1 a row sees
+ *   the last `window` positions up to and including its own; with causal = 0
+ *   it also sees window - 1 positions after it.
+ *   ATTN_ALIGN_KEYLEN is multi-token decode over ragged caches ("Coding
+ *   interview (14)", self-test 5): the Nq rows are the newest Nq tokens of
+ *   each sequence, whose cache plus those tokens fill keys [0, L); with
+ *   causal = 1, row i sees the L - Nq cached keys and new tokens 0..i.  With
+ *   L = Nk for every sequence both alignments agree.  The ABI's other entry
+ *   points use ATTN_ALIGN_NK.
+ *   The prefill kernel visits only the KV tiles that hold visible keys
+ *   (attn_fwd_tile_plan_ex reports them); the decode kernels read each
+ *   sequence's keys from the first one its first row sees up to L.
  *   Workspace: attn_workspace_size(...) bytes, as for attn_fwd_ws.
  * Errors: as attn_fwd_ws. */
+ATTN_API int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse,
+                         int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                         int window, int align, float scale, const int32_t* key_lens,
+                         void* workspace, size_t workspace_bytes, void* stream);
+
+/* attn_fwd_ex with align = ATTN_ALIGN_NK: sliding-window attention. */
 ATTN_API int attn_fwd_window(const void* q, const void* k, const void* v, void* o,
                              float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,
                              int causal, int window, float scale,
@@ -135,9 +154,15 @@ ATTN_API int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal,
                        const int32_t* key_lens, int32_t* first,
                        int32_t* count, void* stream);
 
-/* attn_fwd_tile_plan under a sliding window of `window` keys (0 = none):
- * first = the first KV tile a query tile visits, count = how many in a row
- * (the range covers every visible key of the tile's rows and nothing else). */
+/* attn_fwd_tile_plan under a sliding window of `window` keys (0 = none) and
+ * a query alignment (as attn_fwd_ex): first = the first KV tile a query tile
+ * visits, count = how many in a row (the range covers every visible key of
+ * the tile's rows and no tile without one). */
+ATTN_API int attn_fwd_tile_plan_ex(int B, int Nq, int Nk, int d, int causal,
+                                   int window, int align, const int32_t* key_lens,
+                                   int32_t* first, int32_t* count, void* stream);
+
+/* attn_fwd_tile_plan_ex with align = ATTN_ALIGN_NK. */
 ATTN_API int attn_fwd_tile_plan_window(int B, int Nq, int Nk, int d, int causal,
                                        int window, const int32_t* key_lens,
                                        int32_t* first, int32_t* count, void* stream);

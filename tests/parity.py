@@ -40,7 +40,7 @@ def from_dev(t):
     return synth.bf16_bits_to_f32(bits).astype(np.float64)
 
 
-def run_gpu(inputs, causal, scale, rope=None, window=0):
+def run_gpu(inputs, causal, scale, rope=None, window=0, align=0):
     """Attention through the C ABI; returns (o float64 [B,Hq,Nq,d], lse float64)."""
     import torch
     import exact_scaled_dot_fwd_b200 as eb
@@ -52,7 +52,8 @@ def run_gpu(inputs, causal, scale, rope=None, window=0):
                           pairing=rope["pairing"])
         k = eb.rope_apply(k, base=rope["base"], pos_offset=rope.get("k_pos_offset", 0),
                           pairing=rope["pairing"])
-    o, lse = eb.attn_fwd(q, k, v, causal=causal, scale=scale, key_lens=kl_t, window=window)
+    o, lse = eb.attn_fwd(q, k, v, causal=causal, scale=scale, key_lens=kl_t, window=window,
+                         align=align)
     torch.cuda.synchronize()
     assert eb.device_status() == 0
     return from_dev(o), lse.cpu().numpy().astype(np.float64)
@@ -80,14 +81,15 @@ def compare(o_gpu_rows, lse_gpu_rows, o_ref, lse_ref, what=""):
     return res
 
 
-def check_workload(inputs, shape, causal, scale, rows=None, rope=None, what="", window=0):
+def check_workload(inputs, shape, causal, scale, rows=None, rope=None, what="", window=0,
+                   align=0):
     """Run GPU + oracle on the same inputs; rows = flat row ids or None (all)."""
     B, Hq, Nq, d = shape
-    o, lse = run_gpu(inputs, causal, scale, rope=rope, window=window)
+    o, lse = run_gpu(inputs, causal, scale, rope=rope, window=window, align=align)
     o = o.reshape(-1, d)
     lse = lse.reshape(-1)
     o_ref, lse_ref = oracle.attn_rows(inputs["q"], inputs["k"], inputs["v"], causal, scale,
                                       key_lens=inputs.get("key_lens"), rows=rows,
-                                      rope_cfg=rope, window=window)
+                                      rope_cfg=rope, window=window, align=align)
     sel = slice(None) if rows is None else rows
     return compare(o[sel], lse[sel], o_ref, lse_ref, what)

@@ -72,13 +72,15 @@ def test_attn_fwd_ws_rejects_missing_workspace(L):
     # CPU-only host the call fails before any launch either way)
     rc = L.attn_fwd_ws(P, P, P, P, None, 2, 4, 1, 1, 64, 64, 0, 0.125, None, None, 0, None)
     assert rc in (4, 5)
-    # prefill needs 256 bytes for its scheduler counter
-    assert L.attn_workspace_size(1, 2, 2, 8, 8, 64) == 256
-    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0, 0.125, None, None, 0, None)
+    # prefill (more than 64 query rows per kv head) needs 256 bytes for its
+    # scheduler counter
+    assert L.attn_workspace_size(1, 2, 2, 128, 128, 64) == 256
+    assert L.attn_workspace_size(1, 64, 1, 2, 128, 64) == 256
+    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 0, 0.125, None, None, 0, None)
     assert rc == 4
-    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0, 0.125, None, P, 128, None)
+    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 0, 0.125, None, P, 128, None)
     assert rc == 4
-    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 0, 0.125, None,
+    rc = L.attn_fwd_ws(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 0, 0.125, None,
                        ctypes.c_void_p(0x1010), 256, None)
     assert rc == 3
 
@@ -120,14 +122,25 @@ def test_binding_fails_loudly_without_library(monkeypatch, tmp_path):
 def test_window_entry_points_reject_bad_arguments_on_host(L):
     w = L.attn_fwd_window
     # negative window
-    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, -1, 0.125, None, P, 256, None) == 1
+    assert w(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, -1, 0.125, None, P, 256, None) == 1
     # the checks shared with attn_fwd_ws come first
-    assert w(None, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, 16, 0.125, None, P, 256, None) == 1
-    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 96, 1, 16, 0.125, None, P, 256, None) == 2
-    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, 16, 0.125, None, None, 0, None) == 4
-    assert w(P, P, P, P, None, 1, 2, 2, 8, 8, 64, 1, 16, 0.125, None,
+    assert w(None, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, 16, 0.125, None, P, 256, None) == 1
+    assert w(P, P, P, P, None, 1, 2, 2, 128, 128, 96, 1, 16, 0.125, None, P, 256, None) == 2
+    assert w(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, 16, 0.125, None, None, 0, None) == 4
+    assert w(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, 16, 0.125, None,
              ctypes.c_void_p(0x1010), 256, None) == 3
     t = L.attn_fwd_tile_plan_window
     assert t(1, 8, 8, 64, 1, -1, None, P, P, None) == 1
     assert t(1, 8, 8, 64, 1, 16, None, None, P, None) == 1
     assert t(1, 8, 8, 96, 1, 16, None, P, P, None) == 2
+
+
+def test_ex_entry_points_reject_bad_arguments_on_host(L):
+    x = L.attn_fwd_ex
+    # align must be 0 or 1, window >= 0
+    assert x(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, 0, 2, 0.125, None, P, 256, None) == 1
+    assert x(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, -3, 1, 0.125, None, P, 256, None) == 1
+    assert x(P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, 0, 1, 0.125, None, None, 0, None) == 4
+    t = L.attn_fwd_tile_plan_ex
+    assert t(1, 8, 8, 64, 1, 0, 2, None, P, P, None) == 1
+    assert t(1, 8, 8, 64, 1, 0, 1, None, None, P, None) == 1
