@@ -54,6 +54,8 @@ def lib():
         L.oracle_kv_tiles_ex.argtypes = [i64, i64, i32, i64, i64, i32, i64, i64, i64, vp, vp,
                                          vp]
         L.oracle_kv_tiles_ex.restype = None
+        L.oracle_gather_paged.argtypes = [vp, i64, i64, i64, i64, vp, i64, vp, i64, i64, vp]
+        L.oracle_gather_paged.restype = i32
         _lib = L
     return _lib
 
@@ -172,3 +174,33 @@ def attn_online_rows(q, k, v, causal, scale, block, key_lens=None, rows=None, nt
     if st != 0:
         raise ValueError("oracle_attn_online_rows rejected its arguments")
     return o, lse
+
+
+def gather_paged(cache, block_table, key_lens, Nk):
+    """Paged cache bf16 bits [num_pages, Hkv, page_size, d] + block table
+    int32 [B, max_pages] -> contiguous bf16 bits [B, Hkv, Nk, d] (keys beyond
+    key_lens[b] zero)."""
+    c = np.ascontiguousarray(cache, dtype=np.uint16)
+    bt = np.ascontiguousarray(block_table, dtype=np.int32)
+    kl = np.ascontiguousarray(key_lens, dtype=np.int32)
+    num_pages, Hkv, ps, d = c.shape
+    B, max_pages = bt.shape
+    out = np.empty((B, Hkv, Nk, d), np.uint16)
+    st = lib().oracle_gather_paged(_ptr(c), num_pages, Hkv, ps, d, _ptr(bt), max_pages, _ptr(kl),
+                                   B, Nk, _ptr(out))
+    if st != 0:
+        raise ValueError("oracle_gather_paged rejected its arguments")
+    return out
+
+
+def attn_paged_rows(q, k_cache, v_cache, block_table, key_lens, causal, scale, rows=None,
+                    window=0, nthreads=None):
+    """Attention of q [B, Hq, Nq, d] over a paged cache: the gathered logical
+    cache with each sequence's query rows at its newest positions (align 1)."""
+    B, _, Nq, _ = np.shape(q)
+    max_pages = np.shape(block_table)[1]
+    Nk = int(max(1, max_pages * np.shape(k_cache)[2]))
+    k = gather_paged(k_cache, block_table, key_lens, Nk)
+    v = gather_paged(v_cache, block_table, key_lens, Nk)
+    return attn_rows(q, k, v, causal, scale, key_lens=key_lens, rows=rows, window=window,
+                     align=1, nthreads=nthreads)

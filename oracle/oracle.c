@@ -170,6 +170,43 @@ void oracle_kv_tiles_ex(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
   }
 }
 
+/* ---- paged KV cache ([TIN] PagedAttention; [AME] 20) -------------------- */
+
+/* Logical key j of kv head h of sequence b lives in physical block
+ * block_table[b][j / page_size] at offset j % page_size: cache layout
+ * [num_pages, Hkv, page_size, d], as the pages write a token's K/V into
+ * kv_cache[phys, :, offset, :].  Copies keys [0, key_lens[b]) of every
+ * (b, h) into out [B, Hkv, Nk, d] and zero-fills keys [key_lens[b], Nk).
+ * Returns -1 (and writes nothing further) if a needed table entry lies
+ * outside [0, num_pages). */
+int oracle_gather_paged(const uint16_t* cache, int64_t num_pages, int64_t Hkv,
+                        int64_t page_size, int64_t d,
+                        const int32_t* block_table, int64_t max_pages,
+                        const int32_t* key_lens, int64_t B, int64_t Nk,
+                        uint16_t* out) {
+  if (page_size <= 0 || max_pages * page_size < Nk) return -1;
+  for (int64_t b = 0; b < B; ++b) {
+    int64_t L = key_lens[b];
+    if (L < 0) L = 0;
+    if (L > Nk) L = Nk;
+    for (int64_t h = 0; h < Hkv; ++h) {
+      uint16_t* dst = out + (b * Hkv + h) * Nk * d;
+      for (int64_t j = 0; j < Nk; ++j) {
+        if (j >= L) {
+          memset(dst + j * d, 0, sizeof(uint16_t) * d);
+          continue;
+        }
+        const int64_t page = block_table[b * max_pages + j / page_size];
+        if (page < 0 || page >= num_pages) return -1;
+        const uint16_t* src =
+            cache + ((page * Hkv + h) * page_size + j % page_size) * d;
+        memcpy(dst + j * d, src, sizeof(uint16_t) * d);
+      }
+    }
+  }
+  return 0;
+}
+
 /* ---- attention rows ---------------------------------------------------- */
 
 typedef struct {

@@ -129,6 +129,19 @@ void oracle_kv_tiles_ex(int64_t Nq, int64_t Nk, int causal, int64_t key_len,
                         int64_t qt, int64_t* first, int64_t* last,
                         int64_t* count);
 
+/* Paged KV cache ([TIN] PagedAttention; [AME] 20): key j of kv head h of
+ * sequence b is row j % page_size of head h in physical block
+ * block_table[b * max_pages + j / page_size]; cache [num_pages, Hkv,
+ * page_size, d].  Gathers keys [0, key_lens[b]) into out [B, Hkv, Nk, d]
+ * (zeros beyond key_lens[b]); attention over a paged cache is attention
+ * over this gathered cache.  Returns 0, or -1 for a table entry outside
+ * [0, num_pages) or max_pages * page_size < Nk. */
+int oracle_gather_paged(const uint16_t* cache, int64_t num_pages, int64_t Hkv,
+                        int64_t page_size, int64_t d,
+                        const int32_t* block_table, int64_t max_pages,
+                        const int32_t* key_lens, int64_t B, int64_t Nk,
+                        uint16_t* out);
+
 #ifdef __cplusplus
 }
 #endif

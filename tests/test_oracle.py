@@ -588,3 +588,67 @@ def test_alignment_special_cases():
     # tile sets follow each sequence's own length
     assert oracle.kv_tiles(8, 4096, True, 1000, 128, 128, 0, align=1) == (0, 7, 8)
     assert oracle.kv_tiles(8, 4096, True, 1000, 128, 128, 0, window=300, align=1) == (5, 7, 3)
+
+
+# ------------------------------------------------------- paged KV cache ----
+
+class _PageTable:
+    """The pages' block allocator ('Attention mechanisms ...', section 20;
+    'Transformer internals', PagedAttention): on a block boundary pop a free
+    physical block; a token at position p lives in table[p // block_size] at
+    offset p % block_size."""
+
+    def __init__(self, num_blocks, block_size):
+        self.free = list(range(num_blocks))
+        self.tables, self.block_size = {}, block_size
+
+    def append_token(self, request_id, position):
+        table = self.tables.setdefault(request_id, [])
+        if position % self.block_size == 0:
+            table.append(self.free.pop())
+        return table[position // self.block_size], position % self.block_size
+
+
+@pytest.mark.parametrize("page_size", [8, 16, 32])
+def test_paged_cache_built_token_by_token(page_size):
+    """Append every sequence's tokens one at a time in an interleaved order,
+    writing K/V into kv_cache[phys, :, offset, :] as the pages do; the
+    oracle's gather and paged attention must reproduce the contiguous cache
+    and its attention exactly."""
+    B, Hq, Hkv, Nq, d = 3, 4, 2, 3, 16
+    lens = [37, 5, 64]
+    Nk = max(lens)
+    max_pages = -(-Nk // page_size)
+    k = synth.normal_bf16((B, Hkv, Nk, d), 401)
+    v = synth.normal_bf16((B, Hkv, Nk, d), 402)
+    q = synth.normal_bf16((B, Hq, Nq, d), 403)
+    num_blocks = sum(-(-n // page_size) for n in lens) + 4
+    k_cache = np.full((num_blocks, Hkv, page_size, d), 0x7fc0, np.uint16)   # NaN filler
+    v_cache = k_cache.copy()
+    pt = _PageTable(num_blocks, page_size)
+    for pos in range(Nk):                      # interleave the sequences
+        for b in range(B):
+            if pos < lens[b]:
+                phys, off = pt.append_token(b, pos)
+                k_cache[phys, :, off, :] = k[b, :, pos, :]
+                v_cache[phys, :, off, :] = v[b, :, pos, :]
+    table = np.zeros((B, max_pages), np.int32)
+    for b in range(B):
+        table[b, :len(pt.tables[b])] = pt.tables[b]
+    kl = np.array(lens, np.int32)
+    kg = oracle.gather_paged(k_cache, table, kl, Nk)
+    for b in range(B):
+        assert np.array_equal(kg[b, :, :lens[b]], k[b, :, :lens[b]])
+        assert not kg[b, :, lens[b]:].any()
+    o1, l1 = oracle.attn_paged_rows(q, k_cache, v_cache, table, kl, True, 0.3)
+    o2, l2 = oracle.attn_rows(q, k, v, True, 0.3, key_lens=kl, align=1)
+    assert np.array_equal(o1, o2) and np.array_equal(l1, l2)
+
+
+def test_paged_gather_rejects_bad_table_entries():
+    cache = np.zeros((2, 1, 16, 8), np.uint16)
+    table = np.array([[0, 5]], np.int32)       # block 5 does not exist
+    with pytest.raises(ValueError):
+        oracle.gather_paged(cache, table, np.array([20], np.int32), 32)
+    # entries past the sequence's length are never read
+    assert oracle.gather_paged(cache, table, np.array([16], np.int32), 32).shape == (1, 1, 32, 8)
