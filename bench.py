@@ -394,6 +394,8 @@ def run_ours(args):
         line["decode"] = run_decode(torch, eb, device, stream, peaks, peak_src)
         line["multi_token_decode"] = run_decode(torch, eb, device, stream, peaks, peak_src,
                                                 name="spec_decode")
+        line["paged_decode"] = run_decode(torch, eb, device, stream, peaks, peak_src,
+                                          page_size=16)
     # ---- sliding-window prefill, same run
     if not args.no_window and w.name != "long_window" and rank == 0 and world == 1:
         line["window"] = run_window(torch, eb, device, stream, peaks, peak_src)
@@ -419,9 +421,17 @@ def run_ours(args):
         dist.destroy_process_group()
 
 
-def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa_decode"):
+def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa_decode",
+               page_size=0):
+    """A decode workload in GB/s; page_size > 0 stores its KV cache in pages
+    of that many tokens, shuffled, and runs the paged entry point."""
     w = synth.WORKLOADS[name]
     x = synth.make_inputs(w)
+    if page_size:
+        table, num_pages = synth.paged_layout(x["key_lens"], page_size, w.seed + 6)
+        x["k"] = synth.to_paged(x["k"], table, x["key_lens"], num_pages, page_size, 0)
+        x["v"] = synth.to_paged(x["v"], table, x["key_lens"], num_pages, page_size, 0)
+        table_d = torch.from_numpy(table).to(device)
     per_copy = x["k"].nbytes + x["v"].nbytes
     copies = 2
     Q = to_dev(x["q"], torch, device)
@@ -434,8 +444,12 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa
                      dtype=torch.uint8, device=device)
 
     def step(i):
-        eb.attn_fwd_ws(Q, K[i % copies], V[i % copies], ws, causal=w.causal, scale=w.scale,
-                       key_lens=kl, out=O, lse=LSE, window=w.window, align=w.align)
+        if page_size:
+            eb.attn_fwd_paged(Q, K[i % copies], V[i % copies], table_d, kl, causal=w.causal,
+                              scale=w.scale, window=w.window, workspace=ws, out=O, lse=LSE)
+        else:
+            eb.attn_fwd_ws(Q, K[i % copies], V[i % copies], ws, causal=w.causal, scale=w.scale,
+                           key_lens=kl, out=O, lse=LSE, window=w.window, align=w.align)
 
     for i in range(5):
         step(i)
@@ -445,6 +459,7 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa
     gbs = decode_bytes(w, x["key_lens"]) * n / (ms / 1e3) / 1e9
     return {"metric": "decode GB/s (algorithmic bytes: K/V of valid keys + Q + O + lse)",
             "value": gbs, "unit": "GB/s", "workload": w.name, "steps": n, "ms_per_step": ms / n,
+            "page_size": page_size or None,
             "algorithmic_bytes": decode_bytes(w, x["key_lens"]),
             "l2": f"{copies} rotating KV caches ({copies * per_copy / 1e6:.0f} MB allocated)",
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",

@@ -13,7 +13,8 @@ import ctypes
 import math
 import os
 
-__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_decode_static", "rope_apply",
+__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_paged",
+           "attn_fwd_decode_static", "rope_apply",
            "prefill_tile_shape", "tile_plan", "device_status", "AttnError", "lib",
            "STATUS_NAMES"]
 
@@ -50,6 +51,9 @@ def lib():
         L.attn_fwd_window.restype = i
         L.attn_fwd_ex.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp, vp, sz, vp]
         L.attn_fwd_ex.restype = i
+        L.attn_fwd_paged.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp, i, i, i, i, i, i, i, f, vp,
+                                     vp, sz, vp]
+        L.attn_fwd_paged.restype = i
         L.attn_workspace_size.argtypes = [i, i, i, i, i, i]
         L.attn_workspace_size.restype = sz
         L.rope_apply.argtypes = [vp, vp, i, i, i, i, f, i, i, vp]
@@ -193,6 +197,41 @@ def attn_fwd_ws(q, k, v, workspace, causal=False, scale=None, key_lens=None, out
                                int(bool(causal)), float(scale), _ptr(key_lens), _ptr(workspace),
                                ws_bytes, _stream(stream))
         _raise(rc, "attn_fwd_ws")
+    return (out, lse) if return_lse else out
+
+
+def attn_fwd_paged(q, k_cache, v_cache, block_table, key_lens, causal=True, scale=None,
+                   window=0, workspace=None, out=None, lse=None, return_lse=True, stream=None):
+    """Decode over a paged KV cache: q bf16 [B, Hq, Nq, d] (each sequence's
+    newest Nq tokens), k_cache/v_cache bf16 [num_pages, Hkv, page_size, d],
+    block_table int32 [B, max_pages], key_lens int32 [B] (sequence lengths)."""
+    torch = _torch()
+    _check_tensor(q, "q", torch.bfloat16, 4)
+    _check_tensor(k_cache, "k_cache", torch.bfloat16, 4)
+    _check_tensor(v_cache, "v_cache", torch.bfloat16, 4)
+    _check_tensor(block_table, "block_table", torch.int32, 2)
+    _check_tensor(key_lens, "key_lens", torch.int32, 1)
+    B, Hq, Nq, d = q.shape
+    num_pages, Hkv, page_size, dk = k_cache.shape
+    if tuple(v_cache.shape) != tuple(k_cache.shape) or dk != d or block_table.shape[0] != B:
+        raise ValueError("paged cache shapes do not match q / block_table")
+    max_pages = block_table.shape[1]
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = attn_workspace_size(B, Hq, Hkv, Nq, max_pages * page_size, d)
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().attn_fwd_paged(_ptr(q), _ptr(k_cache), _ptr(v_cache), _ptr(block_table),
+                              max_pages, page_size, num_pages, _ptr(out),
+                              _ptr(lse if return_lse else None), B, Hq, Hkv, Nq, d,
+                              int(bool(causal)), int(window), float(scale), _ptr(key_lens),
+                              _ptr(workspace), ws_bytes, _stream(stream))
+    _raise(rc, "attn_fwd_paged")
     return (out, lse) if return_lse else out
 
 

@@ -168,8 +168,8 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
     mk.causal = causal;
     mk.window = window;
     mk.align = align;
-    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, mk, scale, key_lens, workspace,
-                         p, st);
+    return launch_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, mk, nullptr, scale, key_lens,
+                         workspace, p, st);
   }
   if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
   if (!workspace || workspace_bytes < prefill_workspace_bytes()) return ATTN_EWORKSPACE;
@@ -178,6 +178,42 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
   if (sms <= 0) return ATTN_ECUDA;
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, window, align, scale,
                         key_lens, workspace, sms, st);
+}
+
+int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                   const int32_t* block_table, int max_pages, int page_size, int num_pages,
+                   void* o, float* lse, int B, int Hq, int Hkv, int Nq, int d, int causal,
+                   int window, float scale, const int32_t* key_lens, void* workspace,
+                   size_t workspace_bytes, void* stream) {
+  if (!block_table || !key_lens) return ATTN_EINVAL;
+  if (max_pages <= 0 || num_pages <= 0 || page_size <= 0) return ATTN_EINVAL;
+  if ((long long)max_pages * page_size >= (1ll << 31)) return ATTN_EUNSUPPORTED;
+  const int Nk = max_pages * page_size;   // logical capacity of a sequence
+  int rc = check_common(q, k_cache, v_cache, o, B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != ATTN_OK) return rc;
+  if (window < 0) return ATTN_EINVAL;
+  // whole pages per tile (128 keys for d = 128, 64 for d = 64), 1 KB-aligned boxes
+  const int tile = d == 128 ? 128 : 64;
+  if (page_size % 8 != 0 || tile % page_size != 0) return ATTN_EUNSUPPORTED;
+  if ((long long)num_pages * Hkv * page_size >= (1ll << 31)) return ATTN_EUNSUPPORTED;
+  if (!decode_supported(B, Hq, Hkv, Nq, d)) return ATTN_EUNSUPPORTED;
+  if (lse && !aligned16(lse)) return ATTN_EALIGN;
+  const int sms = current_sms();
+  if (sms <= 0) return ATTN_ECUDA;
+  const DecodePlan p = decode_plan(B, Hq, Hkv, Nq, d, sms);
+  if (!workspace || workspace_bytes < p.workspace_bytes) return ATTN_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
+  DecodeMask mk;
+  mk.causal = causal;
+  mk.window = window;
+  mk.align = 1;   // each sequence's query rows are its newest tokens
+  PagedKv pg;
+  pg.block_table = block_table;
+  pg.max_pages = max_pages;
+  pg.page_size = page_size;
+  pg.num_pages = num_pages;
+  return launch_decode(q, k_cache, v_cache, o, lse, B, Hq, Hkv, Nq, Nk, d, mk, &pg, scale,
+                       key_lens, workspace, p, static_cast<cudaStream_t>(stream));
 }
 
 int attn_fwd_window(const void* q, const void* k, const void* v, void* o, float* lse, int B,

@@ -24,7 +24,11 @@
 //
 // Head dimension 128 runs the tcgen05 split kernel of decode_tc.cu (same
 // work split and partial format); the mma.sync split kernel below serves
-// d = 64.
+// d = 64.  Both read either a contiguous cache or a paged one ("Attention
+// mechanisms ...", section 20: key j in block block_table[b][j / page_size]
+// at offset j % page_size); a paged tile starts on a page boundary and
+// arrives as one TMA box per page, pages past the segment's end coming from
+// a row past the cache (zero fill).
 //
 // Data movement.  K and V tiles of 64 keys arrive by TMA (2D tensor map over
 // the [B*Hkv*Nk, d] cache, 128-byte swizzle) into a 4-stage shared-memory ring
@@ -86,9 +90,12 @@ struct DecodeArgs {
   int Nq, R;                 // query rows per sequence, rows per unit (G * Nq)
   int causal, window, align;
   float scale_log2;
+  // paged cache (kPaged): Nk = max_pages * page_size
+  const int32_t* block_table;
+  int max_pages, page_size, oob_row;   // oob_row: first row past the cache
 };
 
-template <int D, int MT>
+template <int D, int MT, bool kPaged>
 __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
     decode_split_kernel(const __grid_constant__ CUtensorMap tmap_k,
                         const __grid_constant__ CUtensorMap tmap_v, DecodeArgs a) {
@@ -161,6 +168,11 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
     }
     u0 = lo;
   }
+  // first tile of a segment (relative to the unit's first key kl): its
+  // first key, or the start of the page holding it when the cache is paged
+  auto first_tile = [&](const Seg& s, int kl) -> int {
+    return kPaged ? s.lo - (kl + s.lo) % a.page_size : s.lo;
+  };
   auto next_seg = [&](int& u, Seg& s) -> bool {
     while (u < U) {
       const long long p0 = unit_prefix(pb, lens_s, u, Hkv);
@@ -178,32 +190,60 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
 
   if (warp == kConsumerWarps) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && start < end) {
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_v);
+    // Lane 0 waits on the ring and arms the stage's barrier; the loads are
+    // issued by lane 0 (contiguous cache) or by lane p for page p of the
+    // tile (paged: each lane reads its block-table entry one tile ahead).
+    if (start < end) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+      }
       int u = u0, it = 0;
       Seg s;
       bool ok = true;
+      const int npg = kPaged ? kTileKeys / a.page_size : 1;
+      const bool issuer = kPaged ? lane < npg : lane == 0;
       while (ok && next_seg(u, s)) {
-        for (int t = s.lo; t < s.hi; t += kTileKeys, ++it) {
+        const int b = s.u / Hkv, h = s.u - b * Hkv, kl = lo_s[b];
+        const int32_t* table = kPaged ? a.block_table + (size_t)b * a.max_pages : nullptr;
+        // paged: the cache row of this lane's page of the tile at t (or a row
+        // past the cache, which the TMA fills with zeros)
+        auto page_row = [&](int t) -> int {
+          const int pg = (kl + t) / a.page_size + lane;
+          return (lane < npg && pg * a.page_size < kl + s.hi)
+                     ? (table[pg] * Hkv + h) * a.page_size
+                     : a.oob_row;
+        };
+        const int t0 = first_tile(s, kl);
+        int prow = kPaged ? page_row(t0) : 0;
+        const int so = kPaged ? lane * a.page_size * 128 : 0;
+        for (int t = t0; t < s.hi; t += kTileKeys, ++it) {
           const int st = it % kStages;
           const uint32_t ph = (it / kStages) & 1;
-          if (!mbar_wait(&empty[st], ph ^ 1, abort_flag)) { ok = false; break; }
+          const int pnext = (kPaged && t + kTileKeys < s.hi) ? page_row(t + kTileKeys) : 0;
+          const int r = kPaged ? prow : s.u * a.Nk + kl + t;
+          bool w = true;
+          if (lane == 0) {
+            w = mbar_wait(&empty[st], ph ^ 1, abort_flag);
+            if (w) mbar_arrive_expect_tx(&full[st], L::kStageBytes);
+          }
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
           uint8_t* kt = smem + L::kRing + st * L::kStageBytes;
           uint8_t* vt = kt + L::kTileBytes;
-          mbar_arrive_expect_tx(&full[st], L::kStageBytes);
-          const int row = s.u * a.Nk + lo_s[s.u / Hkv] + t;
+          if (issuer) {
 #pragma unroll
-          for (int bx = 0; bx < kBoxes; ++bx) {
-            tma_load_2d(kt + bx * (kTileKeys * 128), &tmap_k, bx * 64, row, &full[st]);
-            tma_load_2d(vt + bx * (kTileKeys * 128), &tmap_v, bx * 64, row, &full[st]);
+            for (int bx = 0; bx < kBoxes; ++bx) {
+              tma_load_2d(kt + bx * (kTileKeys * 128) + so, &tmap_k, bx * 64, r, &full[st]);
+              tma_load_2d(vt + bx * (kTileKeys * 128) + so, &tmap_v, bx * 64, r, &full[st]);
+            }
           }
+          prow = pnext;
         }
       }
-      // drain: every issued stage must land before the CTA may exit
-      const int issued = it;
-      for (int j = issued - kStages > 0 ? issued - kStages : 0; j < issued; ++j)
-        mbar_wait(&full[j % kStages], (j / kStages) & 1, nullptr);
+      // drain: every armed stage must land before the CTA may exit
+      if (lane == 0)
+        for (int j = it - kStages > 0 ? it - kStages : 0; j < it; ++j)
+          mbar_wait(&full[j % kStages], (j / kStages) & 1, nullptr);
     }
     return;
   }
@@ -243,7 +283,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
 #pragma unroll
     for (int n = 0; n < D / 8; ++n) acc[n][0] = acc[n][1] = acc[n][2] = acc[n][3] = 0.f;
 
-    for (int t = s.lo; t < s.hi; t += kTileKeys, ++it) {
+    for (int t = first_tile(s, key_base); t < s.hi; t += kTileKeys, ++it) {
       const int st = it % kStages;
       if (!mbar_wait(&full[st], (it / kStages) & 1, abort_flag)) { alive = false; break; }
       const uint32_t kbase = smem_u32(smem + L::kRing + st * L::kStageBytes);
@@ -271,7 +311,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
 #pragma unroll
         for (int e = 0; e < 4; ++e) {
           const int key = kfirst + n * 8 + 2 * t4 + (e & 1);
-          bool vis = key < s.hi;
+          bool vis = key < s.hi && (!kPaged || key >= s.lo);
           if (row_masks) {   // causal among the new tokens, sliding window
             const int dlt = (e >> 1 ? pos1 : pos0) - (key_base + key);
             vis = vis && (!a.causal || dlt >= 0) &&
@@ -532,10 +572,10 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
 // ------------------------------------------------------------------ host side
 
 namespace {
-template <int D, int MT>
+template <int D, int MT, bool kPaged>
 int launch_decode_t(const DecodePlan& p, const CUtensorMap& tk, const CUtensorMap& tv,
                     const DecodeArgs& a, cudaStream_t st) {
-  auto kern = decode_split_kernel<D, MT>;
+  auto kern = decode_split_kernel<D, MT, kPaged>;
   const int smem = DecodeSmem<D>::kTotal;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ECUDA;
@@ -562,13 +602,10 @@ bool decode_supported(int B, int Hq, int Hkv, int Nq, int d) {
 }
 
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, float scale,
-                  const int32_t* key_lens, void* workspace, const DecodePlan& p,
+                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, const PagedKv* pg,
+                  float scale, const int32_t* key_lens, void* workspace, const DecodePlan& p,
                   cudaStream_t st) {
-  CUtensorMap tk, tv;
-  const uint64_t rows = (uint64_t)B * Hkv * Nk;
-  if (make_tmap_2d_bf16(&tk, k, d, rows, 64, kTileKeys) != ATTN_OK) return ATTN_ECUDA;
-  if (make_tmap_2d_bf16(&tv, v, d, rows, 64, kTileKeys) != ATTN_OK) return ATTN_ECUDA;
+  int rc;
   DecodeArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
   a.key_lens = key_lens;
@@ -578,20 +615,32 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   a.Nq = Nq; a.R = p.R;
   a.causal = mk.causal; a.window = mk.window; a.align = mk.align;
   a.scale_log2 = scale * kLog2e;
-  int rc;
-  if (decode_tc_supported(B, Hq, Hkv, Nq, d)) {
-    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nq, Nk, mk, scale, key_lens, a.part_o,
+  if (d == 128) {   // decode_supported ensures the tcgen05 kernel takes it
+    if (!decode_tc_supported(B, Hq, Hkv, Nq, d)) return ATTN_EUNSUPPORTED;
+    rc = launch_decode_split_tc(q, k, v, B, Hq, Hkv, Nq, Nk, mk, pg, scale, key_lens, a.part_o,
                                 a.part_lse, p.grid, st);
   } else {
+    // contiguous: [B * Hkv * Nk, d] in 64-row boxes; paged: [num_pages * Hkv *
+    // page_size, d] in page_size-row boxes
+    CUtensorMap tk, tv;
+    const uint64_t rows = pg ? (uint64_t)pg->num_pages * Hkv * pg->page_size
+                             : (uint64_t)B * Hkv * Nk;
+    const uint32_t box = pg ? (uint32_t)pg->page_size : (uint32_t)kTileKeys;
+    if (make_tmap_2d_bf16(&tk, k, d, rows, 64, box) != ATTN_OK) return ATTN_ECUDA;
+    if (make_tmap_2d_bf16(&tv, v, d, rows, 64, box) != ATTN_OK) return ATTN_ECUDA;
+    a.block_table = pg ? pg->block_table : nullptr;
+    a.max_pages = pg ? pg->max_pages : 0;
+    a.page_size = pg ? pg->page_size : 0;
+    a.oob_row = (int)rows;
     const int MT = (p.R + 15) / 16;
-    if (d == 128) {
-      rc = MT == 1 ? launch_decode_t<128, 1>(p, tk, tv, a, st)
-         : MT == 2 ? launch_decode_t<128, 2>(p, tk, tv, a, st)
-                   : launch_decode_t<128, 4>(p, tk, tv, a, st);
+    if (pg) {
+      rc = MT == 1 ? launch_decode_t<64, 1, true>(p, tk, tv, a, st)
+         : MT == 2 ? launch_decode_t<64, 2, true>(p, tk, tv, a, st)
+                   : launch_decode_t<64, 4, true>(p, tk, tv, a, st);
     } else {
-      rc = MT == 1 ? launch_decode_t<64, 1>(p, tk, tv, a, st)
-         : MT == 2 ? launch_decode_t<64, 2>(p, tk, tv, a, st)
-                   : launch_decode_t<64, 4>(p, tk, tv, a, st);
+      rc = MT == 1 ? launch_decode_t<64, 1, false>(p, tk, tv, a, st)
+         : MT == 2 ? launch_decode_t<64, 2, false>(p, tk, tv, a, st)
+                   : launch_decode_t<64, 4, false>(p, tk, tv, a, st);
     }
   }
   if (rc != ATTN_OK) return rc;

@@ -85,7 +85,7 @@ int attn_fwd_decode_static(const void* q, const void* k, const void* v, void* o,
   void* scratch = nullptr;
   const int rc = scratch_address(&scratch);
   if (rc != ATTN_OK) return rc;
-  return launch_decode(q, k, v, o, lse, B, Hq, Hkv, 1, Nk, d, DecodeMask(), scale, key_lens,
+  return launch_decode(q, k, v, o, lse, B, Hq, Hkv, 1, Nk, d, DecodeMask(), nullptr, scale, key_lens,
                        scratch, p, static_cast<cudaStream_t>(stream));
 }
 

@@ -21,6 +21,15 @@
 //
 // Warp roles: warps 0-3 softmax (TMEM lane quarters 0-3), warp 4 MMA issuer
 // and TMEM allocator, warp 5 TMA producer.
+//
+// Paged KV cache ("Attention mechanisms ...", section 20; "Transformer
+// internals", PagedAttention): key j of a sequence lives in physical block
+// block_table[b][j / page_size] at offset j % page_size (cache [num_pages,
+// Hkv, page_size, d]).  A 128-key tile starts on a page boundary and arrives
+// as 128 / page_size TMA boxes of page_size rows, one per page, into the same
+// swizzled tile layout; pages past the segment's end are loaded from a row
+// past the cache (the TMA fills zeros), so unused table entries are never
+// read.  Keys of the tile outside the segment are masked.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -76,7 +85,9 @@ struct Smem {
 };
 
 struct Seg {
-  int u, lo, hi;
+  int u, lo, hi;      // unit and its keys [lo, hi), relative to the unit's first key
+  int start, end;     // the same keys as absolute key indices of the sequence
+  int base, n;        // first key of tile 0 (page-aligned when paged), tiles
 };
 
 __device__ __forceinline__ long long unit_prefix(const long long* pb, const int* lens, int u,
@@ -182,9 +193,12 @@ struct DecodeTcArgs {
   int Nq, R;                 // query rows per sequence, rows per unit (G * Nq)
   int causal, window, align;
   float scale_log2;
+  // paged cache (kernel instantiation with kPaged): Nk = max_pages * page_size
+  const int32_t* block_table;
+  int max_pages, page_size, oob_row;   // oob_row: first row past the cache
 };
 
-template <int N>
+template <int N, bool kPaged>
 __global__ void __launch_bounds__(192, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
@@ -273,6 +287,11 @@ __global__ void __launch_bounds__(192, 1)
       const int cur = u++;
       if (hi > lo) {
         s.u = cur; s.lo = (int)(lo - p0); s.hi = (int)(hi - p0);
+        const int kl = lo_s[cur / Hkv];
+        s.start = kl + s.lo;
+        s.end = kl + s.hi;
+        s.base = kPaged ? s.start - s.start % a.page_size : s.start;
+        s.n = (s.end - s.base + kTile - 1) / kTile;
         return true;
       }
     }
@@ -281,43 +300,84 @@ __global__ void __launch_bounds__(192, 1)
 
   if (warp == 5) {
     // ------------------------------------------------------------ producer
-    if (lane == 0 && start < end) {
-      tma_prefetch_desc(&tmap_q);
-      tma_prefetch_desc(&tmap_k);
-      tma_prefetch_desc(&tmap_v);
+    // Lane 0 waits on the rings and arms the barriers.  The K/V loads of a
+    // tile are issued by lane 0 (contiguous cache) or by lane p for page p of
+    // the tile (paged: each lane reads its own block-table entry one tile
+    // ahead, so the reads overlap and the code stays small).
+    if (start < end) {
+      if (lane == 0) {
+        tma_prefetch_desc(&tmap_q);
+        tma_prefetch_desc(&tmap_k);
+        tma_prefetch_desc(&tmap_v);
+      }
       int u = u0, g = 0, qn = 0;
+      int gk = 0, gv = 0;   // K and V tiles whose barriers were armed (for the drain)
       Seg s;
       bool ok = true;
+      const int npg = kPaged ? kTile / a.page_size : 1;
+      const bool issuer = kPaged ? lane < npg : lane == 0;
       while (ok && next_seg(u, s)) {
         const int b = s.u / Hkv, h = s.u - b * Hkv;
-        const int n = (s.hi - s.lo + kTile - 1) / kTile;
-        if (qn > 0 && !mbar_wait(&bars[L::Q_EMPTY], (qn - 1) & 1, abort_flag)) break;
+        const int n = s.n;
+        bool w = true;
+        if (lane == 0) {
+          w = qn == 0 || mbar_wait(&bars[L::Q_EMPTY], (qn - 1) & 1, abort_flag);
+          if (w) {
+            mbar_arrive_expect_tx(&bars[L::Q_FULL], 2 * L::kQBox);
+            for (int bx = 0; bx < 2; ++bx)
+              tma_load_2d(smem + L::kQ + bx * L::kQBox, &tmap_q, bx * 64,
+                          (b * a.Hq + h * a.G) * a.Nq, &bars[L::Q_FULL]);
+          }
+        }
+        if (!__shfl_sync(0xffffffffu, w, 0)) break;
         ++qn;
-        mbar_arrive_expect_tx(&bars[L::Q_FULL], 2 * L::kQBox);
-        for (int bx = 0; bx < 2; ++bx)
-          tma_load_2d(smem + L::kQ + bx * L::kQBox, &tmap_q, bx * 64,
-                      (b * a.Hq + h * a.G) * a.Nq, &bars[L::Q_FULL]);
-        const int row0 = s.u * a.Nk + lo_s[b] + s.lo;
+        const int row0 = s.u * a.Nk + s.base;   // contiguous cache
+        const int32_t* table = kPaged ? a.block_table + (size_t)b * a.max_pages : nullptr;
+        // paged: the cache row of this lane's page of tile j (or a row past
+        // the cache, which the TMA fills with zeros)
+        auto page_row = [&](int j) -> int {
+          const int pg = (s.base + j * kTile) / a.page_size + lane;
+          return (lane < npg && pg * a.page_size < s.end) ? (table[pg] * Hkv + h) * a.page_size
+                                                          : a.oob_row;
+        };
+        int prow = kPaged ? page_row(0) : 0;
+        const uint32_t so = kPaged ? (uint32_t)(lane * a.page_size * 128) : 0u;
         for (int j = 0; j < n; ++j, ++g) {
           const int ks = g % KS, vs = g % VS;
-          if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / KS) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kKV);
-          for (int bx = 0; bx < 2; ++bx)
-            tma_load_2d(smem + L::kK + ks * L::kKV + bx * L::kBox, &tmap_k, bx * 64,
-                        row0 + j * kTile, &bars[L::K_FULL + ks]);
-          if (!mbar_wait(&bars[L::V_EMPTY + vs], ((g / VS) & 1) ^ 1, abort_flag)) { ok = false; break; }
-          mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kKV);
-          for (int bx = 0; bx < 2; ++bx)
-            tma_load_2d(smem + L::kV + vs * L::kKV + bx * L::kBox, &tmap_v, bx * 64,
-                        row0 + j * kTile, &bars[L::V_FULL + vs]);
+          const int pnext = (kPaged && j + 1 < n) ? page_row(j + 1) : 0;
+          const int r = kPaged ? prow : row0 + j * kTile;
+          if (lane == 0) {
+            w = mbar_wait(&bars[L::K_EMPTY + ks], ((g / KS) & 1) ^ 1, abort_flag);
+            if (w) mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kKV);
+          }
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+          ++gk;
+          if (issuer)
+            for (int bx = 0; bx < 2; ++bx)
+              tma_load_2d(smem + L::kK + ks * L::kKV + bx * L::kBox + so, &tmap_k, bx * 64, r,
+                          &bars[L::K_FULL + ks]);
+          if (lane == 0) {
+            w = mbar_wait(&bars[L::V_EMPTY + vs], ((g / VS) & 1) ^ 1, abort_flag);
+            if (w) mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kKV);
+          }
+          if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
+          ++gv;
+          if (issuer)
+            for (int bx = 0; bx < 2; ++bx)
+              tma_load_2d(smem + L::kV + vs * L::kKV + bx * L::kBox + so, &tmap_v, bx * 64, r,
+                          &bars[L::V_FULL + vs]);
+          prow = pnext;
         }
       }
-      // every issued load must land before the CTA may exit
-      for (int j = g - KS > 0 ? g - KS : 0; j < g; ++j)
-        mbar_wait(&bars[L::K_FULL + j % KS], (j / KS) & 1, nullptr);
-      for (int j = g - VS > 0 ? g - VS : 0; j < g; ++j)
-        mbar_wait(&bars[L::V_FULL + j % VS], (j / VS) & 1, nullptr);
-      if (qn > 0) mbar_wait(&bars[L::Q_FULL], (qn - 1) & 1, nullptr);
+      // every issued load must land before the CTA may exit (counted per
+      // ring: a K tile whose V slot never freed was still armed and loaded)
+      if (lane == 0) {
+        for (int j = gk - KS > 0 ? gk - KS : 0; j < gk; ++j)
+          mbar_wait(&bars[L::K_FULL + j % KS], (j / KS) & 1, nullptr);
+        for (int j = gv - VS > 0 ? gv - VS : 0; j < gv; ++j)
+          mbar_wait(&bars[L::V_FULL + j % VS], (j / VS) & 1, nullptr);
+        if (qn > 0) mbar_wait(&bars[L::Q_FULL], (qn - 1) & 1, nullptr);
+      }
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
@@ -348,7 +408,7 @@ __global__ void __launch_bounds__(192, 1)
       Seg s;
       bool ok = true;
       while (ok && next_seg(u, s)) {
-        const int n = (s.hi - s.lo + kTile - 1) / kTile;
+        const int n = s.n;
         if (!mbar_wait(&bars[L::Q_FULL], qf & 1, abort_flag)) break;
         ++qf;
         for (int t = 0; t < 2 && t < n && ok; ++t) {
@@ -391,12 +451,11 @@ __global__ void __launch_bounds__(192, 1)
     Seg s;
     bool ok = start < end;
     while (ok && next_seg(u, s)) {
-      const int n = (s.hi - s.lo + kTile - 1) / kTile;
-      // key index of segment position 0, and the rows' position offset
+      const int n = s.n;
+      // the rows' position offset
       const int sb = s.u / a.Hkv;
       const int Lb = clamp_len(a.key_lens ? a.key_lens[sb] : a.Nk, a.Nk);
       const int off = query_offset(a.Nq, a.Nk, Lb, a.align);
-      const int key0 = lo_s[sb] + s.lo;
       asm volatile("bar.sync 1, 128;" ::: "memory");   // previous segment done with m_s / l_s
       if (Lr < 64) m_s[Lr] = -INFINITY;
       float lp[N];
@@ -410,14 +469,14 @@ __global__ void __launch_bounds__(192, 1)
         float sv[N];
         tmem_ld_row<N>(tmem + lane_off + (uint32_t)(buf * N), sv);
         tc::wait_ld();
-        const bool valid = s.lo + j * kTile + Lr < s.hi;
+        const int kfirst = s.base + j * kTile;   // absolute key of this tile's row 0
+        const bool valid = kfirst + Lr < s.end && (!kPaged || kfirst + Lr >= s.start);
         if (!valid) {
 #pragma unroll
           for (int h = 0; h < N; ++h) sv[h] = -INFINITY;
         }
         // rows (tokens) that do not see every key of this tile: causal keys
         // past row 0's position, window keys before the last row's window
-        const int kfirst = key0 + j * kTile;
         const int klast = kfirst + kTile - 1;
         const bool tile_mask =
             (a.causal && klast > off) ||
@@ -547,10 +606,10 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 namespace {
-template <int N>
+template <int N, bool kPaged>
 int launch_tc_t(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                 const DecodeTcArgs& a, cudaStream_t st) {
-  auto kern = decode_tc_kernel<N>;
+  auto kern = decode_tc_kernel<N, kPaged>;
   const int smem = dtc::Smem<N>::kTotal;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ECUDA;
@@ -564,18 +623,26 @@ bool decode_tc_supported(int B, int Hq, int Hkv, int Nq, int d) {
 }
 
 int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                           int Nq, int Nk, const DecodeMask& mk, float scale,
+                           int Nq, int Nk, const DecodeMask& mk, const PagedKv* pg, float scale,
                            const int32_t* key_lens, float* part_o, float* part_lse, int grid,
                            cudaStream_t st) {
   const int G = Hq / Hkv, R = G * Nq;
   const int N = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
   CUtensorMap tq, tk, tv;
-  const uint64_t rows = (uint64_t)B * Hkv * Nk;
+  // contiguous: [B * Hkv * Nk, d] in 128-row boxes; paged: [num_pages * Hkv *
+  // page_size, d] in page_size-row boxes
+  const uint64_t rows = pg ? (uint64_t)pg->num_pages * Hkv * pg->page_size
+                           : (uint64_t)B * Hkv * Nk;
+  const uint32_t box = pg ? (uint32_t)pg->page_size : (uint32_t)dtc::kTile;
   if (make_tmap_2d_bf16(&tq, q, dtc::kD, (uint64_t)B * Hq * Nq, 64, (uint32_t)N) != ATTN_OK)
     return ATTN_ECUDA;
-  if (make_tmap_2d_bf16(&tk, k, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
-  if (make_tmap_2d_bf16(&tv, v, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
+  if (make_tmap_2d_bf16(&tk, k, dtc::kD, rows, 64, box) != ATTN_OK) return ATTN_ECUDA;
+  if (make_tmap_2d_bf16(&tv, v, dtc::kD, rows, 64, box) != ATTN_OK) return ATTN_ECUDA;
   DecodeTcArgs a;
+  a.block_table = pg ? pg->block_table : nullptr;
+  a.max_pages = pg ? pg->max_pages : 0;
+  a.page_size = pg ? pg->page_size : 0;
+  a.oob_row = (int)rows;
   a.key_lens = key_lens;
   a.part_o = part_o;
   a.part_lse = part_lse;
@@ -583,9 +650,14 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   a.Nq = Nq; a.R = R;
   a.causal = mk.causal; a.window = mk.window; a.align = mk.align;
   a.scale_log2 = scale * kLog2e;
-  if (N == 16) return launch_tc_t<16>(grid, tq, tk, tv, a, st);
-  if (N == 32) return launch_tc_t<32>(grid, tq, tk, tv, a, st);
-  return launch_tc_t<64>(grid, tq, tk, tv, a, st);
+  if (pg) {
+    if (N == 16) return launch_tc_t<16, true>(grid, tq, tk, tv, a, st);
+    if (N == 32) return launch_tc_t<32, true>(grid, tq, tk, tv, a, st);
+    return launch_tc_t<64, true>(grid, tq, tk, tv, a, st);
+  }
+  if (N == 16) return launch_tc_t<16, false>(grid, tq, tk, tv, a, st);
+  if (N == 32) return launch_tc_t<32, false>(grid, tq, tk, tv, a, st);
+  return launch_tc_t<64, false>(grid, tq, tk, tv, a, st);
 }
 
 }  // namespace attn

@@ -35,19 +35,27 @@ struct DecodePlan {
 struct DecodeMask {
   int causal = 0, window = 0, align = 0;
 };
+// Paged KV cache: cache [num_pages, Hkv, page_size, d]; key j of sequence b
+// is row j % page_size of block block_table[b * max_pages + j / page_size].
+struct PagedKv {
+  const int32_t* block_table = nullptr;
+  int max_pages = 0, page_size = 0, num_pages = 0;
+};
 DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int d, int num_sms);
 bool decode_supported(int B, int Hq, int Hkv, int Nq, int d);
 // tcgen05 split kernel (d == 128, up to 64 query rows per kv head); writes
 // the same partial-result format as the mma.sync split kernel.
 bool decode_tc_supported(int B, int Hq, int Hkv, int Nq, int d);
 int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, int Hq, int Hkv,
-                           int Nq, int Nk, const DecodeMask& mk, float scale,
+                           int Nq, int Nk, const DecodeMask& mk, const PagedKv* pg, float scale,
                            const int32_t* key_lens, float* part_o, float* part_lse, int grid,
                            cudaStream_t st);
 // Each sequence's units read keys [lo, L) (decode_key_range in tile_plan.cuh).
+// pg == nullptr: contiguous k/v [B, Hkv, Nk, d]; else a paged cache with
+// Nk = max_pages * page_size.
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, float scale,
-                  const int32_t* key_lens, void* workspace, const DecodePlan& p,
+                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, const PagedKv* pg,
+                  float scale, const int32_t* key_lens, void* workspace, const DecodePlan& p,
                   cudaStream_t st);
 
 // ---- prefill (Nq > 1)

@@ -146,3 +146,42 @@ def sample_rows(w: Workload, per_head_random: int = 55, seed_offset: int = 5) ->
         rows.update(int(x) for x in rng.integers(0, N, size=per_head_random))
         out.extend(bh * N + r for r in sorted(rows))
     return np.array(out, dtype=np.int64)
+
+
+def paged_layout(key_lens, page_size: int, seed: int, spare_pages: int = 3,
+                 shuffle: bool = True):
+    """A seeded paged-cache layout for sequences of the given lengths: each
+    sequence gets ceil(L / page_size) physical pages drawn in random order
+    (or in order, shuffle=False) from a pool with `spare_pages` unused ones.
+    Returns (block_table int32 [B, max_pages] with -1 in unused entries,
+    num_pages)."""
+    kl = np.asarray(key_lens, np.int64)
+    need = [int(-(-int(n) // page_size)) for n in kl]
+    max_pages = max(1, max(need))
+    num_pages = sum(need) + spare_pages
+    rng = np.random.Generator(np.random.PCG64(seed))
+    perm = rng.permutation(num_pages) if shuffle else np.arange(num_pages)
+    table = np.full((len(kl), max_pages), -1, np.int32)
+    at = 0
+    for b, n in enumerate(need):
+        table[b, :n] = perm[at:at + n]
+        at += n
+    return table, num_pages
+
+
+def to_paged(x, block_table, key_lens, num_pages: int, page_size: int, fill_bits: int):
+    """Copy a contiguous cache [B, Hkv, Nk, d] (bf16 bits) into a paged one
+    [num_pages, Hkv, page_size, d]: key j of sequence b goes to block
+    block_table[b, j // page_size], row j % page_size.  Rows of a sequence's
+    last page past its length keep x's values there (x's padding) or, past
+    Nk, the finite PAD_SENTINEL; pages no sequence owns hold `fill_bits`."""
+    B, Hkv, Nk, d = x.shape
+    out = np.full((num_pages, Hkv, page_size, d), fill_bits, np.uint16)
+    pad = bf16_bits_from_f32(np.array([PAD_SENTINEL], np.float32))[0]
+    for b in range(B):
+        n = int(-(-int(key_lens[b]) // page_size))
+        for p in range(n):
+            j0, j1 = p * page_size, min((p + 1) * page_size, Nk)
+            out[block_table[b, p]] = pad
+            out[block_table[b, p], :, :j1 - j0, :] = x[b, :, j0:j1, :]
+    return out

@@ -118,6 +118,32 @@ ATTN_API int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, f
                          int window, int align, float scale, const int32_t* key_lens,
                          void* workspace, size_t workspace_bytes, void* stream);
 
+/* Decode over a paged KV cache ("Attention mechanisms ...", section 20;
+ * "Transformer internals", PagedAttention): logical key j of kv head h of
+ * sequence b lives in physical block p = block_table[b * max_pages +
+ * j / page_size], row j % page_size:
+ *     k_cache, v_cache  bf16 [num_pages, Hkv, page_size, d]   (DEVICE)
+ *     block_table       int32 [B, max_pages]                  (DEVICE)
+ *     key_lens          int32 [B], required (DEVICE): sequence lengths
+ *   q/o bf16 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq] or NULL.  The Nq query rows
+ *   of a sequence are its newest Nq tokens (ATTN_ALIGN_KEYLEN of attn_fwd_ex);
+ *   causal and window as there, with Nk = max_pages * page_size.
+ *   Runs the split-KV decode kernels: (Hq / Hkv) * Nq <= 64.  page_size: a
+ *   multiple of 8 dividing 128 (d = 128) or 64 (d = 64) -- 8, 16, 32, 64
+ *   (and 128 for d = 128).  Only entries j / page_size < ceil(key_lens[b] /
+ *   page_size) of a sequence's table row are read; rows of its last page at
+ *   or beyond key_lens[b] must hold finite values.  A table entry outside
+ *   [0, num_pages) reads zeros (the kernels do not check it).
+ *   Workspace: attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) bytes.
+ * Errors: ATTN_EINVAL (null table or key_lens, bad sizes), ATTN_EUNSUPPORTED
+ * (page_size, more than 64 query rows per kv head, d), then as attn_fwd_ws. */
+ATTN_API int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
+                            const int32_t* block_table, int max_pages, int page_size,
+                            int num_pages, void* o, float* lse, int B, int Hq, int Hkv,
+                            int Nq, int d, int causal, int window, float scale,
+                            const int32_t* key_lens, void* workspace,
+                            size_t workspace_bytes, void* stream);
+
 /* attn_fwd_ex with align = ATTN_ALIGN_NK: sliding-window attention. */
 ATTN_API int attn_fwd_window(const void* q, const void* k, const void* v, void* o,
                              float* lse, int B, int Hq, int Hkv, int Nq, int Nk, int d,

@@ -144,3 +144,23 @@ def test_ex_entry_points_reject_bad_arguments_on_host(L):
     t = L.attn_fwd_tile_plan_ex
     assert t(1, 8, 8, 64, 1, 0, 2, None, P, P, None) == 1
     assert t(1, 8, 8, 64, 1, 0, 1, None, None, P, None) == 1
+
+
+def test_paged_rejects_bad_arguments_on_host(L):
+    f = L.attn_fwd_paged
+    # q, k_cache, v_cache, table, max_pages, page_size, num_pages, o, lse, B, Hq, Hkv, Nq,
+    # d, causal, window, scale, key_lens, workspace, bytes, stream
+    assert f(P, P, P, None, 4, 16, 8, P, None, 1, 4, 1, 1, 128, 1, 0, 0.1, P, P, 1 << 20,
+             None) == 1                                      # no block table
+    assert f(P, P, P, P, 4, 16, 8, P, None, 1, 4, 1, 1, 128, 1, 0, 0.1, None, P, 1 << 20,
+             None) == 1                                      # no key lengths
+    assert f(P, P, P, P, 4, 12, 8, P, None, 1, 4, 1, 1, 128, 1, 0, 0.1, P, P, 1 << 20,
+             None) == 2                                      # page size not a multiple of 8
+    assert f(P, P, P, P, 2, 256, 8, P, None, 1, 4, 1, 1, 128, 1, 0, 0.1, P, P, 1 << 20,
+             None) == 2                                      # page larger than a tile
+    assert f(P, P, P, P, 4, 128, 8, P, None, 1, 4, 1, 1, 64, 1, 0, 0.1, P, P, 1 << 20,
+             None) == 2                                      # d = 64 tiles hold 64 keys
+    assert f(P, P, P, P, 4, 16, 8, P, None, 1, 64, 1, 2, 128, 1, 0, 0.1, P, P, 1 << 20,
+             None) == 2                                      # 128 query rows per kv head
+    assert f(P, P, P, P, 4, 16, 8, P, None, 1, 4, 1, 1, 128, 1, -1, 0.1, P, P, 1 << 20,
+             None) == 1                                      # negative window
