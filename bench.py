@@ -47,12 +47,12 @@ L2_BYTES = 126 * 1024 * 1024
 # reported only while the sources still hash the same.
 KERNEL_SOURCES = {
     "prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
-    "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh"],
+    "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
 }
 NCU_TRAFFIC = {
     # workload: (kernel, source hash, bytes per launch)
-    "mha_prefill": ("prefill", "9389efd25a7c3dc7", 128126976 + 10136832),
-    "mqa_decode": ("decode", "33944cc49cb39b44", 324087552 + 6830592),
+    "mha_prefill": ("prefill", "6191a56c605c70b0", 124861952 + 10512384),
+    "mqa_decode": ("decode", "bad510b57056b510", 324108032 + 4244480),
 }
 
 

@@ -47,8 +47,13 @@ constexpr float kRescaleLog2 = 8.0f;
 
 template <int N>
 struct Smem {
-  static constexpr int KS = N <= 32 ? 3 : 2;   // K ring stages
-  static constexpr int VS = 2;                 // V ring stages
+  // Ring depths.  A K slot frees as soon as its S MMA has run, a V slot only
+  // after the softmax of its tile and the PV MMA, so V needs the deeper ring
+  // to keep enough loads in flight (two V slots held the producer waiting on
+  // V for half of the kernel at 32 heads).  At N = 64 the larger Q and P
+  // buffers leave room for two of each.
+  static constexpr int KS = 2;                 // K ring stages
+  static constexpr int VS = N <= 32 ? 3 : 2;   // V ring stages
   static constexpr int kKV = kTile * kD * 2;   // one K or V tile (32 KB)
   static constexpr int kBox = kTile * 128;     // 64-column box of a K/V tile
   static constexpr int kQBox = N * 128;        // 64-column box of Q (N rows)
@@ -57,8 +62,8 @@ struct Smem {
   static constexpr int kV = kK + KS * kKV;
   static constexpr int kQ = kV + VS * kKV;
   static constexpr int kP = kQ + 2 * kQBox;    // P^T [2 buffers][2 boxes]
-  static constexpr int kScan = kP + 4 * kPBox; // int64 [kMaxB + 1]
-  static constexpr int kLens = kScan + (kMaxB + 1) * 8;   // int [kMaxB] keys per unit
+  static constexpr int kScan = kP + 4 * kPBox; // int [kMaxB + 1] key prefix over b
+  static constexpr int kLens = kScan + (kMaxB + 1) * 4 + 4;   // int [kMaxB] keys per unit
   static constexpr int kLo = kLens + kMaxB * 4;            // int [kMaxB] first key
   static constexpr int kRed = kLo + kMaxB * 4;     // float [4][64]
   static constexpr int kMs = kRed + 4 * 64 * 4;    // float [64] running max (log2 units)
@@ -90,7 +95,8 @@ struct Seg {
   int base, n;        // first key of tile 0 (page-aligned when paged), tiles
 };
 
-__device__ __forceinline__ long long unit_prefix(const long long* pb, const int* lens, int u,
+// (B * Hkv * Nk < 2^31 is checked on the host, so every prefix fits an int.)
+__device__ __forceinline__ long long unit_prefix(const int* pb, const int* lens, int u,
                                                  int Hkv) {
   const int b = u / Hkv, h = u - b * Hkv;
   return (long long)Hkv * pb[b] + (long long)h * lens[b];
@@ -136,6 +142,25 @@ __device__ __forceinline__ void bfly_reduce(float (&v)[N], int lane) {
     const float o = __shfl_xor_sync(0xffffffffu, v[0], 16);
     v[0] = SUM ? v[0] + o : fmaxf(v[0], o);
   }
+}
+
+// Per-head maximum over the warp's 32 keys into red[warp][head]: one
+// warp-wide f32 max reduction (redux.sync) per head; lane h & 31 keeps the
+// result of head h and stores it.
+template <int N>
+__device__ __forceinline__ void col_max_to_red(float* red, int warp, int lane,
+                                               const float (&v)[N]) {
+  float mine[N > 32 ? 2 : 1];
+#pragma unroll
+  for (int i = 0; i < (N > 32 ? 2 : 1); ++i) mine[i] = -INFINITY;
+#pragma unroll
+  for (int h = 0; h < N; ++h) {
+    float r;
+    asm volatile("redux.sync.max.f32 %0, %1, 0xffffffff;" : "=f"(r) : "f"(v[h]));
+    if ((h & 31) == lane) mine[h >> 5] = r;
+  }
+  if (N >= 32 || lane < N) red[warp * 64 + lane] = mine[0];
+  if (N > 32) red[warp * 64 + 32 + lane] = mine[N > 32 ? 1 : 0];
 }
 
 // Store this warp's reduced values into red[warp][head].
@@ -212,7 +237,7 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  long long* pb = reinterpret_cast<long long*>(smem + L::kScan);
+  int* pb = reinterpret_cast<int*>(smem + L::kScan);
   int* lens_s = reinterpret_cast<int*>(smem + L::kLens);
   int* lo_s = reinterpret_cast<int*>(smem + L::kLo);
   float* red = reinterpret_cast<float*>(smem + L::kRed);
@@ -239,7 +264,7 @@ __global__ void __launch_bounds__(192, 1)
   }
   // key lengths (clamped) and their exclusive prefix over b, by warp 5
   if (warp == 5) {
-    long long carry = 0;
+    int carry = 0;
     for (int base = 0; base < B; base += 32) {
       const int b = base + lane;
       int len = 0;
@@ -250,10 +275,10 @@ __global__ void __launch_bounds__(192, 1)
         lens_s[b] = len;   // keys [lo, L) of every unit of sequence b
         lo_s[b] = lo;
       }
-      long long x = len;
+      int x = len;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
-        const long long y = __shfl_up_sync(0xffffffffu, x, o);
+        const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
       if (b < B) pb[b] = carry + x - len;
@@ -502,11 +527,7 @@ __global__ void __launch_bounds__(192, 1)
         }
         // per-head max over the tile's keys
         {
-          float v[N];
-#pragma unroll
-          for (int h = 0; h < N; ++h) v[h] = sv[h];
-          bfly_reduce<N, false>(v, lane);
-          put_red<N>(red, warp, lane, v);
+          col_max_to_red<N>(red, warp, lane, sv);
         }
         if (*abort_flag) { ok = false; break; }
         asm volatile("bar.sync 1, 128;" ::: "memory");
