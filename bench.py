@@ -16,7 +16,9 @@ The JSON line also carries: the roofline of the dominant kernel, the
 end-to-end figure through the public API with host buffers, the oracle timed
 on host cores (rank 0, N=1, bounded sample), SM clocks sampled during the
 timed region, the decode workload (MQA over a ragged KV cache) in GB/s, and
-the sliding-window prefill workload in useful TFLOP/s.
+the sliding-window prefill workload in useful TFLOP/s, the multi-token and
+paged decode workloads, and the GQA RoPE prefill step with separate RoPE
+passes and with q's RoPE fused into the attention kernel.
 """
 from __future__ import annotations
 
@@ -87,6 +89,7 @@ def parse_args():
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-window", action="store_true")
+    p.add_argument("--no-rope", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
@@ -308,7 +311,9 @@ def run_ours(args):
 
     def step(i):
         # one pass of the whole path: the RoPE prologue (when the workload has
-        # one) rotates Q and K, then the attention forward
+        # one) rotates Q and K in two rope_apply passes -- measured faster than
+        # the fused rotation of Q (the bench's rope_prefill object has both) --
+        # then the attention forward
         if w.rope:
             c = i % copies
             eb.rope_apply(Q[c], base=synth.ROPE_BASE, pairing=synth.ROPE_PAIRING_HALF, out=QR)
@@ -399,6 +404,9 @@ def run_ours(args):
     # ---- sliding-window prefill, same run
     if not args.no_window and w.name != "long_window" and rank == 0 and world == 1:
         line["window"] = run_window(torch, eb, device, stream, peaks, peak_src)
+    # ---- GQA prefill with RoPE: separate RoPE passes vs q's RoPE fused
+    if not args.no_rope and not w.rope and rank == 0 and world == 1:
+        line["rope_prefill"] = run_rope(torch, eb, device, stream, peaks, peak_src)
 
     # ---- oracle on host cores (rank 0, N=1 only)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -466,6 +474,47 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa
                          "frac": gbs / peaks["hbm_gbs"],
                          "traffic": ncu_traffic(w.name), "peak_source": peak_src},
             "gpu_launches": 2 * n}
+
+
+def run_rope(torch, eb, device, stream, peaks, peak_src, steps=None):
+    """The GQA RoPE prefill step two ways (inputs larger than L2, one copy):
+    rope_apply on Q and K then attention, and rope_apply on K then attention
+    with q's RoPE fused in.  Useful FLOPs of the attention (4*B*Hq*N*N*d / 2)
+    over the whole step."""
+    w = synth.WORKLOADS["gqa_rope_prefill"]
+    x = synth.make_inputs(w)
+    q, k, v = (to_dev(x[n], torch, device) for n in ("q", "k", "v"))
+    qr, kr = torch.empty_like(q), torch.empty_like(k)
+    O = torch.empty_like(q)
+    LSE = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
+    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d),
+                     dtype=torch.uint8, device=device)
+    wsr = torch.empty(eb.lib().attn_rope_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d),
+                      dtype=torch.uint8, device=device)
+    rb, rp = synth.ROPE_BASE, synth.ROPE_PAIRING_HALF
+
+    def separate(i):
+        eb.rope_apply(q, base=rb, pairing=rp, out=qr)
+        eb.rope_apply(k, base=rb, pairing=rp, out=kr)
+        eb.attn_fwd_ws(qr, kr, v, ws, causal=True, scale=w.scale, out=O, lse=LSE)
+
+    def fused(i):
+        eb.rope_apply(k, base=rb, pairing=rp, out=kr)
+        eb.attn_fwd_rope(q, kr, v, causal=True, scale=w.scale, rope_base=rb, rope_pairing=rp,
+                         workspace=wsr, out=O, lse=LSE)
+
+    out = {"metric": "useful TFLOP/s of the whole step (RoPE + attention)", "unit": "TFLOP/s",
+           "workload": w.name}
+    for name, fn in (("separate", separate), ("fused_q", fused)):
+        for i in range(3):
+            fn(i)
+        probe = time_steps(fn, 2, torch, None, stream) / 2
+        n = steps or max(5, int(1000.0 / max(probe, 1e-3)))
+        ms = time_steps(fn, n, torch, None, stream)
+        out[name] = {"value": w.flops() * n / (ms / 1e3) / 1e12, "ms_per_step": ms / n,
+                     "steps": n, "gpu_launches": n * (3 if name == "separate" else 3)}
+    out["value"] = out["fused_q"]["value"]
+    return out
 
 
 def run_window(torch, eb, device, stream, peaks, peak_src, steps=None):

@@ -13,7 +13,7 @@ import ctypes
 import math
 import os
 
-__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_paged",
+__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_paged", "attn_fwd_rope",
            "attn_fwd_decode_static", "rope_apply",
            "prefill_tile_shape", "tile_plan", "device_status", "AttnError", "lib",
            "STATUS_NAMES"]
@@ -54,6 +54,11 @@ def lib():
         L.attn_fwd_paged.argtypes = [vp, vp, vp, vp, i, i, i, vp, vp, i, i, i, i, i, i, i, f, vp,
                                      vp, sz, vp]
         L.attn_fwd_paged.restype = i
+        L.attn_fwd_rope.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, f, i, i, vp, sz,
+                                    vp]
+        L.attn_fwd_rope.restype = i
+        L.attn_rope_workspace_size.argtypes = [i, i, i, i, i, i]
+        L.attn_rope_workspace_size.restype = sz
         L.attn_workspace_size.argtypes = [i, i, i, i, i, i]
         L.attn_workspace_size.restype = sz
         L.rope_apply.argtypes = [vp, vp, i, i, i, i, f, i, i, vp]
@@ -232,6 +237,36 @@ def attn_fwd_paged(q, k_cache, v_cache, block_table, key_lens, causal=True, scal
                               int(bool(causal)), int(window), float(scale), _ptr(key_lens),
                               _ptr(workspace), ws_bytes, _stream(stream))
     _raise(rc, "attn_fwd_paged")
+    return (out, lse) if return_lse else out
+
+
+def attn_fwd_rope(q, k_rot, v, causal=False, scale=None, key_lens=None, rope_base=10000.0,
+                  rope_pairing=0, q_pos_offset=0, workspace=None, out=None, lse=None,
+                  return_lse=True, stream=None):
+    """Attention with q's RoPE fused in: q un-rotated [B, Hq, Nq, d], k_rot
+    keys already rotated (rope_apply), v [B, Hkv, Nk, d]."""
+    torch = _torch()
+    for t, n in ((q, "q"), (k_rot, "k_rot"), (v, "v")):
+        _check_tensor(t, n, torch.bfloat16, 4)
+    B, Hq, Hkv, Nq, Nk, d = _shapes(q, k_rot, v)
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    if key_lens is not None:
+        _check_tensor(key_lens, "key_lens", torch.int32, 1)
+    if out is None:
+        out = torch.empty_like(q)
+    if return_lse and lse is None:
+        lse = torch.empty((B, Hq, Nq), dtype=torch.float32, device=q.device)
+    if workspace is None:
+        n = int(lib().attn_rope_workspace_size(B, Hq, Hkv, Nq, Nk, d))
+        workspace = torch.empty(max(n, 256), dtype=torch.uint8, device=q.device)
+    ws_bytes = workspace.numel() * workspace.element_size()
+    rc = lib().attn_fwd_rope(_ptr(q), _ptr(k_rot), _ptr(v), _ptr(out),
+                             _ptr(lse if return_lse else None), B, Hq, Hkv, Nq, Nk, d,
+                             int(bool(causal)), float(scale), _ptr(key_lens), float(rope_base),
+                             int(rope_pairing), int(q_pos_offset), _ptr(workspace), ws_bytes,
+                             _stream(stream))
+    _raise(rc, "attn_fwd_rope")
     return (out, lse) if return_lse else out
 
 

@@ -177,7 +177,51 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
   const int sms = current_sms();
   if (sms <= 0) return ATTN_ECUDA;
   return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, window, align, scale,
-                        key_lens, workspace, sms, st);
+                        key_lens, nullptr, 0, workspace, sms, st);
+}
+
+size_t attn_rope_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  const size_t base = attn_workspace_size(B, Hq, Hkv, Nq, Nk, d);
+  if (base == 0 || d <= 0) return 0;
+  // decode shapes: the rotated q; prefill: the (cos, sin) table of the rows
+  const size_t extra = decode_supported(B, Hq, Hkv, Nq, d)
+                           ? (size_t)B * Hq * Nq * d * 2
+                           : (size_t)Nq * (d / 2) * sizeof(float2);
+  return ((base + 255) & ~size_t(255)) + ((extra + 255) & ~size_t(255));
+}
+
+int attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                  int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                  const int32_t* key_lens, float rope_base, int rope_pairing, int q_pos_offset,
+                  void* workspace, size_t workspace_bytes, void* stream) {
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != ATTN_OK) return rc;
+  if (!std::isfinite(rope_base) || !(rope_base > 0.f)) return ATTN_EINVAL;
+  if (rope_pairing != 0 && rope_pairing != 1) return ATTN_EINVAL;
+  if (q_pos_offset < 0 || (long long)q_pos_offset + Nq > (1ll << 31) - 1) return ATTN_EINVAL;
+  if (lse && !aligned16(lse)) return ATTN_EALIGN;
+  const size_t need = attn_rope_workspace_size(B, Hq, Hkv, Nq, Nk, d);
+  if (need == 0) return ATTN_ECUDA;
+  if (!workspace || workspace_bytes < need) return ATTN_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
+  const size_t base = (attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) + 255) & ~size_t(255);
+  void* extra = static_cast<uint8_t*>(workspace) + base;
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (decode_supported(B, Hq, Hkv, Nq, d)) {
+    // decode shapes: rotate q into the workspace, then the decode kernels
+    rc = launch_rope(q, extra, B, Hq, Nq, d, rope_base, q_pos_offset, rope_pairing, st);
+    if (rc != ATTN_OK) return rc;
+    return attn_fwd_ws(extra, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens,
+                       workspace, base, stream);
+  }
+  if (!prefill_supported(d)) return ATTN_EUNSUPPORTED;
+  const int sms = current_sms();
+  if (sms <= 0) return ATTN_ECUDA;
+  float2* tab = static_cast<float2*>(extra);
+  rc = launch_rope_table(tab, Nq, d, rope_base, q_pos_offset, st);
+  if (rc != ATTN_OK) return rc;
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, 0, 0, scale, key_lens,
+                        tab, rope_pairing, workspace, sms, st);
 }
 
 int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,

@@ -64,13 +64,15 @@ size_t prefill_workspace_bytes();   // scheduler counter
 void prefill_tile_shape(int d, int* Br, int* Bc);
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
-                   float scale, const int32_t* key_lens, void* workspace, int num_sms,
-                   cudaStream_t st);
+                   float scale, const int32_t* key_lens, const float2* rope_tab,
+                   int rope_pairing, void* workspace, int num_sms, cudaStream_t st);
 int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window, int align,
                      const int32_t* key_lens, int32_t* first, int32_t* count, cudaStream_t st);
 
 // ---- RoPE
 int launch_rope(const void* x_in, void* x_out, int B, int H, int N, int d, float base,
                 int pos_offset, int pairing, cudaStream_t st);
+// (cos, sin) of positions pos_offset .. pos_offset + N - 1: tab[t * d/2 + i]
+int launch_rope_table(float2* tab, int N, int d, float base, int pos_offset, cudaStream_t st);
 
 }  // namespace attn

@@ -37,6 +37,14 @@
 // than 8 (log2 units); otherwise the stale max is kept (P <= 2^8, exact in
 // the final O / l because O and l share the same reference).
 //
+// Fused RoPE of Q (kRope instantiation): after a Q tile lands, the softmax
+// warpgroup of its slot -- idle until the tile's first scores exist --
+// rotates it in shared memory, one row per thread (row i at position
+// q_pos_offset + i, cos/sin from a table built for the call, the arithmetic
+// of rope_math.cuh), and releases it to the MMA issuer on Q_READY.  K is
+// expected rotated (a KV cache stores keys rotated once); rotating K here
+// would redo the work for every query tile that reads the K tile.
+//
 // Sliding window ("Attention mechanisms ...", section 11): a query tile
 // visits the contiguous KV-tile range that covers its rows' windows.  When
 // the two tiles of an item start at different KV tiles, both walk the union
@@ -48,6 +56,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "rope_math.cuh"
 #include "tcgen05.cuh"
 #include "tile_plan.cuh"
 
@@ -88,7 +97,8 @@ struct Smem {
     MMA_DONE = O_FULL + 2,
     ITEM_FULL = MMA_DONE + 1,            // [kItemSlots]
     ITEM_EMPTY = ITEM_FULL + kItemSlots, // [kItemSlots]
-    NUM_BARS = ITEM_EMPTY + kItemSlots
+    Q_READY = ITEM_EMPTY + kItemSlots,   // [2] rotated Q tile in place (fused RoPE)
+    NUM_BARS = Q_READY + 2
   };
   static constexpr int kItems = kBar + NUM_BARS * 8;      // int [kItemSlots]
   static constexpr int kTmemSlot = kItems + kItemSlots * 4;
@@ -118,6 +128,8 @@ struct FwdArgs {
   int B, Hq, Hkv, Nq, Nk, causal;
   int window;       // sliding window in keys, 0 = none
   int align;        // query positions: 0 end at key Nk - 1, 1 at key key_lens[b] - 1
+  const float2* rope_tab;   // fused RoPE of Q: (cos, sin) [Nq][d/2] (kRope)
+  int rope_pairing;         // 0: (i, i + d/2), 1: (2i, 2i + 1)
   int head_pairs;   // 1: tiles are heads (2p, 2p+1) at one row tile; 0: row tiles 2p, 2p+1
   int ntq;          // ceil(Nq / 128)
   int units;        // items per cost rank (head_pairs: B*Hq/2, else B*Hq)
@@ -210,7 +222,87 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window)
 
 }  // namespace pf
 
-template <int D, bool kWindow>
+// Rotate row r of the Q tile at `qs` (two or one 64-column boxes, 128-byte
+// swizzle) in place; `pos_row` indexes the (cos, sin) table.  Two 16-byte
+// chunks per step keep their table loads in flight together.
+template <int D>
+__device__ __forceinline__ void rope_q_row(uint8_t* qs, int r, int pos_row, const FwdArgs& a) {
+  constexpr int kBox = 128 * 128;
+  constexpr int kHalf = D / 2;
+  auto lo = [](uint32_t w) { return __uint_as_float(w << 16); };
+  auto hi = [](uint32_t w) { return __uint_as_float(w & 0xffff0000u); };
+  const float4* tab = reinterpret_cast<const float4*>(a.rope_tab + (size_t)pos_row * kHalf);
+  if (a.rope_pairing == 0) {
+    // half pairs (i, i + D/2): chunk c of the first half with chunk c of the
+    // second (D = 128: the same swizzled offset in the other box; D = 64:
+    // chunk c + 4 of the same row)
+#pragma unroll
+    for (int c0 = 0; c0 < D / 16; c0 += 2) {
+      uint4 va[2], vb[2];
+      float4 cs[2][4];   // (cos, sin) of pairs 8c .. 8c+7
+      uint8_t* pa[2];
+      uint8_t* pb[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = c0 + u;
+        pa[u] = qs + sw128_offset(r, c);
+        pb[u] = D == 128 ? pa[u] + kBox : qs + sw128_offset(r, c + 4);
+        va[u] = *reinterpret_cast<const uint4*>(pa[u]);
+        vb[u] = *reinterpret_cast<const uint4*>(pb[u]);
+#pragma unroll
+        for (int q = 0; q < 4; ++q) cs[u][q] = tab[4 * c + q];
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t wa[4] = {va[u].x, va[u].y, va[u].z, va[u].w};
+        const uint32_t wb[4] = {vb[u].x, vb[u].y, vb[u].z, vb[u].w};
+        uint32_t oa[4], ob[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          float ra0, rb0, ra1, rb1;
+          rope_rotate(lo(wa[k]), lo(wb[k]), make_float2(cs[u][k].x, cs[u][k].y), ra0, rb0);
+          rope_rotate(hi(wa[k]), hi(wb[k]), make_float2(cs[u][k].z, cs[u][k].w), ra1, rb1);
+          oa[k] = pack_bf16x2(ra0, ra1);
+          ob[k] = pack_bf16x2(rb0, rb1);
+        }
+        *reinterpret_cast<uint4*>(pa[u]) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
+        *reinterpret_cast<uint4*>(pb[u]) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
+      }
+    }
+  } else {
+    // adjacent pairs (2i, 2i + 1): 4 pairs per 16-byte chunk
+#pragma unroll
+    for (int c0 = 0; c0 < D / 8; c0 += 2) {
+      uint4 v[2];
+      float4 cs[2][2];   // (cos, sin) of pairs 4c .. 4c+3
+      uint8_t* p[2];
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = c0 + u;
+        p[u] = qs + (c >> 3) * kBox + sw128_offset(r, c & 7);
+        v[u] = *reinterpret_cast<const uint4*>(p[u]);
+        cs[u][0] = tab[2 * c];
+        cs[u][1] = tab[2 * c + 1];
+      }
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+        uint32_t o[4];
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 cc = cs[u][k >> 1];
+          const float2 c2 = (k & 1) ? make_float2(cc.z, cc.w) : make_float2(cc.x, cc.y);
+          float r0, r1;
+          rope_rotate(lo(w[k]), hi(w[k]), c2, r0, r1);
+          o[k] = pack_bf16x2(r0, r1);
+        }
+        *reinterpret_cast<uint4*>(p[u]) = make_uint4(o[0], o[1], o[2], o[3]);
+      }
+    }
+  }
+}
+
+template <int D, bool kWindow, bool kRope>
 __global__ void __launch_bounds__(pf::kThreads, 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, FwdArgs a) {
@@ -248,6 +340,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       uint32_t cnt = 1;
       if (i == L::P_FULL || i == L::P_FULL + 1) cnt = 128;
       if (i >= L::ITEM_EMPTY && i < L::ITEM_EMPTY + kItemSlots) cnt = kItemReaders;
+      if (i == L::Q_READY || i == L::Q_READY + 1) cnt = 128;   // a slot's softmax warpgroup
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -375,7 +468,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         return false;
       };
       auto issue_first_s = [&](const Counts& it, int t, int ks) -> bool {
-        if (!mbar_wait(&bars[L::Q_FULL + t], qf[t] & 1, abort_flag)) return false;
+        if (!mbar_wait(&bars[(kRope ? L::Q_READY : L::Q_FULL) + t], qf[t] & 1, abort_flag))
+          return false;
         ++qf[t];
         tc::fence_after();
         issue_s(t, ks);
@@ -445,13 +539,22 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t scol = 128u * t, ocol = 256u + D * t;
     const float sl2 = a.scale_log2;
-    int sw = 0, ow = 0, k = 0;
+    int sw = 0, ow = 0, k = 0, rq = 0;
     bool ok = true;
     for (int idx; ok && (idx = next_item(k)) >= 0;) {
       const Item it = make_item(a, idx, window);
       const Tile T = t == 0 ? it.tl[0] : it.tl[1];
       if (T.row_tile >= a.ntq) continue;
       const int row = T.row_tile * kM + r;
+      if constexpr (kRope) {
+        if (T.count > 0) {   // this slot loaded a Q tile for the item: rotate it
+          if (!mbar_wait(&bars[L::Q_FULL + t], rq & 1, abort_flag)) { ok = false; break; }
+          ++rq;
+          if (row < a.Nq) rope_q_row<D>(smem + L::kQ + t * L::kTile, r, row, a);
+          fence_proxy_async_smem();   // the tensor core reads what this thread wrote
+          mbar_arrive(&bars[L::Q_READY + t]);
+        }
+      }
       int vlo, vhi;   // this row's visible keys [vlo, vhi)
       visible_range(row, it.off, a.causal, it.L, window, &vlo, &vhi);
       float m_run = -INFINITY, l_run = 0.f;
@@ -620,8 +723,8 @@ void prefill_tile_shape(int d, int* Br, int* Bc) {
 
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
-                   float scale, const int32_t* key_lens, void* workspace, int num_sms,
-                   cudaStream_t st) {
+                   float scale, const int32_t* key_lens, const float2* rope_tab,
+                   int rope_pairing, void* workspace, int num_sms, cudaStream_t st) {
   CUtensorMap tq, tk, tv;
   if (make_tmap_3d_bf16(&tq, q, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tk, k, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
@@ -634,6 +737,8 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nq = Nq; a.Nk = Nk; a.causal = causal;
   a.window = window;
   a.align = align;
+  a.rope_tab = rope_tab;
+  a.rope_pairing = rope_pairing;
   a.ntq = (Nq + pf::kM - 1) / pf::kM;
   a.head_pairs = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
   a.scale_log2 = scale * kLog2e;
@@ -659,9 +764,15 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   if (cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) != cudaSuccess) return ATTN_ECUDA;
   // a window shifts each tile's first visible key: a separate instantiation
   // keeps that arithmetic out of the unwindowed kernel
-  const bool win = window > 0;
-  auto kern = d == 128 ? (win ? prefill_tc_kernel<128, true> : prefill_tc_kernel<128, false>)
-                       : (win ? prefill_tc_kernel<64, true> : prefill_tc_kernel<64, false>);
+  const bool win = window > 0, rope = rope_tab != nullptr;
+  using Kern = void (*)(CUtensorMap, CUtensorMap, CUtensorMap, FwdArgs);
+  Kern kern;
+  if (d == 128)
+    kern = rope ? (win ? prefill_tc_kernel<128, true, true> : prefill_tc_kernel<128, false, true>)
+                : (win ? prefill_tc_kernel<128, true, false> : prefill_tc_kernel<128, false, false>);
+  else
+    kern = rope ? (win ? prefill_tc_kernel<64, true, true> : prefill_tc_kernel<64, false, true>)
+                : (win ? prefill_tc_kernel<64, true, false> : prefill_tc_kernel<64, false, false>);
   const int smem = d == 128 ? pf::Smem<128>::kTotal : pf::Smem<64>::kTotal;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ECUDA;

@@ -15,6 +15,7 @@
 
 #include "common.cuh"
 #include "kernels.h"
+#include "rope_math.cuh"
 
 namespace attn {
 
@@ -46,12 +47,9 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(RopeArgs a) {
   float* sn = tab + kPos * half;
   for (int idx = threadIdx.x; idx < npos * half; idx += blockDim.x) {
     const int p = idx / half, i = idx - p * half;
-    const double theta = pow(a.base, -2.0 * (double)i / (double)a.d);
-    const double ang = (double)(a.pos_offset + t0 + p) * theta;
-    double s, c;
-    sincos(ang, &s, &c);
-    cs[idx] = (float)c;
-    sn[idx] = (float)s;
+    const float2 c = rope_cos_sin((long long)a.pos_offset + t0 + p, i, a.d, a.base);
+    cs[idx] = c.x;
+    sn[idx] = c.y;
   }
   __syncthreads();
 
@@ -75,8 +73,9 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(RopeArgs a) {
       for (int k = 0; k < 4; ++k) {
         const int i = 4 * c + k;
         const float x0 = bf16_lo(w[k]), x1 = bf16_hi(w[k]);
-        const float cc = cp[i], ss = sp[i];
-        o[k] = pack_bf16x2(x0 * cc - x1 * ss, x0 * ss + x1 * cc);
+        float r0, r1;
+        rope_rotate(x0, x1, make_float2(cp[i], sp[i]), r0, r1);
+        o[k] = pack_bf16x2(r0, r1);
       }
       *reinterpret_cast<uint4*>(a.y + row + 8 * c) = make_uint4(o[0], o[1], o[2], o[3]);
     } else {
@@ -91,9 +90,11 @@ __global__ void __launch_bounds__(kThreads) rope_kernel(RopeArgs a) {
         const int i = 8 * c + 2 * k;
         const float a0 = bf16_lo(wa[k]), a1 = bf16_hi(wa[k]);
         const float b0 = bf16_lo(wb[k]), b1 = bf16_hi(wb[k]);
-        const float c0 = cp[i], s0 = sp[i], c1 = cp[i + 1], s1 = sp[i + 1];
-        oa[k] = pack_bf16x2(a0 * c0 - b0 * s0, a1 * c1 - b1 * s1);
-        ob[k] = pack_bf16x2(a0 * s0 + b0 * c0, a1 * s1 + b1 * c1);
+        float ra0, rb0, ra1, rb1;
+        rope_rotate(a0, b0, make_float2(cp[i], sp[i]), ra0, rb0);
+        rope_rotate(a1, b1, make_float2(cp[i + 1], sp[i + 1]), ra1, rb1);
+        oa[k] = pack_bf16x2(ra0, ra1);
+        ob[k] = pack_bf16x2(rb0, rb1);
       }
       *reinterpret_cast<uint4*>(a.y + row + 8 * c) = make_uint4(oa[0], oa[1], oa[2], oa[3]);
       *reinterpret_cast<uint4*>(a.y + row + half + 8 * c) = make_uint4(ob[0], ob[1], ob[2], ob[3]);
@@ -111,12 +112,9 @@ __global__ void __launch_bounds__(kThreads) rope_kernel_scalar(RopeArgs a) {
   float* sn = tab + kPos * half;
   for (int idx = threadIdx.x; idx < npos * half; idx += blockDim.x) {
     const int p = idx / half, i = idx - p * half;
-    const double theta = pow(a.base, -2.0 * (double)i / (double)a.d);
-    const double ang = (double)(a.pos_offset + t0 + p) * theta;
-    double s, c;
-    sincos(ang, &s, &c);
-    cs[idx] = (float)c;
-    sn[idx] = (float)s;
+    const float2 c = rope_cos_sin((long long)a.pos_offset + t0 + p, i, a.d, a.base);
+    cs[idx] = c.x;
+    sn[idx] = c.y;
   }
   __syncthreads();
   const int bh0 = blockIdx.y * kHeads;
@@ -131,10 +129,30 @@ __global__ void __launch_bounds__(kThreads) rope_kernel_scalar(RopeArgs a) {
     const int ib = a.pairing ? 2 * i + 1 : i + half;
     const float x0 = __bfloat162float(a.x[row + ia]);
     const float x1 = __bfloat162float(a.x[row + ib]);
-    const float cc = cs[p * half + i], ss = sn[p * half + i];
-    a.y[row + ia] = __float2bfloat16_rn(x0 * cc - x1 * ss);
-    a.y[row + ib] = __float2bfloat16_rn(x0 * ss + x1 * cc);
+    float r0, r1;
+    rope_rotate(x0, x1, make_float2(cs[p * half + i], sn[p * half + i]), r0, r1);
+    a.y[row + ia] = __float2bfloat16_rn(r0);
+    a.y[row + ib] = __float2bfloat16_rn(r1);
   }
+}
+
+// (cos, sin) table for positions pos_offset .. pos_offset + N - 1: tab[t * d/2 + i].
+__global__ void rope_table_kernel(float2* tab, int N, int d, double base, int pos_offset) {
+  const int half = d / 2;
+  const long long n = (long long)N * half;
+  for (long long idx = blockIdx.x * (long long)blockDim.x + threadIdx.x; idx < n;
+       idx += (long long)gridDim.x * blockDim.x) {
+    const int t = (int)(idx / half), i = (int)(idx - (long long)t * half);
+    tab[idx] = rope_cos_sin((long long)pos_offset + t, i, d, base);
+  }
+}
+
+int launch_rope_table(float2* tab, int N, int d, float base, int pos_offset, cudaStream_t st) {
+  const long long n = (long long)N * (d / 2);
+  if (n == 0) return ATTN_OK;
+  const int blocks = (int)((n + 255) / 256 < 4096 ? (n + 255) / 256 : 4096);
+  rope_table_kernel<<<blocks, 256, 0, st>>>(tab, N, d, (double)base, pos_offset);
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
 int launch_rope(const void* x_in, void* x_out, int B, int H, int N, int d, float base,

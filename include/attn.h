@@ -168,6 +168,28 @@ ATTN_API size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int 
 ATTN_API int rope_apply(const void* x_in, void* x_out, int B, int H, int N, int d,
                float base, int pos_offset, int pairing, void* stream);
 
+/* Attention with the RoPE prologue of q fused in: as attn_fwd_ws, but q holds
+ * UN-rotated queries; row i of q is rotated at position q_pos_offset + i with
+ * rope_apply's frequencies, pairing and arithmetic (bit for bit the values
+ * rope_apply would store), then attends.  k must hold keys already rotated
+ * (rope_apply at their positions; a KV cache stores them that way).
+ *   Prefill shapes rotate each Q tile in shared memory after its TMA load
+ *   (the prefill kernel's Q producer warp), with a (cos, sin) table of the
+ *   Nq positions built in the workspace; decode shapes ((Hq/Hkv) * Nq <= 64)
+ *   rotate q into the workspace and run the decode kernels.
+ *   rope_base > 0, rope_pairing 0 (i, i + d/2) or 1 (2i, 2i + 1),
+ *   q_pos_offset >= 0.  Workspace: attn_rope_workspace_size(...) bytes
+ *   (256-byte aligned, contents need no initialisation).
+ * Errors: as attn_fwd_ws. */
+ATTN_API int attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse,
+                           int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                           float scale, const int32_t* key_lens, float rope_base,
+                           int rope_pairing, int q_pos_offset, void* workspace,
+                           size_t workspace_bytes, void* stream);
+
+/* Bytes of workspace attn_fwd_rope needs (0 for invalid sizes). */
+ATTN_API size_t attn_rope_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+
 /* Tile shape (query rows Br, keys Bc) the prefill kernel uses for head
  * dimension d.  Returns ATTN_EUNSUPPORTED for other d. */
 ATTN_API int attn_prefill_tile_shape(int d, int* Br, int* Bc);

@@ -164,3 +164,16 @@ def test_paged_rejects_bad_arguments_on_host(L):
              None) == 2                                      # 128 query rows per kv head
     assert f(P, P, P, P, 4, 16, 8, P, None, 1, 4, 1, 1, 128, 1, -1, 0.1, P, P, 1 << 20,
              None) == 1                                      # negative window
+
+
+def test_fused_rope_rejects_bad_arguments_on_host(L):
+    f = L.attn_fwd_rope
+    # prefill shape: workspace = 256 (counter) + the (cos, sin) table of 128 rows
+    need = L.attn_rope_workspace_size(1, 2, 2, 128, 128, 64)
+    assert need == 256 + 128 * 32 * 8
+    args = (P, P, P, P, None, 1, 2, 2, 128, 128, 64, 1, 0.125, None)
+    assert f(*args, 0.0, 0, 0, P, need, None) == 1            # base
+    assert f(*args, 1e4, 2, 0, P, need, None) == 1            # pairing
+    assert f(*args, 1e4, 0, -1, P, need, None) == 1           # position offset
+    assert f(*args, 1e4, 0, 0, P, need - 1, None) == 4        # workspace too small
+    assert f(*args, 1e4, 0, 0, ctypes.c_void_p(0x1010), need, None) == 3

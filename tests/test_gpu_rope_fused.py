@@ -1,0 +1,81 @@
+"""The RoPE prologue of q fused into attention (attn_fwd_rope) against the
+unfused pipeline and the oracle.
+
+The fused path rotates q with rope_apply's arithmetic ("Transformer
+Architecture Breakdown ...", section 3.1; "Coding interview (14)", section
+3.5), so attention over (fused q, rope_apply(k)) must equal attention over
+(rope_apply(q), rope_apply(k)) bit for bit; against the fp64 oracle (which
+models the bf16 rounding of the rotated rows) the usual tolerances hold:
+O max-abs <= 2e-2, mean-abs <= 2e-3, lse <= 1e-3."""
+import math
+
+import numpy as np
+import pytest
+
+import oracle
+from exact_scaled_dot_fwd_b200 import synth
+
+from parity import compare, from_dev, rand_inputs, to_dev
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def torch():
+    import torch as t
+    from exact_scaled_dot_fwd_b200 import build
+    build.build()
+    return t
+
+
+CASES = [
+    # B, Hq, Hkv, Nq, Nk, d, causal, pairing, q_pos_offset, k_pos_offset
+    (2, 8, 2, 300, 300, 128, True, 0, 0, 0),        # prefill, half pairing
+    (1, 4, 4, 257, 257, 64, True, 1, 0, 0),         # d = 64, adjacent pairing
+    (2, 4, 4, 200, 700, 128, True, 0, 500, 0),      # queries at the end of the keys
+    (1, 6, 3, 129, 129, 64, False, 0, 7, 7),        # offsets, not causal
+    (2, 32, 8, 1024, 1024, 128, True, 1, 0, 0),     # GQA head pairs
+    (3, 8, 2, 4, 900, 128, True, 0, 896, 0),        # decode shape (32 rows per kv head)
+    (2, 4, 1, 1, 500, 64, False, 1, 499, 0),        # single-token decode, d = 64
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "x".join(map(str, c)))
+def test_fused_rope_matches_unfused_bitwise(torch, case):
+    import exact_scaled_dot_fwd_b200 as eb
+    B, Hq, Hkv, Nq, Nk, d, causal, pairing, qoff, koff = case
+    x = rand_inputs(B, Hq, Hkv, Nq, Nk, d, seed=9900 + Nq + Nk + d)
+    q, k, v = (to_dev(x[n], torch) for n in ("q", "k", "v"))
+    scale = 1 / math.sqrt(d)
+    kr = eb.rope_apply(k, base=10000.0, pos_offset=koff, pairing=pairing)
+    qr = eb.rope_apply(q, base=10000.0, pos_offset=qoff, pairing=pairing)
+    o1, l1 = eb.attn_fwd(qr, kr, v, causal=causal, scale=scale)
+    o2, l2 = eb.attn_fwd_rope(q, kr, v, causal=causal, scale=scale, rope_base=10000.0,
+                              rope_pairing=pairing, q_pos_offset=qoff)
+    torch.cuda.synchronize()
+    assert eb.device_status() == 0
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    # and both agree with the oracle (rotated rows rounded to bf16)
+    rope = dict(base=10000.0, pairing=pairing, q_pos_offset=qoff, k_pos_offset=koff,
+                round_bf16=True)
+    o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], causal, scale, rope_cfg=rope)
+    compare(from_dev(o2).reshape(-1, d), l2.cpu().numpy().astype(np.float64).reshape(-1),
+            o_ref, lse_ref, what=str(case))
+
+
+def test_fused_rope_gqa_workload_sampled_rows(torch):
+    import exact_scaled_dot_fwd_b200 as eb
+    w = synth.WORKLOADS["gqa_rope_prefill"]
+    x = synth.make_inputs(w)
+    q, k, v = (to_dev(x[n], torch) for n in ("q", "k", "v"))
+    kr = eb.rope_apply(k, base=synth.ROPE_BASE, pairing=synth.ROPE_PAIRING_HALF)
+    o, lse = eb.attn_fwd_rope(q, kr, v, causal=True, scale=w.scale, rope_base=synth.ROPE_BASE,
+                              rope_pairing=synth.ROPE_PAIRING_HALF)
+    torch.cuda.synchronize()
+    rows = synth.sample_rows(w, per_head_random=11)
+    rope = dict(base=synth.ROPE_BASE, pairing=synth.ROPE_PAIRING_HALF, q_pos_offset=0,
+                k_pos_offset=0, round_bf16=True)
+    o_ref, lse_ref = oracle.attn_rows(x["q"], x["k"], x["v"], True, w.scale, rows=rows,
+                                      rope_cfg=rope)
+    compare(from_dev(o).reshape(-1, w.d)[rows], lse.cpu().numpy().astype(np.float64).reshape(-1)[rows],
+            o_ref, lse_ref, what=w.name)
