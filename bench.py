@@ -53,7 +53,7 @@ KERNEL_SOURCES = {
 }
 NCU_TRAFFIC = {
     # workload: (kernel, source hash, bytes per launch)
-    "mha_prefill": ("prefill", "6191a56c605c70b0", 124861952 + 10512384),
+    "mha_prefill": ("prefill", "429f44777b3430af", 128382464 + 10732544),
     "mqa_decode": ("decode", "bad510b57056b510", 324108032 + 4244480),
 }
 
