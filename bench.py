@@ -53,8 +53,8 @@ KERNEL_SOURCES = {
 }
 NCU_TRAFFIC = {
     # workload: (kernel, source hash, bytes per launch)
-    "mha_prefill": ("prefill", "429f44777b3430af", 128382464 + 10732544),
-    "mqa_decode": ("decode", "bad510b57056b510", 324108032 + 4244480),
+    "mha_prefill": ("prefill", "364317d010ce4926", 136833280 + 12229120),
+    "mqa_decode": ("decode", "fbeda4030074503e", 324113408 + 5059072),
 }
 
 

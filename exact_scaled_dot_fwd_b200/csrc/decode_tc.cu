@@ -409,25 +409,26 @@ __global__ void __launch_bounds__(192, 1)
     if (lane == 0 && start < end) {
       const uint32_t k_base = smem_u32(smem + L::kK), v_base = smem_u32(smem + L::kV);
       const uint32_t q_base = smem_u32(smem + L::kQ), p_base = smem_u32(smem + L::kP);
+      // descriptors built once per call; a k-step only moves the start
+      // address field (address >> 4 in bits 0-13, no carry below 256 KB)
       auto issue_s = [&](int g) {
-        const uint32_t kb = k_base + (g % KS) * L::kKV;
+        const uint64_t dk = tc::smem_desc_sw128(k_base + (g % KS) * L::kKV, 16, 1024);
+        const uint64_t dq = tc::smem_desc_sw128(q_base, 16, 1024);
+        const uint32_t dt = tmem + (uint32_t)((g & 1) * N);
+        tc::mma_ss(dt, dk, dq, kIdescS, 0u);
 #pragma unroll
-        for (int kk = 0; kk < kD / 16; ++kk) {
-          tc::mma_ss(tmem + (uint32_t)((g & 1) * N),
-                     tc::smem_desc_sw128(kb + (kk >> 2) * L::kBox + (kk & 3) * 32, 16, 1024),
-                     tc::smem_desc_sw128(q_base + (kk >> 2) * L::kQBox + (kk & 3) * 32, 16, 1024),
-                     kIdescS, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 1; kk < kD / 16; ++kk)
+          tc::mma_ss(dt, dk + (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4),
+                     dq + (uint64_t)(((kk >> 2) * L::kQBox + (kk & 3) * 32) >> 4), kIdescS, 1u);
       };
       auto issue_pv = [&](int g, bool acc) {
-        const uint32_t vb = v_base + (g % VS) * L::kKV;
-        const uint32_t pbuf = p_base + (g & 1) * 2 * L::kPBox;
+        const uint64_t dv = tc::smem_desc_sw128(v_base + (g % VS) * L::kKV, L::kBox, 1024);
+        const uint64_t dp = tc::smem_desc_sw128(p_base + (g & 1) * 2 * L::kPBox, 16, 1024);
+        tc::mma_ss(tmem + 2u * N, dv, dp, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk) {
-          tc::mma_ss(tmem + 2u * N, tc::smem_desc_sw128(vb + kk * 16 * 128, L::kBox, 1024),
-                     tc::smem_desc_sw128(pbuf + (kk >> 2) * L::kPBox + (kk & 3) * 32, 16, 1024),
-                     kIdescPV, (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < kTile / 16; ++kk)
+          tc::mma_ss(tmem + 2u * N, dv + (uint64_t)((kk * 16 * 128) >> 4),
+                     dp + (uint64_t)(((kk >> 2) * L::kPBox + (kk & 3) * 32) >> 4), kIdescPV, 1u);
       };
       int u = u0, g = 0, qf = 0;
       Seg s;

@@ -432,23 +432,29 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       const uint32_t q_base = smem_u32(smem + L::kQ);
       const uint32_t k_base = smem_u32(smem + L::kK);
       const uint32_t v_base = smem_u32(smem + L::kV);
+      // Descriptors are built once per call; a k-step only moves the start
+      // address field (bits 0-13 hold address >> 4, and shared memory stays
+      // below 256 KB, so the add never carries out of it).  The issuing
+      // thread is on the critical path: about 600 cycles per call were
+      // measured with per-step descriptor construction.
       auto issue_s = [&](int t, int ks) {
-        const uint32_t qa = q_base + t * L::kTile, kb = k_base + ks * L::kTile;
+        const uint64_t da = tc::smem_desc_sw128(q_base + t * L::kTile, 16, 1024);
+        const uint64_t db = tc::smem_desc_sw128(k_base + ks * L::kTile, 16, 1024);
+        const uint32_t dt = tmem + 128u * t;
+        tc::mma_ss(dt, da, db, kIdescS, 0u);
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::kBox + (kk & 3) * 32;
-          tc::mma_ss(tmem + 128u * t, tc::smem_desc_sw128(qa + off, 16, 1024),
-                     tc::smem_desc_sw128(kb + off, 16, 1024), kIdescS, kk > 0 ? 1u : 0u);
+        for (int kk = 1; kk < D / 16; ++kk) {
+          const uint64_t off = (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4);
+          tc::mma_ss(dt, da + off, db + off, kIdescS, 1u);
         }
       };
       auto issue_pv = [&](int t, int vs, bool acc) {
-        const uint32_t vb = v_base + vs * L::kTile;
+        const uint64_t dv = tc::smem_desc_sw128(v_base + vs * L::kTile, L::kBox, 1024);
+        const uint32_t dt = tmem + 256u + D * t, pa = tmem + 128u * t;
+        tc::mma_ts(dt, pa, dv, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 0; kk < kN / 16; ++kk) {
-          tc::mma_ts(tmem + 256u + D * t, tmem + 128u * t + kk * 8,
-                     tc::smem_desc_sw128(vb + kk * 16 * 128, L::kBox, 1024), kIdescPV,
-                     (acc || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 1; kk < kN / 16; ++kk)
+          tc::mma_ts(dt, pa + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, 1u);
       };
       // Each slot's work is one stream of KV tiles across items: in the step
       // that finishes item i for one slot, the S MMA of item i+1's first
