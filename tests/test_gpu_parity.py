@@ -254,3 +254,23 @@ def test_rope_relative_position_on_gpu(torch):
         dots.append(float((rq * rk).sum()))
     # equal up to the bf16 rounding of the rotated vectors
     assert max(dots) - min(dots) < 0.05 * (1 + abs(dots[0]))
+
+
+# Shapes the decode kernels do not take (more than 64 query rows per kv head,
+# or more than 2048 sequences) run the prefill kernel, Nq = 1 included.
+ROUTED_TO_PREFILL = [
+    # B, Hq, Hkv, Nq, Nk, d, causal, key_lens
+    (2, 128, 1, 1, 300, 128, False, [300, 17]),     # 128 query heads on one kv head
+    (2, 64, 2, 3, 500, 64, True, [500, 250]),       # 96 rows per kv head, d = 64
+    (2100, 2, 2, 1, 40, 128, False, None),          # more sequences than the decode scan holds
+]
+
+
+@pytest.mark.parametrize("case", ROUTED_TO_PREFILL, ids=lambda c: "x".join(map(str, c[:6])))
+def test_decode_shapes_routed_to_prefill(torch, case):
+    B, Hq, Hkv, Nq, Nk, d, causal, kl = case
+    x = rand_inputs(B, Hq, Hkv, Nq, Nk, d, seed=8800 + B + Hq, key_lens=kl)
+    rows = None
+    if B * Hq * Nq > 20000:   # sample rows of the large batch
+        rows = np.arange(0, B * Hq * Nq, 37, dtype=np.int64)
+    check_workload(x, (B, Hq, Nq, d), causal, 1 / math.sqrt(d), rows=rows, what=str(case))
