@@ -74,9 +74,9 @@ struct Seg {
 
 // Prefix of unit u: keys of all units before u (units are b-major, h-minor).
 __device__ __forceinline__ long long unit_prefix(const long long* pb, const int* lens, int u,
-                                                 int Hkv) {
+                                                 int Hkv, int seg) {
   const int b = u / Hkv, h = u - b * Hkv;
-  return (long long)Hkv * pb[b] + (long long)h * lens[b];
+  return (long long)Hkv * pb[b] + (long long)h * virtual_len(lens[b], seg);
 }
 
 }  // namespace
@@ -89,6 +89,7 @@ struct DecodeArgs {
   int B, Hq, Hkv, Nk, G, grid;
   int Nq, R;                 // query rows per sequence, rows per unit (G * Nq)
   int causal, window, align;
+  int seg_cost;              // virtual keys in front of every non-empty unit
   float scale_log2;
   // paged cache (kPaged): Nk = max_pages * page_size
   const int32_t* block_table;
@@ -142,13 +143,14 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
         lens_s[b] = len;   // keys [lo, L) of every unit of sequence b
         lo_s[b] = lo;
       }
-      long long x = len;
+      const int vlen = virtual_len(len, a.seg_cost);
+      long long x = vlen;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const long long y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
-      if (b < B) pb[b] = carry + x - len;
+      if (b < B) pb[b] = carry + x - vlen;
       carry += __shfl_sync(0xffffffffu, x, 31);
     }
     if (lane == 0) pb[B] = carry;
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
     int lo = 0, hi = U - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (unit_prefix(pb, lens_s, mid, Hkv) <= start) lo = mid; else hi = mid - 1;
+      if (unit_prefix(pb, lens_s, mid, Hkv, a.seg_cost) <= start) lo = mid; else hi = mid - 1;
     }
     u0 = lo;
   }
@@ -175,13 +177,15 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
   };
   auto next_seg = [&](int& u, Seg& s) -> bool {
     while (u < U) {
-      const long long p0 = unit_prefix(pb, lens_s, u, Hkv);
+      const long long p0 = unit_prefix(pb, lens_s, u, Hkv, a.seg_cost);
       if (p0 >= end) return false;
-      const long long p1 = p0 + lens_s[u / Hkv];
-      const long long lo = start > p0 ? start : p0, hi = end < p1 ? end : p1;
+      const int len = lens_s[u / Hkv];
+      const long long r0 = p0 + (len > 0 ? a.seg_cost : 0);   // the unit's first real key
+      const long long p1 = r0 + len;
+      const long long lo = start > r0 ? start : r0, hi = end < p1 ? end : p1;
       const int cur = u++;
       if (hi > lo) {
-        s.u = cur; s.lo = (int)(lo - p0); s.hi = (int)(hi - p0);
+        s.u = cur; s.lo = (int)(lo - r0); s.hi = (int)(hi - r0);
         return true;
       }
     }
@@ -450,6 +454,7 @@ struct CombineArgs {
   int B, Hq, Hkv, Nk, G, grid;
   int Nq, R;
   int window, align;
+  int seg_cost;
 };
 
 constexpr int kCombineThreads = 256;
@@ -471,8 +476,9 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
     const int Lb = clamp_len(a.key_lens ? a.key_lens[bb] : a.Nk, a.Nk);
     int lo;
     const int len = decode_key_range(Lb, query_offset(a.Nq, a.Nk, Lb, a.align), a.window, &lo);
-    total += len;
-    if (bb < b) before += len;
+    const int vlen = virtual_len(len, a.seg_cost);
+    total += vlen;
+    if (bb < b) before += vlen;
     if (bb == b) s_len = len;
   }
 #pragma unroll
@@ -488,7 +494,8 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
   if (threadIdx.x == 0) {
     long long pb = 0, tot = 0;
     for (int w = 0; w < (int)(blockDim.x >> 5); ++w) { pb += s_red[0][w]; tot += s_red[1][w]; }
-    s_pb[0] = (long long)a.Hkv * pb + (long long)h * s_len;   // unit start
+    s_pb[0] = (long long)a.Hkv * pb + (long long)h * virtual_len(s_len, a.seg_cost) +
+              (s_len > 0 ? a.seg_cost : 0);                   // the unit's first real key
     s_pb[1] = (long long)a.Hkv * tot;                         // T
   }
   __syncthreads();
@@ -601,10 +608,17 @@ bool decode_supported(int B, int Hq, int Hkv, int Nq, int d) {
   return (d == 64 || d == 128) && Nq >= 1 && R >= 1 && R <= 64 && B <= kMaxScanB;
 }
 
+// Virtual keys charged to every non-empty unit in the work split: about the
+// cost of starting a segment, in keys (see virtual_len in tile_plan.cuh).
+constexpr int kSegCost = 320;
+
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
-                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk, const PagedKv* pg,
+                  int Hkv, int Nq, int Nk, int d, const DecodeMask& mk_in, const PagedKv* pg,
                   float scale, const int32_t* key_lens, void* workspace, const DecodePlan& p,
                   cudaStream_t st) {
+  DecodeMask mk = mk_in;
+  // the split's key prefix is an int: keep the virtual total below 2^31
+  mk.seg_cost = (long long)B * Hkv * ((long long)Nk + kSegCost) < (1ll << 31) ? kSegCost : 0;
   int rc;
   DecodeArgs a;
   a.q = static_cast<const __nv_bfloat16*>(q);
@@ -614,6 +628,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = p.G; a.grid = p.grid;
   a.Nq = Nq; a.R = p.R;
   a.causal = mk.causal; a.window = mk.window; a.align = mk.align;
+  a.seg_cost = mk.seg_cost;
   a.scale_log2 = scale * kLog2e;
   if (d == 128) {   // decode_supported ensures the tcgen05 kernel takes it
     if (!decode_tc_supported(B, Hq, Hkv, Nq, d)) return ATTN_EUNSUPPORTED;
@@ -653,6 +668,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   c.B = B; c.Hq = Hq; c.Hkv = Hkv; c.Nk = Nk; c.G = p.G; c.grid = p.grid;
   c.Nq = Nq; c.R = p.R;
   c.window = mk.window; c.align = mk.align;
+  c.seg_cost = mk.seg_cost;
   // shared memory: the unit's slot lse's ([slots][heads of the block], at most
   // grid + 1 slots) + [heads of the block]
   const int hb = kCombineThreads / d;

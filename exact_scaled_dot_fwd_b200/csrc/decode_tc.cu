@@ -97,9 +97,9 @@ struct Seg {
 
 // (B * Hkv * Nk < 2^31 is checked on the host, so every prefix fits an int.)
 __device__ __forceinline__ long long unit_prefix(const int* pb, const int* lens, int u,
-                                                 int Hkv) {
+                                                 int Hkv, int seg) {
   const int b = u / Hkv, h = u - b * Hkv;
-  return (long long)Hkv * pb[b] + (long long)h * lens[b];
+  return (long long)Hkv * pb[b] + (long long)h * virtual_len(lens[b], seg);
 }
 
 // One butterfly step across lanes `OFF` apart: each lane keeps the half of
@@ -217,6 +217,7 @@ struct DecodeTcArgs {
   int B, Hq, Hkv, Nk, G, grid;
   int Nq, R;                 // query rows per sequence, rows per unit (G * Nq)
   int causal, window, align;
+  int seg_cost;              // virtual keys in front of every non-empty unit
   float scale_log2;
   // paged cache (kernel instantiation with kPaged): Nk = max_pages * page_size
   const int32_t* block_table;
@@ -275,13 +276,14 @@ __global__ void __launch_bounds__(192, 1)
         lens_s[b] = len;   // keys [lo, L) of every unit of sequence b
         lo_s[b] = lo;
       }
-      int x = len;
+      const int vlen = virtual_len(len, a.seg_cost);
+      int x = vlen;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const int y = __shfl_up_sync(0xffffffffu, x, o);
         if (lane >= o) x += y;
       }
-      if (b < B) pb[b] = carry + x - len;
+      if (b < B) pb[b] = carry + x - vlen;
       carry += __shfl_sync(0xffffffffu, x, 31);
     }
     if (lane == 0) pb[B] = carry;
@@ -299,19 +301,21 @@ __global__ void __launch_bounds__(192, 1)
     int lo = 0, hi = U - 1;
     while (lo < hi) {
       const int mid = (lo + hi + 1) >> 1;
-      if (unit_prefix(pb, lens_s, mid, Hkv) <= start) lo = mid; else hi = mid - 1;
+      if (unit_prefix(pb, lens_s, mid, Hkv, a.seg_cost) <= start) lo = mid; else hi = mid - 1;
     }
     u0 = lo;
   }
   auto next_seg = [&](int& u, Seg& s) -> bool {
     while (u < U) {
-      const long long p0 = unit_prefix(pb, lens_s, u, Hkv);
+      const long long p0 = unit_prefix(pb, lens_s, u, Hkv, a.seg_cost);
       if (p0 >= end) return false;
-      const long long p1 = p0 + lens_s[u / Hkv];
-      const long long lo = start > p0 ? start : p0, hi = end < p1 ? end : p1;
+      const int len = lens_s[u / Hkv];
+      const long long r0 = p0 + (len > 0 ? a.seg_cost : 0);   // the unit's first real key
+      const long long p1 = r0 + len;
+      const long long lo = start > r0 ? start : r0, hi = end < p1 ? end : p1;
       const int cur = u++;
       if (hi > lo) {
-        s.u = cur; s.lo = (int)(lo - p0); s.hi = (int)(hi - p0);
+        s.u = cur; s.lo = (int)(lo - r0); s.hi = (int)(hi - r0);
         const int kl = lo_s[cur / Hkv];
         s.start = kl + s.lo;
         s.end = kl + s.hi;
@@ -671,6 +675,7 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.Nk = Nk; a.G = G; a.grid = grid;
   a.Nq = Nq; a.R = R;
   a.causal = mk.causal; a.window = mk.window; a.align = mk.align;
+  a.seg_cost = mk.seg_cost;
   a.scale_log2 = scale * kLog2e;
   if (pg) {
     if (N == 16) return launch_tc_t<16, true>(grid, tq, tk, tv, a, st);

@@ -34,6 +34,9 @@ struct DecodePlan {
 // alignment (0: rows end at key Nk - 1; 1: at key key_lens[b] - 1).
 struct DecodeMask {
   int causal = 0, window = 0, align = 0;
+  // virtual keys charged to every non-empty unit in the work split (see
+  // virtual_len in tile_plan.cuh); set by launch_decode
+  int seg_cost = 0;
 };
 // Paged KV cache: cache [num_pages, Hkv, page_size, d]; key j of sequence b
 // is row j % page_size of block block_table[b * max_pages + j / page_size].

@@ -116,4 +116,13 @@ __host__ __device__ __forceinline__ int decode_key_range(int L, int off, int win
   return L - l;
 }
 
+// Decode work split: the units' keys are laid end to end and split evenly
+// over the CTAs, with `seg` virtual keys in front of every non-empty unit --
+// the cost of starting a segment (its Q, the first tile's pipeline, the
+// partial result) in keys, so a CTA whose range holds a unit start gets
+// fewer real keys.
+__host__ __device__ __forceinline__ int virtual_len(int len, int seg) {
+  return len > 0 ? len + seg : 0;
+}
+
 }  // namespace attn
