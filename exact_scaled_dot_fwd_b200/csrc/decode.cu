@@ -441,10 +441,10 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
 }
 
 // Combine: one CTA per (unit, kCombineThreads / D rows), one thread per
-// output element.  The log-sum-exps of the unit's slots are staged in shared
-// memory, per row lse = log2 sum_s 2^lse_s, then every (row, d) output sums
-// its slots' partials weighted by 2^(lse_s - lse) with independent loads.
-// A row no slot saw a key for (masked everywhere) gets O = 0, lse = -inf.
+// output element, which merges the unit's slots for its (row, d) with the
+// running-max recurrence of the online softmax over the slots: lse =
+// log2 sum_s 2^lse_s, O = sum_s 2^(lse_s - lse) O_s.  A row no slot saw a key
+// for (masked everywhere) gets O = 0, lse = -inf.
 struct CombineArgs {
   const int32_t* key_lens;
   const float* part_o;
@@ -461,7 +461,7 @@ constexpr int kCombineThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(CombineArgs a) {
-  extern __shared__ float cs[];          // lse_s [ns][G], then L2 [G]
+  extern __shared__ float cs[];          // int flags [ns]: slots written by this launch
   __shared__ long long s_red[2][kCombineThreads / 32];
   __shared__ long long s_pb[2];
   __shared__ int s_len;
@@ -523,56 +523,48 @@ __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(Combine
   auto nonempty = [&](int c) -> bool { return T * c / a.grid < T * (c + 1) / a.grid; };
   // launched as a programmatic dependent of the split kernel: everything
   // above reads only inputs; the partials are ready after this wait
+  // which of the unit's slots this launch wrote (CTAs with empty key ranges
+  // write none; their slots hold stale data), settled before the wait
+  int* written = reinterpret_cast<int*>(cs);   // [ns]
+  for (int k = threadIdx.x; k < ns; k += blockDim.x) written[k] = nonempty(c0 + k) ? 1 : 0;
+  __syncthreads();
   asm volatile("griddepcontrol.wait;" ::: "memory");
-  float* lse_s = cs;                  // [ns][HB]
-  float* L2 = cs + (size_t)ns * HB;   // [HB]
-  for (int idx = threadIdx.x; idx < ns * gn; idx += blockDim.x) {
-    const int k = idx / gn, g = idx - k * gn;
-    lse_s[k * HB + g] =
-        nonempty(c0 + k) ? a.part_lse[((size_t)(c0 + k) + u) * G + g0 + g] : -INFINITY;
-  }
-  __syncthreads();
-  if (threadIdx.x < gn) {
-    const int g = threadIdx.x;
-    float mx = -INFINITY;
-    for (int k = 0; k < ns; ++k) mx = fmaxf(mx, lse_s[k * HB + g]);
-    float l2 = -INFINITY;   // no slot saw a visible key for this row
-    if (mx != -INFINITY) {
-      float sum = 0.f;
-      for (int k = 0; k < ns; ++k) sum += exp2_approx(lse_s[k * HB + g] - mx);
-      l2 = mx + __log2f(sum);
-    }
-    L2[g] = l2;
-    if (a.lse) a.lse[row0 + g] = l2 == -INFINITY ? -INFINITY : l2 * kLn2;
-  }
-  __syncthreads();
+  // one thread per output: the slots' log-sum-exps and partials are loaded
+  // together and merged with the running-max recurrence over the slots
   for (int idx = threadIdx.x; idx < gn * D; idx += blockDim.x) {
     const int g = idx / D, c = idx - g * D;
-    const float l2 = L2[g];
-    if (l2 == -INFINITY) {
-      orow[idx] = __float2bfloat16(0.f);
-      continue;
-    }
-    const float* src = a.part_o + (((size_t)c0 + u) * G + g0 + g) * D + c;
-    const size_t stride = (size_t)G * D;   // next slot
-    float acc = 0.f;
+    const float* lsrc = a.part_lse + ((size_t)c0 + u) * G + g0 + g;
+    const float* osrc = a.part_o + (((size_t)c0 + u) * G + g0 + g) * D + c;
+    const size_t ls = (size_t)G, os = (size_t)G * D;   // next slot
+    float m = -INFINITY, acc = 0.f, sum = 0.f;
     int k = 0;
+    auto merge = [&](float lk, float xk) {
+      if (lk == -INFINITY) return;   // no visible key of this row in the slot
+      if (lk > m) {
+        const float f = m == -INFINITY ? 0.f : exp2_approx(m - lk);
+        acc *= f;
+        sum *= f;
+        m = lk;
+      }
+      const float w = exp2_approx(lk - m);
+      acc = fmaf(w, xk, acc);
+      sum += w;
+    };
     for (; k + 4 <= ns; k += 4) {
-      const float w0 = exp2_approx(lse_s[(k + 0) * HB + g] - l2);
-      const float w1 = exp2_approx(lse_s[(k + 1) * HB + g] - l2);
-      const float w2 = exp2_approx(lse_s[(k + 2) * HB + g] - l2);
-      const float w3 = exp2_approx(lse_s[(k + 3) * HB + g] - l2);
-      const float x0 = w0 != 0.f ? src[(k + 0) * stride] : 0.f;
-      const float x1 = w1 != 0.f ? src[(k + 1) * stride] : 0.f;
-      const float x2 = w2 != 0.f ? src[(k + 2) * stride] : 0.f;
-      const float x3 = w3 != 0.f ? src[(k + 3) * stride] : 0.f;
-      acc += (w0 * x0 + w1 * x1) + (w2 * x2 + w3 * x3);
+      float lk[4], xk[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const bool wr = written[k + e] != 0;
+        lk[e] = wr ? lsrc[(k + e) * ls] : -INFINITY;
+        xk[e] = wr ? osrc[(k + e) * os] : 0.f;
+      }
+#pragma unroll
+      for (int e = 0; e < 4; ++e) merge(lk[e], xk[e]);
     }
-    for (; k < ns; ++k) {
-      const float w = exp2_approx(lse_s[k * HB + g] - l2);
-      if (w != 0.f) acc += w * src[k * stride];
-    }
-    orow[idx] = __float2bfloat16(acc);
+    for (; k < ns; ++k)
+      if (written[k]) merge(lsrc[k * ls], osrc[k * os]);
+    orow[idx] = __float2bfloat16(sum > 0.f ? acc / sum : 0.f);
+    if (c == 0 && a.lse) a.lse[row0 + g] = sum > 0.f ? (m + __log2f(sum)) * kLn2 : -INFINITY;
   }
 }
 
