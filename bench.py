@@ -53,8 +53,8 @@ KERNEL_SOURCES = {
 }
 NCU_TRAFFIC = {
     # workload: (kernel, source hash, bytes per launch)
-    "mha_prefill": ("prefill", "364317d010ce4926", 136833280 + 12229120),
-    "mqa_decode": ("decode", "fbeda4030074503e", 324113408 + 5059072),
+    "mha_prefill": ("prefill", "13690b3af29eb735", 131180800 + 12398848),
+    "mqa_decode": ("decode", "6d67e14f67118d61", 322994688 + 4797952),
 }
 
 
