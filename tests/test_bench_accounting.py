@@ -1,0 +1,49 @@
+"""bench.py's work accounting on the CPU: which workloads are judged on HBM
+bytes, the algorithmic bytes of a decode step, and the FLOPs of a windowed
+workload, each against a count made independently here."""
+import os
+import sys
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+import bench  # noqa: E402
+from exact_scaled_dot_fwd_b200 import synth  # noqa: E402
+
+
+def test_memory_bound_workloads():
+    W = synth.WORKLOADS
+    assert bench.memory_bound(W["mqa_decode"])        # 32 rows per kv head
+    assert bench.memory_bound(W["spec_decode"])       # 4 heads x 4 tokens
+    for name in ("mha_prefill", "gqa_rope_prefill", "long_causal", "cross_padded", "long_window"):
+        assert not bench.memory_bound(W[name]), name
+
+
+def test_decode_bytes_count_each_valid_key_once():
+    w = synth.WORKLOADS["mqa_decode"]
+    kl = synth.uniform_key_lens(w.B, w.key_lens[0], w.key_lens[1], w.seed + 4)
+    kv = sum(int(L) * w.Hkv * w.d * 2 * 2 for L in kl)          # K and V, bf16
+    qo = w.B * w.Hq * w.Nq * w.d * 2 * 2                           # Q and O, bf16
+    lse = w.B * w.Hq * w.Nq * 4
+    assert bench.decode_bytes(w, kl) == kv + qo + lse
+    # the same formula at several rows per kv head (multi-token decode)
+    s = synth.WORKLOADS["spec_decode"]
+    kl2 = synth.uniform_key_lens(s.B, s.key_lens[0], s.key_lens[1], s.seed + 4)
+    assert bench.decode_bytes(s, kl2) == (float(kl2.sum()) * s.Hkv * s.d * 4
+                                           + s.B * s.Hq * s.Nq * (s.d * 4 + 4))
+
+
+def test_window_flops_count_visible_pairs():
+    """4 d FLOPs per (row, key) pair inside a causal window, counted by brute
+    force on a small shape and by the closed form on the bench workload."""
+    n, w, d, B, H = 300, 37, 8, 2, 3
+    small = synth.Workload("t", 99, B, H, H, n, n, d, True, window=w)
+    i = np.arange(n)[:, None]
+    j = np.arange(n)[None, :]
+    pairs = int(((j <= i) & (i - j < w)).sum())
+    assert small.flops() == 4.0 * B * H * d * pairs
+    lw = synth.WORKLOADS["long_window"]
+    N, W = lw.Nq, lw.window
+    assert lw.flops() == 4.0 * lw.B * lw.Hq * lw.d * (W * (W + 1) // 2 + (N - W) * W)
