@@ -53,7 +53,7 @@ KERNEL_SOURCES = {
 }
 NCU_TRAFFIC = {
     # workload: (kernel, source hash, bytes per launch)
-    "mha_prefill": ("prefill", "13690b3af29eb735", 131180800 + 12398848),
+    "mha_prefill": ("prefill", "4cd70c7687185cb2", 130960384 + 11369216),
     "mqa_decode": ("decode", "6d67e14f67118d61", 322994688 + 4797952),
 }
 

@@ -361,6 +361,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       tma_prefetch_desc(&tk);
       tma_prefetch_desc(&tv);
       int g = 0, k = 0;
+      int gk = 0;   // K tiles whose barrier was armed (one more than g if a V wait gave up)
       bool ok = true;
       int idx = (int)atomicAdd(a.sched, 1u);
       while (ok) {
@@ -382,6 +383,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
           const int ks = g % kKS;
           if (!mbar_wait(&bars[L::K_EMPTY + ks], ((g / kKS) & 1) ^ 1, abort_flag)) { ok = false; break; }
           mbar_arrive_expect_tx(&bars[L::K_FULL + ks], L::kTile);
+          ++gk;
           for (int bx = 0; bx < kBoxes; ++bx)
             tma_load_2d(smem + L::kK + ks * L::kTile + bx * L::kBox, &tk, bx * 64,
                         it.kv_row0 + j * kN, &bars[L::K_FULL + ks]);
@@ -395,8 +397,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         idx = nxt;
       }
       // every issued load must land before the CTA may exit (normally they
-      // have all been consumed already, and these waits return at once)
-      for (int j = g - kKS > 0 ? g - kKS : 0; j < g; ++j)
+      // have all been consumed already, and these waits return at once);
+      // counted per ring: a K tile whose V slot never freed was still loaded
+      for (int j = gk - kKS > 0 ? gk - kKS : 0; j < gk; ++j)
         mbar_wait(&bars[L::K_FULL + j % kKS], (j / kKS) & 1, nullptr);
       for (int j = g - kVS > 0 ? g - kVS : 0; j < g; ++j)
         mbar_wait(&bars[L::V_FULL + j % kVS], (j / kVS) & 1, nullptr);
