@@ -512,7 +512,9 @@ def run_rope(torch, eb, device, stream, peaks, peak_src, steps=None):
         n = steps or max(5, int(1000.0 / max(probe, 1e-3)))
         ms = time_steps(fn, n, torch, None, stream)
         out[name] = {"value": w.flops() * n / (ms / 1e3) / 1e12, "ms_per_step": ms / n,
-                     "steps": n, "gpu_launches": n * (3 if name == "separate" else 3)}
+                     # separate: 2 rope_apply + attention; fused: rope_apply on K,
+                     # the cos/sin table, attention
+                     "steps": n, "gpu_launches": 3 * n}
     out["value"] = out["fused_q"]["value"]
     return out
 
