@@ -623,9 +623,12 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         // pass 2: P = 2^(s * scale * log2e - m) as bf16 pairs over the first
         // 64 columns of S (chunk c reads S columns [64 c, 64 c + 64) and
         // writes P columns [32 c, 32 c + 32), which were already read)
+        // Unmasked tiles scale, shift and sum on packed f32x2 pairs (one
+        // instruction per two scores; the row sum keeps two partial sums).
         const float m_use = m_run == -INFINITY ? 0.f : m_run;
         float rs = 0.f;
         if (!masked) {
+          const float2 c_sl2 = make_float2(sl2, sl2), c_m = make_float2(-m_use, -m_use);
 #pragma unroll
           for (int c8 = 0; c8 < kN / 64; ++c8) {
             float sv[64];
@@ -633,15 +636,15 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
             tc::wait_ld();
             uint32_t pk[32];
+            float2 rs2 = make_float2(0.f, 0.f);
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
-              const float x0 = fmaf(sv[2 * e], sl2, -m_use);
-              const float x1 = fmaf(sv[2 * e + 1], sl2, -m_use);
-              const float p0 = exp2_approx(x0);
-              const float p1 = exp2_approx(x1);
-              rs += p0 + p1;
-              pk[e] = pack_bf16x2(p0, p1);
+              const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), c_sl2, c_m);
+              const float2 p = make_float2(exp2_approx(x.x), exp2_approx(x.y));
+              rs2 = __fadd2_rn(rs2, p);
+              pk[e] = pack_bf16x2(p.x, p.y);
             }
+            rs += rs2.x + rs2.y;
             tc::st16(tmem + lane_off + scol + 32 * c8, pk);
             tc::st16(tmem + lane_off + scol + 32 * c8 + 16, pk + 16);
           }
