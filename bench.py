@@ -211,6 +211,24 @@ def oracle_sample(w, seconds, seed=12345, rows_per_batch=None):
     return used_f, used_t, used_rows, threads
 
 
+def cpu_baseline_entry(w, unit, seconds):
+    """The bench line's cpu_baseline object: the oracle on a uniform row
+    sample of workload w, in the line's unit, with rows/s and the whole
+    workload's time extrapolated from the sample."""
+    f, t, rows, thr = oracle_sample(w, seconds)
+    e = {"value": f / t / 1e12, "unit": "TFLOP/s (useful, sampled rows)",
+         "cores": thr, "kind": "oracle",
+         "sample": f"{rows} uniformly drawn query rows of {w.name}, fp64, {t:.1f} s",
+         "rows_per_s": rows / t,
+         # uniform row sample: the whole workload costs total_rows / rows times as much
+         "full_workload_s_extrapolated": t * (w.B * w.Hq * w.Nq) / rows}
+    if unit == "GB/s":
+        # bytes the sampled rows read (K and V of the visible keys: 4 d bytes per key)
+        e["value"] = (f / (4.0 * w.d)) * w.d * 4 / t / 1e9
+        e["unit"] = "GB/s (K/V bytes of sampled rows)"
+    return e
+
+
 # ------------------------------------------------------------------- ours ---
 
 def to_dev(bits, torch, device):
@@ -410,17 +428,7 @@ def run_ours(args):
 
     # ---- oracle on host cores (rank 0, N=1 only)
     if not args.no_cpu and rank == 0 and world == 1:
-        f, t, rows, thr = oracle_sample(w, args.cpu_seconds)
-        line["cpu_baseline"] = {
-            "value": (f / t) / (1e12 if unit == "TFLOP/s" else 1.0) if unit == "TFLOP/s"
-            else None,
-            "unit": "TFLOP/s (useful, sampled rows)" if unit == "TFLOP/s" else "n/a",
-            "cores": thr, "kind": "oracle",
-            "sample": f"{rows} uniformly drawn query rows of {w.name}, fp64, {t:.1f} s"}
-        if unit == "GB/s":
-            # bytes the sampled rows read (K and V of the visible keys)
-            line["cpu_baseline"]["value"] = (f / (4.0 * w.d)) * w.d * 4 / t / 1e9
-            line["cpu_baseline"]["unit"] = "GB/s (K/V bytes of sampled rows)"
+        line["cpu_baseline"] = cpu_baseline_entry(w, unit, args.cpu_seconds)
 
     if rank == 0:
         print(json.dumps(line), flush=True)
@@ -609,7 +617,10 @@ def run_reference(args):
                        "Nk": w.Nk, "d": w.d, "causal": w.causal, "window": w.window,
                        "align": w.align},
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
-                             "sample": sample},
+                             "sample": sample,
+                             "rows_per_s": steps * rows_per_step / t_total,
+                             "full_workload_s_extrapolated":
+                                 t_total * total_rows / (steps * rows_per_step)},
             "e2e": {"value": value, "unit": unit, "h2d_bytes_per_step": 0,
                     "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)

@@ -47,3 +47,15 @@ def test_window_flops_count_visible_pairs():
     lw = synth.WORKLOADS["long_window"]
     N, W = lw.Nq, lw.window
     assert lw.flops() == 4.0 * lw.B * lw.Hq * lw.d * (W * (W + 1) // 2 + (N - W) * W)
+
+
+def test_cpu_baseline_entry_reports_rate_and_extrapolation():
+    w = synth.WORKLOADS["tiny_causal"]
+    e = bench.cpu_baseline_entry(w, "TFLOP/s", seconds=0.05)
+    assert e["kind"] == "oracle" and e["cores"] >= 1 and e["value"] > 0
+    assert e["unit"].startswith("TFLOP/s")
+    # rows/s times the extrapolated time is the workload's row count
+    total_rows = w.B * w.Hq * w.Nq
+    assert abs(e["rows_per_s"] * e["full_workload_s_extrapolated"] - total_rows) < 1e-6 * total_rows
+    g = bench.cpu_baseline_entry(w, "GB/s", seconds=0.05)
+    assert g["unit"].startswith("GB/s") and g["value"] > 0
