@@ -13,8 +13,8 @@ import ctypes
 import math
 import os
 
-__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_fwd_paged", "attn_fwd_rope",
-           "attn_fwd_decode_static", "rope_apply",
+__all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_set_workspace",
+           "attn_fwd_paged", "attn_fwd_rope", "attn_fwd_decode_static", "rope_apply",
            "prefill_tile_shape", "tile_plan", "device_status", "AttnError", "lib",
            "STATUS_NAMES"]
 
@@ -61,6 +61,8 @@ def lib():
         L.attn_rope_workspace_size.restype = sz
         L.attn_workspace_size.argtypes = [i, i, i, i, i, i]
         L.attn_workspace_size.restype = sz
+        L.attn_set_workspace.argtypes = [vp, sz]
+        L.attn_set_workspace.restype = i
         L.rope_apply.argtypes = [vp, vp, i, i, i, i, f, i, i, vp]
         L.rope_apply.restype = i
         L.attn_prefill_tile_shape.argtypes = [i, ctypes.POINTER(i), ctypes.POINTER(i)]
@@ -167,6 +169,30 @@ def attn_fwd(q, k, v, causal=False, scale=None, key_lens=None, out=None, lse=Non
                         _stream(stream))
     _raise(rc, "attn_fwd")
     return (out, lse) if return_lse else out
+
+
+_registered_ws = {}   # device index -> the tensor registered there (kept alive)
+
+
+def attn_set_workspace(workspace=None, device=None):
+    """Register a caller-owned uint8 CUDA tensor (256-byte aligned) as the
+    workspace of attn_fwd on its device, or, with None, go back to the
+    library's own workspace on `device` (default: the current device).  The
+    tensor is kept referenced here while it is registered."""
+    torch = _torch()
+    if workspace is None:
+        dev = torch.cuda.current_device() if device is None else torch.device(device).index
+        with torch.cuda.device(dev):
+            rc = lib().attn_set_workspace(None, 0)
+        _raise(rc, "attn_set_workspace")
+        _registered_ws.pop(dev, None)
+        return
+    _check_tensor(workspace, "workspace", torch.uint8, 1)
+    dev = workspace.device.index
+    with torch.cuda.device(dev):
+        rc = lib().attn_set_workspace(_ptr(workspace), workspace.numel())
+    _raise(rc, "attn_set_workspace")
+    _registered_ws[dev] = workspace
 
 
 def attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) -> int:

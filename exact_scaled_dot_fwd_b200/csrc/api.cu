@@ -46,10 +46,13 @@ int current_sms() {
   return n;
 }
 
-// Library-owned decode workspace, one per device, grown on demand.
+// attn_fwd's workspace, one per device: the library's own (grown on demand)
+// unless the caller registered a buffer of its own with attn_set_workspace.
 struct OwnedWorkspace {
   void* ptr = nullptr;
   size_t bytes = 0;
+  void* user = nullptr;     // caller-owned, never freed here
+  size_t user_bytes = 0;
 };
 constexpr int kMaxDevices = 64;
 OwnedWorkspace g_ws[kMaxDevices];
@@ -290,7 +293,12 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ECUDA;
     std::lock_guard<std::mutex> lock(g_ws_mu);
     OwnedWorkspace& w = g_ws[dev];
-    if (w.bytes < need) {
+    if (w.user) {
+      // a registered buffer is never replaced behind the caller's back
+      if (w.user_bytes < need) return ATTN_EWORKSPACE;
+      ws = w.user;
+      ws_bytes = w.user_bytes;
+    } else if (w.bytes < need) {
       // the old buffer may still be in use by queued work on some stream
       if (w.ptr && cudaDeviceSynchronize() != cudaSuccess) return ATTN_ECUDA;
       if (w.ptr) cudaFree(w.ptr);
@@ -302,8 +310,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
       }
       w.bytes = need;
     }
-    ws = w.ptr;
-    ws_bytes = w.bytes;
+    if (!w.user) {
+      ws = w.ptr;
+      ws_bytes = w.bytes;
+    }
   }
   return attn_fwd_ws(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, key_lens, ws, ws_bytes,
                      stream);
@@ -361,6 +371,17 @@ int attn_debug_timeout_probe(unsigned long long limit_ns, void* stream) {
   if (limit_ns == 0 || limit_ns > 1000000000ull) return ATTN_EINVAL;
   timeout_probe_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(limit_ns);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
+int attn_set_workspace(void* ptr, size_t bytes) {
+  if ((ptr == nullptr) != (bytes == 0)) return ATTN_EINVAL;
+  if ((reinterpret_cast<uintptr_t>(ptr) & 255u) != 0) return ATTN_EALIGN;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return ATTN_ECUDA;
+  std::lock_guard<std::mutex> lock(g_ws_mu);
+  g_ws[dev].user = ptr;
+  g_ws[dev].user_bytes = bytes;
+  return ATTN_OK;
 }
 
 int attn_device_status(void* stream, int reset) {

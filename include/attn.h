@@ -73,10 +73,12 @@ typedef enum {
  *   partial results; prefill: the work-item counter of its scheduler, zeroed
  *   in-stream before each launch): this entry point uses a workspace owned by
  *   the library (allocated on first use per device, grown on demand, released
- *   at process exit); calls that overlap on the GPU share it and must not run
- *   concurrently -- use attn_fwd_ws for concurrent streams.
+ *   at process exit), or the caller's buffer registered for the current
+ *   device with attn_set_workspace; calls that overlap on the GPU share it and
+ *   must not run concurrently -- use attn_fwd_ws for concurrent streams.
  * Errors: ATTN_EINVAL / EUNSUPPORTED / EALIGN before any launch; ATTN_ECUDA
- * if a launch or the workspace allocation fails. */
+ * if a launch or the workspace allocation fails; ATTN_EWORKSPACE if a
+ * registered workspace is smaller than attn_workspace_size(...). */
 ATTN_API int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
              int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
              float scale, const int32_t* key_lens, void* stream);
@@ -155,6 +157,24 @@ ATTN_API int attn_fwd_window(const void* q, const void* k, const void* v, void* 
  * (0 for invalid sizes). */
 ATTN_API size_t attn_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d);
 
+/* Registers a caller-owned DEVICE buffer as attn_fwd's workspace on the
+ * current device, in place of the library's own; ptr = NULL with bytes = 0
+ * returns to the library's own.  (The pages define no library interface;
+ * this is the allocation side of the boundary, for callers that manage device
+ * memory themselves.)
+ *   ptr: 256-byte aligned, bytes > 0; the library never frees it, never grows
+ *   it and never allocates in its place: an attn_fwd call that needs more
+ *   than `bytes` (attn_workspace_size) returns ATTN_EWORKSPACE before any
+ *   launch.  The caller keeps the buffer alive, and untouched by other work,
+ *   until every attn_fwd call that used it has completed on its stream and it
+ *   has been unregistered or replaced.  Registration is per device and
+ *   process-wide (all threads); it does not affect attn_fwd_ws and the other
+ *   entry points that take their workspace as an argument.
+ * Errors: ATTN_EINVAL if exactly one of ptr / bytes is zero, ATTN_EALIGN for
+ * a misaligned ptr (both before any CUDA call), ATTN_ECUDA if no device is
+ * current. */
+ATTN_API int attn_set_workspace(void* ptr, size_t bytes);
+
 /* RoPE prologue ("Transformer Architecture Breakdown ...", section 3.1;
  * "Coding interview (14)", section 3.5): for each row x of x_in at position
  * t = pos_offset + row index along N, and i = 0..d/2-1,
@@ -174,8 +194,9 @@ ATTN_API int rope_apply(const void* x_in, void* x_out, int B, int H, int N, int 
  * rope_apply would store), then attends.  k must hold keys already rotated
  * (rope_apply at their positions; a KV cache stores them that way).
  *   Prefill shapes rotate each Q tile in shared memory after its TMA load
- *   (the prefill kernel's Q producer warp), with a (cos, sin) table of the
- *   Nq positions built in the workspace; decode shapes ((Hq/Hkv) * Nq <= 64)
+ *   (each thread of the tile's softmax warpgroup rotates its own row), with a
+ *   (cos, sin) table of the Nq positions built in the workspace; decode
+ *   shapes ((Hq/Hkv) * Nq <= 64)
  *   rotate q into the workspace and run the decode kernels.
  *   rope_base > 0, rope_pairing 0 (i, i + d/2) or 1 (2i, 2i + 1),
  *   q_pos_offset >= 0.  Workspace: attn_rope_workspace_size(...) bytes

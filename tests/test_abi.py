@@ -177,3 +177,12 @@ def test_fused_rope_rejects_bad_arguments_on_host(L):
     assert f(*args, 1e4, 0, -1, P, need, None) == 1           # position offset
     assert f(*args, 1e4, 0, 0, P, need - 1, None) == 4        # workspace too small
     assert f(*args, 1e4, 0, 0, ctypes.c_void_p(0x1010), need, None) == 3
+
+
+def test_set_workspace_rejects_bad_arguments_on_host(L):
+    # only the checks made before any CUDA call: a pointer without a size, a
+    # size without a pointer, a pointer off a 256-byte boundary
+    assert L.attn_set_workspace(P, 0) == 1
+    assert L.attn_set_workspace(None, 256) == 1
+    assert L.attn_set_workspace(ctypes.c_void_p(0x1010), 256) == 3
+    assert L.attn_set_workspace(ctypes.c_void_p(0x1080), 4096) == 3
