@@ -15,7 +15,10 @@
 // Work split.  Unit u = (b, kv head h) owns len_u = clamp(key_lens[b], 0, Nk)
 // keys.  The units' keys are laid end to end (T keys in total) and CTA c of a
 // one-wave grid takes the global key range [c*T/G, (c+1)*T/G), which may cover
-// the tail of one unit and the head of the next.  Each (CTA, unit) piece is a
+// the tail of one unit and the head of the next.  Every non-empty unit is
+// laid out with seg_cost virtual keys in front of its real ones (about the
+// cost of starting a segment, in keys), so a CTA whose range spans many short
+// units gets fewer real keys.  Each (CTA, unit) piece is a
 // segment: the CTA runs the online-softmax recurrence over it and writes a
 // partial (O_s / l_s, log2 l_s + m_s) into slot c + u (unique: a later CTA
 // never touches an earlier unit).  The combine pass merges the slots of each

@@ -13,9 +13,10 @@
 // at once; "Coding interview (14)", self-test 5), R = G * Nq <= 64; these rows
 // are contiguous in q, o and lse.  One softmax thread owns one
 // key (one TMEM lane of S^T) and, for O^T, one dimension of d.  The per-head
-// maximum over the tile's keys is a butterfly transpose-reduce across the
-// warp plus a four-entry exchange in shared memory; per-head running sums
-// stay per thread until the segment ends.  P^T goes to shared memory (bf16,
+// maximum over the tile's keys is one warp-wide redux.sync max per head plus
+// a four-entry exchange (one per warp) in shared memory; per-head running
+// sums stay per thread until the segment ends, where a butterfly
+// transpose-reduce across the warp sums them.  P^T goes to shared memory (bf16,
 // the B operand of the PV MMA).  S^T is double-buffered in TMEM, so the S MMA
 // of tile j+2 and the loads run while the softmax works on tile j.
 //
