@@ -26,6 +26,7 @@ import argparse
 import json
 import math
 import os
+import re
 import statistics
 import subprocess
 import sys
@@ -46,24 +47,37 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM traffic per launch of the dominant kernel, from one ncu capture each
 # (dram__bytes_read.sum + dram__bytes_write.sum; summaries in profiles/),
 # with a hash of the kernel's source files at capture time.  The figure is
-# reported only while the sources still hash the same.
+# reported only while the sources still hash the same.  The hash covers the
+# code only: comments are dropped and whitespace runs collapse to one space,
+# so a comment edit keeps the capture while any change to the code voids it.
 KERNEL_SOURCES = {
     "prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh", "rope_math.cuh"],
     "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
 }
 NCU_TRAFFIC = {
     # workload: (kernel, source hash, bytes per launch)
-    "mha_prefill": ("prefill", "e4d5e81ff50a5429", 131482624 + 11721472),
-    "mqa_decode": ("decode", "6d67e14f67118d61", 322994688 + 4797952),
+    "mha_prefill": ("prefill", "2196b26240cb2407", 131482624 + 11721472),
+    "mqa_decode": ("decode", "3f64d81e21fa07a0", 322994688 + 4797952),
 }
+
+
+_COMMENT_OR_LITERAL = re.compile(r'//[^\n]*|/\*.*?\*/|"(?:\\.|[^\\"\n])*"|\'(?:\\.|[^\\\'\n])*\'',
+                                 re.S)
+
+
+def code_tokens(src):
+    """C/C++/CUDA source without comments (string and character literals
+    kept as written), whitespace runs collapsed to one space."""
+    kept = _COMMENT_OR_LITERAL.sub(lambda m: m.group(0) if m.group(0)[0] in "\"'" else " ", src)
+    return " ".join(kept.split())
 
 
 def source_hash(kernel):
     import hashlib
     m = hashlib.sha256()
     for f in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(ROOT, "exact_scaled_dot_fwd_b200", "csrc", f), "rb") as fh:
-            m.update(fh.read())
+        with open(os.path.join(ROOT, "exact_scaled_dot_fwd_b200", "csrc", f)) as fh:
+            m.update(code_tokens(fh.read()).encode())
     return m.hexdigest()[:16]
 
 

@@ -59,3 +59,24 @@ def test_cpu_baseline_entry_reports_rate_and_extrapolation():
     assert abs(e["rows_per_s"] * e["full_workload_s_extrapolated"] - total_rows) < 1e-6 * total_rows
     g = bench.cpu_baseline_entry(w, "GB/s", seconds=0.05)
     assert g["unit"].startswith("GB/s") and g["value"] > 0
+
+
+def test_traffic_hash_follows_code_not_comments():
+    src = ('int f(int x) {  // doubles x\n'
+           '  /* block\n     comment */ return 2 * x;\n}\n'
+           'const char* s = "// kept: inside a string";\n')
+    base = bench.code_tokens(src)
+    assert "doubles" not in base and "block" not in base
+    assert "// kept: inside a string" in base
+    # comment text, comment layout and blank lines do not matter ...
+    assert bench.code_tokens(src.replace("doubles x", "returns twice x\n\n// more")) == base
+    assert bench.code_tokens(src.replace("  return", "\n\n  return")) == base
+    # ... the code does
+    assert bench.code_tokens(src.replace("2 * x", "3 * x")) != base
+    assert bench.code_tokens(src.replace("inside a string", "inside a strinG")) != base
+
+
+def test_stored_traffic_matches_current_kernels():
+    # the stored captures belong to the kernels as they are now
+    assert bench.ncu_traffic("mha_prefill") is not None
+    assert bench.ncu_traffic("mqa_decode") is not None
