@@ -77,6 +77,8 @@ def test_traffic_hash_follows_code_not_comments():
 
 
 def test_stored_traffic_matches_current_kernels():
-    # the stored captures belong to the kernels as they are now
+    # The stored captures belong to the kernels' code as it is now.  A change
+    # to a kernel's code fails this test until its traffic is captured again
+    # (ncu) and stored with the new hash.
     assert bench.ncu_traffic("mha_prefill") is not None
     assert bench.ncu_traffic("mqa_decode") is not None
