@@ -186,3 +186,15 @@ def test_set_workspace_rejects_bad_arguments_on_host(L):
     assert L.attn_set_workspace(None, 256) == 1
     assert L.attn_set_workspace(ctypes.c_void_p(0x1010), 256) == 3
     assert L.attn_set_workspace(ctypes.c_void_p(0x1080), 4096) == 3
+
+
+def test_size_limits_rejected_on_host(L):
+    # flat row counts must stay below 2^31 (int32 indexing inside the kernels)
+    assert fwd(L, B=1 << 16, Hq=1 << 14, Hkv=1 << 14, Nq=2, Nk=2) == 2      # B*Hq*Nq = 2^31
+    assert fwd(L, B=1, Hq=2, Hkv=2, Nq=8, Nk=1 << 30) == 2                # B*Hkv*Nk = 2^31
+    # paged: logical capacity and physical cache rows
+    pg = L.attn_fwd_paged
+    assert pg(P, P, P, P, 1 << 20, 1 << 11, 4, P, None, 1, 2, 1, 1, 128, 0, 0, 0.1, P,
+              None, 0, None) == 2                                           # max_pages*page = 2^31
+    assert pg(P, P, P, P, 4, 16, 1 << 27, P, None, 1, 2, 1, 1, 128, 0, 0, 0.1, P,
+              None, 0, None) == 2                                           # num_pages*Hkv*page = 2^31
