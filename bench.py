@@ -110,6 +110,22 @@ def parse_args():
     return p.parse_args()
 
 
+# B200 datasheet figures (dense bf16 tensor, HBM3e): context beside the
+# measured peaks, which are the roofline denominators.
+NOMINAL_PEAKS = {"tensor": 2250.0, "hbm": 8000.0}
+
+
+def roofline(bound, achieved, peaks, peak_src, workload):
+    """The roofline object of a bench line: `achieved` against the measured
+    peak (frac) and, labelled separately, against the nominal one."""
+    peak = peaks["bf16_tflops"] if bound == "tensor" else peaks["hbm_gbs"]
+    nominal = NOMINAL_PEAKS[bound]
+    return {"bound": bound, "achieved": achieved, "peak": peak,
+            "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak,
+            "traffic": ncu_traffic(workload), "peak_source": peak_src,
+            "nominal_peak": nominal, "frac_of_nominal": achieved / nominal}
+
+
 def load_peaks():
     path = os.path.join(ROOT, "MEASURED_PEAKS.json")
     try:
@@ -374,16 +390,12 @@ def run_ours(args):
         unit, work = "GB/s", decode_bytes(w, x["key_lens"])
         value = world * work * steps / (ms / 1e3) / 1e9
         kval = work * steps / (ms_kernel / 1e3) / 1e9
-        roof = {"bound": "hbm", "achieved": kval, "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": kval / peaks["hbm_gbs"],
-                "traffic": ncu_traffic(w.name), "peak_source": peak_src}
+        roof = roofline("hbm", kval, peaks, peak_src, w.name)
     else:
         unit, work = "TFLOP/s", w.flops()
         value = world * work * steps / (ms / 1e3) / 1e12
         kval = work * steps / (ms_kernel / 1e3) / 1e12
-        roof = {"bound": "tensor", "achieved": kval, "peak": peaks["bf16_tflops"],
-                "unit": "TFLOP/s", "frac": kval / peaks["bf16_tflops"],
-                "traffic": ncu_traffic(w.name), "peak_source": peak_src}
+        roof = roofline("tensor", kval, peaks, peak_src, w.name)
     line = {
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
@@ -492,9 +504,7 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa
             "page_size": page_size or None,
             "algorithmic_bytes": decode_bytes(w, x["key_lens"]),
             "l2": f"{copies} rotating KV caches ({copies * per_copy / 1e6:.0f} MB allocated)",
-            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": gbs / peaks["hbm_gbs"],
-                         "traffic": ncu_traffic(w.name), "peak_source": peak_src},
+            "roofline": roofline("hbm", gbs, peaks, peak_src, w.name),
             "gpu_launches": 2 * n}
 
 
@@ -566,9 +576,7 @@ def run_window(torch, eb, device, stream, peaks, peak_src, steps=None):
             "unit": "TFLOP/s", "workload": w.name, "window": w.window, "steps": n,
             "ms_per_step": ms / n, "flops_per_step": w.flops(),
             "l2": f"inputs {mb:.0f} MB > 126 MB L2",
-            "roofline": {"bound": "tensor", "achieved": tf, "peak": peaks["bf16_tflops"],
-                         "unit": "TFLOP/s", "frac": tf / peaks["bf16_tflops"],
-                         "traffic": ncu_traffic(w.name), "peak_source": peak_src},
+            "roofline": roofline("tensor", tf, peaks, peak_src, w.name),
             "gpu_launches": n}
 
 

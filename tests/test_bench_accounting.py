@@ -82,3 +82,15 @@ def test_stored_traffic_matches_current_kernels():
     # (ncu) and stored with the new hash.
     assert bench.ncu_traffic("mha_prefill") is not None
     assert bench.ncu_traffic("mqa_decode") is not None
+
+
+def test_roofline_object_reports_measured_and_nominal_fractions():
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1400.0}
+    t = bench.roofline("tensor", 750.0, peaks, "measured", "no_such_workload")
+    assert t["unit"] == "TFLOP/s" and t["peak"] == 1500.0 and abs(t["frac"] - 0.5) < 1e-12
+    assert t["nominal_peak"] == 2250.0 and abs(t["frac_of_nominal"] - 750.0 / 2250.0) < 1e-12
+    assert t["traffic"] is None                     # no capture stored for this workload
+    h = bench.roofline("hbm", 4800.0, peaks, "fallback", "mqa_decode")
+    assert h["unit"] == "GB/s" and abs(h["frac"] - 0.8) < 1e-12 and h["peak_source"] == "fallback"
+    assert abs(h["frac_of_nominal"] - 0.6) < 1e-12
+    assert h["traffic"] == bench.ncu_traffic("mqa_decode")
