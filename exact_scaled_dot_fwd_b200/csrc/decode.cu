@@ -14,7 +14,8 @@
 //
 // Work split.  Unit u = (b, kv head h) owns len_u = clamp(key_lens[b], 0, Nk)
 // keys.  The units' keys are laid end to end (T keys in total) and CTA c of a
-// one-wave grid takes the global key range [c*T/G, (c+1)*T/G), which may cover
+// one-wave grid of `grid` CTAs takes the global key range
+// [c*T/grid, (c+1)*T/grid), which may cover
 // the tail of one unit and the head of the next.  Every non-empty unit is
 // laid out with seg_cost virtual keys in front of its real ones (about the
 // cost of starting a segment, in keys), so a CTA whose range spans many short
