@@ -9,11 +9,13 @@
  *
  *   [CIA] "Coding interview (14): attention from scratch" (arganzheng.life),
  *         sections 3.1 softmax, 3.2 sdpa, 3.4 GQA, 3.5 RoPE, 3.6 KV cache,
- *         3.7 online softmax.
+ *         3.7 online softmax; self-test 5 (new tokens after a cache).
  *   [TAB] "Transformer Architecture Breakdown: Self-Attention, MHA/GQA/MQA,
  *         RoPE & FlashAttention 1/2/3" (airsota.com), sections 1.2, 3.1, 4.2.
  *   [AME] "Attention mechanisms: from alignment to efficient long context"
- *         (fahimfaisal.info), sections 3, 5, 9, 19.
+ *         (fahimfaisal.info), sections 3, 5, 9, 11 sliding window, 19,
+ *         20 PagedAttention.
+ *   [TIN] "Transformer Internals" (vanos001.github.io), Paged Attention.
  *   [TAD] "Transformer Architecture Deconstructed: Attention, Geometric
  *         Scaling, and Memory IO" (byronfinn.github.io), "Online Softmax and
  *         Blocked Incremental Computation".
