@@ -266,8 +266,8 @@ def to_dev(bits, torch, device):
 
 
 def memory_bound(w):
-    """Decode-shaped workloads (at most 64 query rows per kv head) are judged
-    on HBM bytes; the rest on tensor FLOPs."""
+    """Decode-shaped workloads (at most 64 query rows per kv head) are measured
+    in HBM bytes; the rest in tensor FLOPs."""
     return w.Nq * (w.Hq // w.Hkv) <= 64
 
 

@@ -60,7 +60,7 @@ std::mutex g_ws_mu;
 
 struct WorkspaceReaper {
   ~WorkspaceReaper() {
-    // process exit: the driver may already be tearing down; ignore errors
+    // process exit: the CUDA driver may already be tearing down; ignore errors
     for (auto& w : g_ws)
       if (w.ptr) cudaFree(w.ptr);
   }
@@ -134,7 +134,7 @@ const char* attn_strerror(int status) {
   switch (status) {
     case ATTN_OK: return "ATTN_OK";
     case ATTN_EINVAL: return "ATTN_EINVAL: invalid argument";
-    case ATTN_EUNSUPPORTED: return "ATTN_EUNSUPPORTED: shape not supported by this build";
+    case ATTN_EUNSUPPORTED: return "ATTN_EUNSUPPORTED: shape not supported by this library";
     case ATTN_EALIGN: return "ATTN_EALIGN: pointer not 16-byte aligned";
     case ATTN_EWORKSPACE: return "ATTN_EWORKSPACE: workspace missing or too small";
     case ATTN_ECUDA: return "ATTN_ECUDA: CUDA call failed";

@@ -54,7 +54,7 @@ extern "C" {
 typedef enum {
   ATTN_OK = 0,
   ATTN_EINVAL = 1,        /* null required pointer, bad size, Hq % Hkv != 0, bad scale */
-  ATTN_EUNSUPPORTED = 2,  /* a shape this build does not implement (e.g. d not 64/128) */
+  ATTN_EUNSUPPORTED = 2,  /* a shape this library does not implement (e.g. d not 64/128) */
   ATTN_EALIGN = 3,        /* a pointer not 16-byte aligned */
   ATTN_EWORKSPACE = 4,    /* workspace missing or smaller than attn_workspace_size() */
   ATTN_ECUDA = 5,         /* a CUDA runtime / driver call failed (launch, attribute) */

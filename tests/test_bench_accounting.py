@@ -1,4 +1,4 @@
-"""bench.py's work accounting on the CPU: which workloads are judged on HBM
+"""bench.py's work accounting on the CPU: which workloads are measured in HBM
 bytes, the algorithmic bytes of a decode step, and the FLOPs of a windowed
 workload, each against a count made independently here."""
 import os

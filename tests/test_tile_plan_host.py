@@ -25,7 +25,7 @@ import oracle
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 CSRC = os.path.join(ROOT, "exact_scaled_dot_fwd_b200", "csrc")
 
-DRIVER = r"""
+WRAPPER = r"""
 #define __host__
 #define __device__
 #define __forceinline__ inline
@@ -54,8 +54,8 @@ def P(tmp_path_factory):
     if gxx is None:
         pytest.skip("g++ not available")
     d = tmp_path_factory.mktemp("tile_plan")
-    src = d / "driver.cpp"
-    src.write_text(DRIVER)
+    src = d / "wrapper.cpp"
+    src.write_text(WRAPPER)
     so = d / "libplan.so"
     subprocess.run([gxx, "-std=c++17", "-O1", "-fPIC", "-shared", "-I", CSRC, str(src), "-o",
                     str(so)], check=True, capture_output=True)
