@@ -76,3 +76,24 @@ def test_to_paged_round_trip():
     last = table[0, (Nk - 1) // page_size]
     pad = synth.bf16_bits_from_f32(np.array([synth.PAD_SENTINEL], np.float32))[0]
     assert np.all(cache[last, :, Nk % page_size:, :] == pad)
+
+
+def test_sample_rows_cover_edges_of_every_head():
+    w = synth.WORKLOADS["gqa_rope_prefill"]
+    rows = synth.sample_rows(w, per_head_random=23)
+    N = w.Nq
+    assert np.all(np.diff(rows) > 0)                     # sorted, unique
+    assert rows.min() >= 0 and rows.max() < w.B * w.Hq * N
+    by_head = {}
+    for r in rows:
+        by_head.setdefault(int(r) // N, set()).add(int(r) % N)
+    assert sorted(by_head) == list(range(w.B * w.Hq))
+    edges = {0, 1, 127, 128, 129, 255, 256, N - 129, N - 1}
+    for bh, got in by_head.items():
+        assert edges <= got, bh
+        assert len(got) <= len(edges) + 23
+    assert np.array_equal(rows, synth.sample_rows(w, per_head_random=23))
+    # short sequences keep only the edge rows that exist
+    tiny = synth.WORKLOADS["tiny"]
+    t = synth.sample_rows(tiny, per_head_random=0)
+    assert set(int(r) % tiny.Nq for r in t) == {0, 1, 127, 128, 129, 255, tiny.Nq - 129}
