@@ -62,8 +62,9 @@ typedef enum {
 } attn_status;
 
 /* Exact attention forward.  Dispatch: calls with at most 64 query rows per kv
- * head ((Hq / Hkv) * Nq <= 64: single-token decode, multi-token decode) run
- * the split-KV decode kernel followed by the log-sum-exp combine pass; all
+ * head ((Hq / Hkv) * Nq <= 64: single-token decode, multi-token decode) and
+ * B <= 2048 run the split-KV decode kernel followed by the log-sum-exp
+ * combine pass; all
  * others run the tiled prefill kernel (TMA + tcgen05/TMEM, persistent, one
  * CTA per SM).
  *   d: 64 or 128.  scale: finite and > 0 (usually 1/sqrt(d); "Transformer
@@ -130,15 +131,18 @@ ATTN_API int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, f
  *   q/o bf16 [B, Hq, Nq, d], lse fp32 [B, Hq, Nq] or NULL.  The Nq query rows
  *   of a sequence are its newest Nq tokens (ATTN_ALIGN_KEYLEN of attn_fwd_ex);
  *   causal and window as there, with Nk = max_pages * page_size.
- *   Runs the split-KV decode kernels: (Hq / Hkv) * Nq <= 64.  page_size: a
+ *   Runs the split-KV decode kernels: (Hq / Hkv) * Nq <= 64, B <= 2048.  page_size: a
  *   multiple of 8 dividing 128 (d = 128) or 64 (d = 64) -- 8, 16, 32, 64
  *   (and 128 for d = 128).  Only entries j / page_size < ceil(key_lens[b] /
  *   page_size) of a sequence's table row are read; rows of its last page at
- *   or beyond key_lens[b] must hold finite values.  A table entry outside
- *   [0, num_pages) reads zeros (the kernels do not check it).
+ *   or beyond key_lens[b] must hold finite values.  The kernels do not
+ *   check table entries: one outside [0, num_pages) reads zeros, or, when
+ *   (entry * Hkv + h) * page_size overflows 32 bits, some other page of the
+ *   cache; no entry makes a kernel read outside k_cache / v_cache.
  *   Workspace: attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) bytes.
  * Errors: ATTN_EINVAL (null table or key_lens, bad sizes), ATTN_EUNSUPPORTED
- * (page_size, more than 64 query rows per kv head, d), then as attn_fwd_ws. */
+ * (page_size, more than 64 query rows per kv head or 2048 sequences, d), then
+ * as attn_fwd_ws. */
 ATTN_API int attn_fwd_paged(const void* q, const void* k_cache, const void* v_cache,
                             const int32_t* block_table, int max_pages, int page_size,
                             int num_pages, void* o, float* lse, int B, int Hq, int Hkv,
