@@ -15,8 +15,8 @@ import os
 
 __all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_set_workspace",
            "attn_fwd_paged", "attn_fwd_rope", "attn_fwd_decode_static", "rope_apply",
-           "prefill_tile_shape", "tile_plan", "device_status", "AttnError", "lib",
-           "STATUS_NAMES"]
+           "prefill_tile_shape", "tile_plan", "device_status", "attn_last_device_status",
+           "AttnError", "lib", "STATUS_NAMES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 LIB_PATH = os.path.join(_HERE, "libattn_b200.so")
@@ -75,6 +75,8 @@ def lib():
         L.attn_fwd_tile_plan_ex.restype = i
         L.attn_device_status.argtypes = [vp, i]
         L.attn_device_status.restype = i
+        L.attn_last_device_status.argtypes = [vp]
+        L.attn_last_device_status.restype = i
         L.attn_strerror.argtypes = [i]
         L.attn_strerror.restype = ctypes.c_char_p
         L.attn_abi_version.argtypes = []
@@ -360,3 +362,8 @@ def tile_plan(B, Nq, Nk, d, causal, key_lens=None, device="cuda", stream=None, w
 def device_status(reset=True, stream=None) -> int:
     """Synchronise and read the library's device status word (0 = OK)."""
     return int(lib().attn_device_status(_stream(stream), int(bool(reset))))
+
+
+def attn_last_device_status(stream=None) -> int:
+    """Synchronise, return the status since the last read and clear it."""
+    return int(lib().attn_last_device_status(_stream(stream)))

@@ -373,6 +373,8 @@ int attn_debug_timeout_probe(unsigned long long limit_ns, void* stream) {
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 
+int attn_last_device_status(void* stream) { return attn_device_status(stream, 1); }
+
 int attn_set_workspace(void* ptr, size_t bytes) {
   if ((ptr == nullptr) != (bytes == 0)) return ATTN_EINVAL;
   if ((reinterpret_cast<uintptr_t>(ptr) & 255u) != 0) return ATTN_EALIGN;

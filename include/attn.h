@@ -272,6 +272,10 @@ ATTN_API size_t attn_decode_static_max_bytes(void);
  * clears the device status word. */
 ATTN_API int attn_device_status(void* stream, int reset);
 
+/* attn_device_status(stream, 1): the status since the last read, then
+ * cleared (read-and-clear, like cudaGetLastError). */
+ATTN_API int attn_last_device_status(void* stream);
+
 /* Failure-detection test hook: launches one tiny kernel whose single thread
  * waits on a barrier that nothing ever completes, giving up after limit_ns
  * (1 ns .. 1 s).  The wait's limit expires, the kernel records ATTN_ETIMEOUT

@@ -28,6 +28,10 @@ def test_wait_limit_reports_timeout_and_context_survives():
     assert L.attn_debug_timeout_probe(ctypes.c_ulonglong(20_000_000), stream) == 0
     assert eb.device_status(reset=True) == 6          # ATTN_ETIMEOUT
     assert eb.device_status(reset=True) == 0          # cleared
+    # the same through the read-and-clear entry point
+    assert L.attn_debug_timeout_probe(ctypes.c_ulonglong(20_000_000), stream) == 0
+    assert eb.attn_last_device_status() == 6
+    assert eb.attn_last_device_status() == 0
     # the context is intact: a normal call still matches the oracle
     B, H, N, d = 1, 2, 200, 64
     q = synth.normal_bf16((B, H, N, d), 1)
