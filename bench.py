@@ -3,22 +3,25 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--config NAME] [--impl ours|reference]
 
-One step = one attn_fwd call over one batch of the workload (default: causal
-MHA prefill, B=4, H=16, N=2048, d=128).  Inputs are resident in HBM; each
-step reads one of several input copies whose total exceeds the 126 MB L2, so
-no step finds its inputs in cache.  W untimed warm-up steps precede K timed
-steps bracketed by a barrier and a device synchronisation; the time is the
-maximum over ranks of CUDA-event time on the launching stream.  For N > 1
-(torchrun) every rank runs an independent batch (weak scaling, no
-collective on the data path).
+One step = one pass of the hot path over one batch of the workload (default:
+the long-context causal prefill, B=1, H=32, N=32768, d=128, the largest
+single-GPU configuration).  Inputs are resident in HBM; each step reads one
+of several input copies whose total exceeds the 126 MB L2 (one copy when a
+single one already does), so no step finds its inputs in cache.  W untimed
+warm-up steps precede K timed steps bracketed by a barrier and a device
+synchronisation; the time is the maximum over ranks of CUDA-event time on
+the launching stream.  For N > 1 (torchrun) every rank runs an independent
+batch (weak scaling, no collective on the data path).
 
-The JSON line also carries: the roofline of the dominant kernel, the
+The JSON line also carries: the roofline of the dominant kernel (with the
+stored ncu counters of its capture while the kernel code is unchanged), the
 end-to-end figure through the public API with host buffers, the oracle timed
 on host cores (rank 0, N=1, bounded sample), SM clocks sampled during the
-timed region, the decode workload (MQA over a ragged KV cache) in GB/s, and
-the sliding-window prefill workload in useful TFLOP/s, the multi-token and
-paged decode workloads, and the GQA RoPE prefill step with separate RoPE
-passes and with q's RoPE fused into the attention kernel.
+timed region, the decode workload (MQA over a ragged KV cache) in GB/s, the
+sliding-window prefill workload in useful TFLOP/s, the multi-token and paged
+decode workloads, the GQA RoPE prefill step with separate RoPE passes and
+with q's RoPE fused into the attention kernel, and the attention kernel alone
+on the other prefill workloads (MHA prefill, padded cross attention, GQA).
 """
 from __future__ import annotations
 
@@ -54,10 +57,18 @@ KERNEL_SOURCES = {
     "prefill": ["prefill.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh", "rope_math.cuh"],
     "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
 }
+# workload: (kernel, source hash, DRAM bytes read + written per launch).
 NCU_TRAFFIC = {
-    # workload: (kernel, source hash, bytes per launch)
     "mha_prefill": ("prefill", "2196b26240cb2407", 131482624 + 11721472),
     "mqa_decode": ("decode", "3f64d81e21fa07a0", 322994688 + 4797952),
+}
+# Further counters of the same captures (same keys and hash rule): the
+# tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
+# % of peak over the launch) and the DRAM throughput of a decode launch
+# (dram__bytes.sum.per_second, GB/s).
+NCU_COUNTERS = {
+    "mha_prefill": ("prefill", "2196b26240cb2407", {"tensor_pipe_pct": 31.5}),
+    "mqa_decode": ("decode", "3f64d81e21fa07a0", {"dram_gbs": 5534.0}),
 }
 
 
@@ -81,17 +92,27 @@ def source_hash(kernel):
     return m.hexdigest()[:16]
 
 
+def _stored(table, workload):
+    entry = table.get(workload)
+    if entry is None:
+        return None
+    kernel, digest, value = entry
+    try:
+        return value if source_hash(kernel) == digest else None
+    except OSError:
+        return None
+
+
 def ncu_traffic(workload):
     """Measured DRAM bytes per launch, or None when not captured for this
     workload or when the kernel changed since the capture."""
-    entry = NCU_TRAFFIC.get(workload)
-    if entry is None:
-        return None
-    kernel, digest, nbytes = entry
-    try:
-        return nbytes if source_hash(kernel) == digest else None
-    except OSError:
-        return None
+    return _stored(NCU_TRAFFIC, workload)
+
+
+def ncu_counters(workload):
+    """The other stored counters of the workload's capture ({} when none
+    match the current code)."""
+    return dict(_stored(NCU_COUNTERS, workload) or {})
 
 
 def parse_args():
@@ -99,12 +120,15 @@ def parse_args():
     p.add_argument("--gpus", type=int, default=1)
     p.add_argument("--steps", type=int, default=None)
     p.add_argument("--warmup", type=int, default=5)
-    p.add_argument("--config", default="mha_prefill", choices=sorted(synth.WORKLOADS))
+    p.add_argument("--config", default="long_causal", choices=sorted(synth.WORKLOADS))
     p.add_argument("--impl", default="ours", choices=["ours", "reference"])
     p.add_argument("--no-decode", action="store_true")
     p.add_argument("--no-window", action="store_true")
     p.add_argument("--no-rope", action="store_true")
     p.add_argument("--no-e2e", action="store_true")
+    p.add_argument("--no-extra", action="store_true",
+                   help="skip the other prefill workloads (MHA prefill, padded cross attention, "
+                        "the GQA attention kernel alone)")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
     return p.parse_args()
@@ -117,13 +141,39 @@ NOMINAL_PEAKS = {"tensor": 2250.0, "hbm": 8000.0}
 
 def roofline(bound, achieved, peaks, peak_src, workload):
     """The roofline object of a bench line: `achieved` against the measured
-    peak (frac) and, labelled separately, against the nominal one."""
+    peak (frac) and, labelled separately, against the nominal one; with the
+    stored ncu counters of the workload's dominant kernel when they match
+    the current code."""
     peak = peaks["bf16_tflops"] if bound == "tensor" else peaks["hbm_gbs"]
     nominal = NOMINAL_PEAKS[bound]
-    return {"bound": bound, "achieved": achieved, "peak": peak,
-            "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak,
-            "traffic": ncu_traffic(workload), "peak_source": peak_src,
-            "nominal_peak": nominal, "frac_of_nominal": achieved / nominal}
+    r = {"bound": bound, "achieved": achieved, "peak": peak,
+         "unit": "TFLOP/s" if bound == "tensor" else "GB/s", "frac": achieved / peak,
+         "traffic": ncu_traffic(workload), "peak_source": peak_src,
+         "nominal_peak": nominal, "frac_of_nominal": achieved / nominal}
+    c = ncu_counters(workload)
+    if bound == "tensor":
+        r["ncu_tensor_pipe_pct"] = c.get("tensor_pipe_pct")
+    else:
+        r["ncu_dram_gbs"] = c.get("dram_gbs")
+    return r
+
+
+def config_of(w, copies, per_copy, world):
+    """The line's config object; both arms report the same one."""
+    return {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
+            "Nk": w.Nk, "d": w.d, "causal": w.causal, "rope": w.rope,
+            "key_lens": list(w.key_lens) if w.key_lens else None,
+            "window": w.window, "align": w.align,
+            "l2": f"{copies} rotating input copies ({copies * per_copy / 1e6:.0f} MB > "
+                  f"126 MB L2)",
+            "parallelism": f"replicas x{world} (independent batch per GPU)"}
+
+
+def input_copies(w):
+    """Copies of the inputs a step rotates over so that their total exceeds
+    twice the L2 (1 when one copy already does), and the bytes of one copy."""
+    per_copy = 2 * (w.B * w.Hq * w.Nq * w.d + 2 * w.B * w.Hkv * w.Nk * w.d)
+    return max(1, min(8, math.ceil(2 * L2_BYTES / per_copy))), per_copy
 
 
 def load_peaks():
@@ -336,8 +386,7 @@ def run_ours(args):
     # every rank processes its own batch: shift the seed by the rank
     wr = synth.Workload(**{**w.__dict__, "number": w.number + 100 * rank}) if rank else w
     x = synth.make_inputs(wr)
-    per_copy = sum(x[n].nbytes for n in ("q", "k", "v"))
-    copies = max(1, min(8, math.ceil(2 * L2_BYTES / per_copy)))
+    copies, per_copy = input_copies(w)
     Q = [to_dev(x["q"], torch, device) for _ in range(copies)]
     K = [to_dev(x["k"], torch, device) for _ in range(copies)]
     V = [to_dev(x["v"], torch, device) for _ in range(copies)]
@@ -400,17 +449,14 @@ def run_ours(args):
         "metric": METRIC, "value": value, "unit": unit, "n_gpus": world, "steps": steps,
         "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
-        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
-                   "Nk": w.Nk, "d": w.d, "causal": w.causal, "rope": w.rope,
-                   "key_lens": list(w.key_lens) if w.key_lens else None,
-                   "window": w.window, "align": w.align,
-                   "l2": f"{copies} rotating input copies ({copies * per_copy / 1e6:.0f} MB > "
-                         f"126 MB L2)",
-                   "parallelism": f"replicas x{world} (independent batch per GPU)"},
+        "config": config_of(w, copies, per_copy, world),
         "roofline": roof,
         "gpu_launches": steps * launches_per_step,
         "clocks": clocks,
     }
+    if clocks.get("sm_mhz"):
+        # step time x median SM clock: comparable across runs at different clocks
+        clocks["ms_x_mhz"] = ms_step * clocks["sm_mhz"]
 
     # ---- end to end through the public API with pinned host buffers
     if not args.no_e2e:
@@ -451,6 +497,11 @@ def run_ours(args):
     # ---- GQA prefill with RoPE: separate RoPE passes vs q's RoPE fused
     if not args.no_rope and not w.rope and rank == 0 and world == 1:
         line["rope_prefill"] = run_rope(torch, eb, device, stream, peaks, peak_src)
+    # ---- the other prefill workloads, each its attention kernel alone
+    if not args.no_extra and rank == 0 and world == 1:
+        for name in ("mha_prefill", "cross_padded", "gqa_rope_prefill", "long_causal"):
+            if name != w.name:
+                line[name] = run_prefill(torch, eb, device, stream, peaks, peak_src, name)
 
     # ---- oracle on host cores (rank 0, N=1 only)
     if not args.no_cpu and rank == 0 and world == 1:
@@ -551,6 +602,45 @@ def run_rope(torch, eb, device, stream, peaks, peak_src, steps=None):
     return out
 
 
+def run_prefill(torch, eb, device, stream, peaks, peak_src, name, steps=None):
+    """The attention kernel alone on a prefill workload (inputs rotating over
+    copies larger than L2; a RoPE workload's q and k are rotated once,
+    outside the timed region)."""
+    w = synth.WORKLOADS[name]
+    x = synth.make_inputs(w)
+    copies, per_copy = input_copies(w)
+    Q = [to_dev(x["q"], torch, device) for _ in range(copies)]
+    K = [to_dev(x["k"], torch, device) for _ in range(copies)]
+    V = [to_dev(x["v"], torch, device) for _ in range(copies)]
+    if w.rope:
+        for c in range(copies):
+            eb.rope_apply(Q[c], base=synth.ROPE_BASE, pairing=synth.ROPE_PAIRING_HALF, out=Q[c])
+            eb.rope_apply(K[c], base=synth.ROPE_BASE, pairing=synth.ROPE_PAIRING_HALF, out=K[c])
+    kl = None if x["key_lens"] is None else torch.from_numpy(x["key_lens"]).to(device)
+    O = torch.empty_like(Q[0])
+    LSE = torch.empty((w.B, w.Hq, w.Nq), dtype=torch.float32, device=device)
+    ws = torch.empty(eb.attn_workspace_size(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d),
+                     dtype=torch.uint8, device=device)
+
+    def step(i):
+        c = i % copies
+        eb.attn_fwd_ws(Q[c], K[c], V[c], ws, causal=w.causal, scale=w.scale, key_lens=kl,
+                       out=O, lse=LSE, window=w.window, align=w.align)
+
+    for i in range(3):
+        step(i)
+    probe = time_steps(step, 3, torch, None, stream) / 3
+    n = steps or max(10, int(1000.0 / max(probe, 1e-3)))
+    ms = time_steps(step, n, torch, None, stream)
+    tf = w.flops() * n / (ms / 1e3) / 1e12
+    return {"metric": "attention fwd TFLOPS (formula FLOPs 4*B*Hq*Nq*Nk*d, halved for causal)",
+            "value": tf, "unit": "TFLOP/s", "workload": w.name, "steps": n,
+            "ms_per_step": ms / n, "flops_per_step": w.flops(),
+            "config": config_of(w, copies, per_copy, 1),
+            "roofline": roofline("tensor", tf, peaks, peak_src, w.name),
+            "gpu_launches": n}
+
+
 def run_window(torch, eb, device, stream, peaks, peak_src, steps=None):
     """The sliding-window prefill workload (inputs larger than L2, one copy)."""
     w = synth.WORKLOADS["long_window"]
@@ -635,9 +725,7 @@ def run_reference(args):
             "n_gpus": world, "steps": steps, "warmup": args.warmup,
             "ms_per_step": 1e3 * t_total / steps, "higher_is_better": True, "scaling": "weak",
             "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq,
-                       "Nk": w.Nk, "d": w.d, "causal": w.causal, "window": w.window,
-                       "align": w.align},
+            "config": config_of(w, *input_copies(w), world),
             "cpu_baseline": {"value": value, "unit": unit, "cores": threads, "kind": "oracle",
                              "sample": sample,
                              "rows_per_s": steps * rows_per_step / t_total,

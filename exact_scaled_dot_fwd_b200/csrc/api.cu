@@ -7,6 +7,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <vector>
 
 #include "attn.h"
 #include "common.cuh"
@@ -48,6 +49,10 @@ int current_sms() {
 
 // attn_fwd's workspace, one per device: the library's own (grown on demand)
 // unless the caller registered a buffer of its own with attn_set_workspace.
+// A buffer that is outgrown is retired, not freed: work already queued on
+// some stream (or launched by another host thread that read the old pointer)
+// may still use it, and freeing it would need a device-wide synchronisation.
+// Retired buffers are released at process exit with the current one.
 struct OwnedWorkspace {
   void* ptr = nullptr;
   size_t bytes = 0;
@@ -56,6 +61,7 @@ struct OwnedWorkspace {
 };
 constexpr int kMaxDevices = 64;
 OwnedWorkspace g_ws[kMaxDevices];
+std::vector<void*> g_retired;
 std::mutex g_ws_mu;
 
 struct WorkspaceReaper {
@@ -63,6 +69,7 @@ struct WorkspaceReaper {
     // process exit: the CUDA driver may already be tearing down; ignore errors
     for (auto& w : g_ws)
       if (w.ptr) cudaFree(w.ptr);
+    for (void* p : g_retired) cudaFree(p);
   }
 } g_reaper;
 
@@ -139,6 +146,7 @@ const char* attn_strerror(int status) {
     case ATTN_EWORKSPACE: return "ATTN_EWORKSPACE: workspace missing or too small";
     case ATTN_ECUDA: return "ATTN_ECUDA: CUDA call failed";
     case ATTN_ETIMEOUT: return "ATTN_ETIMEOUT: a kernel gave up waiting on a barrier";
+    case ATTN_ERANGE: return "ATTN_ERANGE: a kernel met an out-of-range block-table entry";
     default: return "unknown attn status";
   }
 }
@@ -299,15 +307,10 @@ int attn_fwd(const void* q, const void* k, const void* v, void* o, float* lse, i
       ws = w.user;
       ws_bytes = w.user_bytes;
     } else if (w.bytes < need) {
-      // the old buffer may still be in use by queued work on some stream
-      if (w.ptr && cudaDeviceSynchronize() != cudaSuccess) return ATTN_ECUDA;
-      if (w.ptr) cudaFree(w.ptr);
-      w.ptr = nullptr;
-      w.bytes = 0;
-      if (cudaMalloc(&w.ptr, need) != cudaSuccess) {
-        w.ptr = nullptr;
-        return ATTN_ECUDA;
-      }
+      void* p = nullptr;
+      if (cudaMalloc(&p, need) != cudaSuccess) return ATTN_ECUDA;
+      if (w.ptr) g_retired.push_back(w.ptr);
+      w.ptr = p;
       w.bytes = need;
     }
     if (!w.user) {

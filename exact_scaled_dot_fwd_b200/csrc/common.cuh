@@ -90,6 +90,20 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return mbar_wait_for(bar, parity, abort_flag, kWaitLimitNs);
 }
 
+// Cache row of block-table entry `entry` for kv head h of a paged cache
+// [num_pages, Hkv, page_size, d] viewed as rows of d elements.  An entry
+// outside [0, num_pages) is never turned into an address: the row past the
+// cache (`oob_row`, which a TMA load fills with zeros) is returned and the
+// device status word records ATTN_ERANGE.
+__device__ __forceinline__ int paged_cache_row(int entry, int num_pages, int Hkv, int h,
+                                               int page_size, int oob_row) {
+  if ((unsigned)entry >= (unsigned)num_pages) {
+    atomicExch(&g_device_status, (int)ATTN_ERANGE);
+    return oob_row;
+  }
+  return (entry * Hkv + h) * page_size;
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

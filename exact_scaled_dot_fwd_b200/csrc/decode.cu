@@ -97,7 +97,7 @@ struct DecodeArgs {
   float scale_log2;
   // paged cache (kPaged): Nk = max_pages * page_size
   const int32_t* block_table;
-  int max_pages, page_size, oob_row;   // oob_row: first row past the cache
+  int max_pages, page_size, num_pages, oob_row;   // oob_row: first row past the cache
 };
 
 template <int D, int MT, bool kPaged>
@@ -219,7 +219,7 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
         auto page_row = [&](int t) -> int {
           const int pg = (kl + t) / a.page_size + lane;
           return (lane < npg && pg * a.page_size < kl + s.hi)
-                     ? (table[pg] * Hkv + h) * a.page_size
+                     ? paged_cache_row(table[pg], a.num_pages, Hkv, h, a.page_size, a.oob_row)
                      : a.oob_row;
         };
         const int t0 = first_tile(s, kl);
@@ -642,6 +642,7 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
     a.block_table = pg ? pg->block_table : nullptr;
     a.max_pages = pg ? pg->max_pages : 0;
     a.page_size = pg ? pg->page_size : 0;
+    a.num_pages = pg ? pg->num_pages : 0;
     a.oob_row = (int)rows;
     const int MT = (p.R + 15) / 16;
     if (pg) {

@@ -30,7 +30,9 @@
 // as 128 / page_size TMA boxes of page_size rows, one per page, into the same
 // swizzled tile layout; pages past the segment's end are loaded from a row
 // past the cache (the TMA fills zeros), so unused table entries are never
-// read.  Keys of the tile outside the segment are masked.
+// read, and an entry outside [0, num_pages) is replaced by that row and
+// reported (ATTN_ERANGE in the device status word).  Keys of the tile
+// outside the segment are masked.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
@@ -222,7 +224,7 @@ struct DecodeTcArgs {
   float scale_log2;
   // paged cache (kernel instantiation with kPaged): Nk = max_pages * page_size
   const int32_t* block_table;
-  int max_pages, page_size, oob_row;   // oob_row: first row past the cache
+  int max_pages, page_size, num_pages, oob_row;   // oob_row: first row past the cache
 };
 
 template <int N, bool kPaged>
@@ -367,8 +369,9 @@ __global__ void __launch_bounds__(192, 1)
         // the cache, which the TMA fills with zeros)
         auto page_row = [&](int j) -> int {
           const int pg = (s.base + j * kTile) / a.page_size + lane;
-          return (lane < npg && pg * a.page_size < s.end) ? (table[pg] * Hkv + h) * a.page_size
-                                                          : a.oob_row;
+          return (lane < npg && pg * a.page_size < s.end)
+                     ? paged_cache_row(table[pg], a.num_pages, Hkv, h, a.page_size, a.oob_row)
+                     : a.oob_row;
         };
         int prow = kPaged ? page_row(0) : 0;
         const uint32_t so = kPaged ? (uint32_t)(lane * a.page_size * 128) : 0u;
@@ -669,6 +672,7 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   a.block_table = pg ? pg->block_table : nullptr;
   a.max_pages = pg ? pg->max_pages : 0;
   a.page_size = pg ? pg->page_size : 0;
+  a.num_pages = pg ? pg->num_pages : 0;
   a.oob_row = (int)rows;
   a.key_lens = key_lens;
   a.part_o = part_o;

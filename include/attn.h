@@ -58,7 +58,8 @@ typedef enum {
   ATTN_EALIGN = 3,        /* a pointer not 16-byte aligned */
   ATTN_EWORKSPACE = 4,    /* workspace missing or smaller than attn_workspace_size() */
   ATTN_ECUDA = 5,         /* a CUDA runtime / driver call failed (launch, attribute) */
-  ATTN_ETIMEOUT = 6       /* a kernel gave up waiting on a barrier (device status) */
+  ATTN_ETIMEOUT = 6,      /* a kernel gave up waiting on a barrier (device status) */
+  ATTN_ERANGE = 7         /* a kernel met an out-of-range block-table entry (device status) */
 } attn_status;
 
 /* Exact attention forward.  Dispatch: calls with at most 64 query rows per kv
@@ -73,10 +74,15 @@ typedef enum {
  *   lse may be NULL.  Both paths need scratch device memory (decode: its
  *   partial results; prefill: the work-item counter of its scheduler, zeroed
  *   in-stream before each launch): this entry point uses a workspace owned by
- *   the library (allocated on first use per device, grown on demand, released
- *   at process exit), or the caller's buffer registered for the current
- *   device with attn_set_workspace; calls that overlap on the GPU share it and
- *   must not run concurrently -- use attn_fwd_ws for concurrent streams.
+ *   the library, or the caller's buffer registered for the current device
+ *   with attn_set_workspace.  The library's own is allocated with cudaMalloc
+ *   on the first call per device and again whenever a call needs more; an
+ *   outgrown buffer is kept (not freed, so no device-wide synchronisation is
+ *   needed and work still queued on it is safe) until process exit.  The
+ *   host side is thread-safe, but every call on a device shares the one
+ *   buffer on the GPU: calls that overlap on the GPU (other streams, other
+ *   host threads) must not run concurrently -- use attn_fwd_ws, with a
+ *   workspace per stream, for that.
  * Errors: ATTN_EINVAL / EUNSUPPORTED / EALIGN before any launch; ATTN_ECUDA
  * if a launch or the workspace allocation fails; ATTN_EWORKSPACE if a
  * registered workspace is smaller than attn_workspace_size(...). */
@@ -135,10 +141,12 @@ ATTN_API int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, f
  *   multiple of 8 dividing 128 (d = 128) or 64 (d = 64) -- 8, 16, 32, 64
  *   (and 128 for d = 128).  Only entries j / page_size < ceil(key_lens[b] /
  *   page_size) of a sequence's table row are read; rows of its last page at
- *   or beyond key_lens[b] must hold finite values.  The kernels do not
- *   check table entries: one outside [0, num_pages) reads zeros, or, when
- *   (entry * Hkv + h) * page_size overflows 32 bits, some other page of the
- *   cache; no entry makes a kernel read outside k_cache / v_cache.
+ *   or beyond key_lens[b] must hold finite values.  The kernels check every
+ *   table entry they read: an entry outside [0, num_pages) is never used as
+ *   an address -- that page's keys and values read as zeros -- and the device
+ *   status word records ATTN_ERANGE (attn_device_status returns it after the
+ *   stream passes the call).  No entry makes a kernel read outside k_cache /
+ *   v_cache.
  *   Workspace: attn_workspace_size(B, Hq, Hkv, Nq, Nk, d) bytes.
  * Errors: ATTN_EINVAL (null table or key_lens, bad sizes), ATTN_EUNSUPPORTED
  * (page_size, more than 64 query rows per kv head or 2048 sequences, d), then
@@ -203,8 +211,14 @@ ATTN_API int rope_apply(const void* x_in, void* x_out, int B, int H, int N, int 
  *   shapes ((Hq/Hkv) * Nq <= 64)
  *   rotate q into the workspace and run the decode kernels.
  *   rope_base > 0, rope_pairing 0 (i, i + d/2) or 1 (2i, 2i + 1),
- *   q_pos_offset >= 0.  Workspace: attn_rope_workspace_size(...) bytes
- *   (256-byte aligned, contents need no initialisation).
+ *   q_pos_offset >= 0.  Positions: row i of EVERY sequence is rotated at
+ *   q_pos_offset + i, matching the ATTN_ALIGN_NK query positions this entry
+ *   point attends with (q_pos_offset = Nk - Nq puts the rows at the end of
+ *   the keys).  Ragged caches whose newest tokens sit at key_lens[b] - Nq + i
+ *   need per-sequence positions: rotate q with rope_apply per sequence and
+ *   call attn_fwd_ex with ATTN_ALIGN_KEYLEN instead.
+ *   Workspace: attn_rope_workspace_size(...) bytes (256-byte aligned,
+ *   contents need no initialisation).
  * Errors: as attn_fwd_ws. */
 ATTN_API int attn_fwd_rope(const void* q, const void* k, const void* v, void* o, float* lse,
                            int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
@@ -266,10 +280,11 @@ ATTN_API int attn_fwd_decode_static(const void* q, const void* k, const void* v,
 /* Size in bytes of the device array attn_fwd_decode_static works in. */
 ATTN_API size_t attn_decode_static_max_bytes(void);
 
-/* Synchronises `stream`, then returns ATTN_ETIMEOUT if any kernel of this
- * library on the current device gave up on a barrier wait since the last
- * reset, else ATTN_OK (ATTN_ECUDA if the synchronisation failed).  reset != 0
- * clears the device status word. */
+/* Synchronises `stream`, then returns the device status word of the current
+ * device: ATTN_ETIMEOUT if a kernel of this library gave up on a barrier
+ * wait, ATTN_ERANGE if a paged decode met an out-of-range block-table entry
+ * (the last such event since the last reset), else ATTN_OK (ATTN_ECUDA if
+ * the synchronisation failed).  reset != 0 clears the word. */
 ATTN_API int attn_device_status(void* stream, int reset);
 
 /* attn_device_status(stream, 1): the status since the last read, then

