@@ -131,6 +131,10 @@ def parse_args():
                         "the GQA attention kernel alone)")
     p.add_argument("--no-cpu", action="store_true")
     p.add_argument("--cpu-seconds", type=float, default=12.0)
+    p.add_argument("--profile-heads", type=int, default=0,
+                   help="cut the workload down to this many query heads (kv heads in "
+                        "proportion): the smaller case an ncu capture of a large workload "
+                        "runs on; its DRAM traffic scales with the heads")
     return p.parse_args()
 
 
@@ -156,6 +160,18 @@ def roofline(bound, achieved, peaks, peak_src, workload):
     else:
         r["ncu_dram_gbs"] = c.get("dram_gbs")
     return r
+
+
+def profile_case(w, heads):
+    """The workload with `heads` query heads and the kv heads in proportion
+    (heads = 0: unchanged)."""
+    if not heads:
+        return w
+    g = w.Hq // w.Hkv
+    if heads % g or heads > w.Hq:
+        raise SystemExit(f"--profile-heads {heads}: must be a multiple of {g} and <= {w.Hq}")
+    import dataclasses
+    return dataclasses.replace(w, Hq=heads, Hkv=heads // g)
 
 
 def config_of(w, copies, per_copy, world):
@@ -382,7 +398,7 @@ def run_ours(args):
     peaks, peak_src = load_peaks()
     stream = torch.cuda.current_stream()
 
-    w = synth.WORKLOADS[args.config]
+    w = profile_case(synth.WORKLOADS[args.config], args.profile_heads)
     # every rank processes its own batch: shift the seed by the rank
     wr = synth.Workload(**{**w.__dict__, "number": w.number + 100 * rank}) if rank else w
     x = synth.make_inputs(wr)

@@ -15,7 +15,7 @@ import os
 
 __all__ = ["attn_fwd", "attn_fwd_ws", "attn_workspace_size", "attn_set_workspace",
            "attn_fwd_paged", "attn_fwd_rope", "attn_fwd_decode_static", "rope_apply",
-           "prefill_tile_shape", "tile_plan", "device_status", "attn_last_device_status",
+           "prefill_tile_shape", "tile_plan", "prefill_trace", "device_status", "attn_last_device_status",
            "AttnError", "lib", "STATUS_NAMES"]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -73,6 +73,9 @@ def lib():
         L.attn_fwd_tile_plan_window.restype = i
         L.attn_fwd_tile_plan_ex.argtypes = [i, i, i, i, i, i, i, vp, vp, vp, vp]
         L.attn_fwd_tile_plan_ex.restype = i
+        L.attn_fwd_trace.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, i, i, f, vp, vp, sz,
+                                     vp, vp]
+        L.attn_fwd_trace.restype = i
         L.attn_device_status.argtypes = [vp, i]
         L.attn_device_status.restype = i
         L.attn_last_device_status.argtypes = [vp]
@@ -421,6 +424,30 @@ def tile_plan(B, Nq, Nk, d, causal, key_lens=None, device="cuda", stream=None, w
                                      _ptr(key_lens), _ptr(first), _ptr(count), _stream(stream))
     _raise(rc, "attn_fwd_tile_plan_ex")
     return first, count
+
+
+def prefill_trace(q, k, v, causal=False, scale=None, key_lens=None, window=0, align=0,
+                  stream=None):
+    """Run the prefill kernel with its trace hook: returns (o, lse, trace),
+    trace int32 [B, Hq, nqt, 3] = {first, last, count} of the KV tiles whose
+    scores the kernel computed for each query tile ({-1, -1, 0} for none)."""
+    B, Hq, Hkv, Nq, Nk, d = _qkv(q, k, v)
+    _check_io(q, key_lens, None, None, B, Hq, Nq, extra=[(k, "k"), (v, "v")])
+    if scale is None:
+        scale = 1.0 / math.sqrt(d)
+    torch = _torch()
+    br, _ = prefill_tile_shape(d)
+    nqt = -(-Nq // br)
+    trace = torch.tensor([-1, -1, 0], dtype=torch.int32, device=q.device).repeat(B * Hq * nqt)
+    out, lse = _outputs(q, None, None, True, B, Hq, Nq)
+    ws = _scratch(attn_workspace_size(B, Hq, Hkv, Nq, Nk, d), q.device, stream)
+    with torch.cuda.device(q.device):
+        rc = lib().attn_fwd_trace(_ptr(q), _ptr(k), _ptr(v), _ptr(out), _ptr(lse), B, Hq, Hkv,
+                                  Nq, Nk, d, int(bool(causal)), int(window), int(align),
+                                  float(scale), _ptr(key_lens), _ptr(ws), ws.numel(),
+                                  _ptr(trace), _stream(stream))
+    _raise(rc, "attn_fwd_trace")
+    return out, lse, trace.view(B, Hq, nqt, 3)
 
 
 def device_status(reset=True, stream=None) -> int:

@@ -191,6 +191,25 @@ int attn_fwd_ex(const void* q, const void* k, const void* v, void* o, float* lse
                         key_lens, nullptr, 0, workspace, sms, st);
 }
 
+int attn_fwd_trace(const void* q, const void* k, const void* v, void* o, float* lse, int B,
+                   int Hq, int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
+                   float scale, const int32_t* key_lens, void* workspace, size_t workspace_bytes,
+                   int32_t* trace, void* stream) {
+  if (!trace) return ATTN_EINVAL;
+  int rc = check_common(q, k, v, o, B, Hq, Hkv, Nq, Nk, d, causal, scale);
+  if (rc != ATTN_OK) return rc;
+  if (window < 0 || (align != 0 && align != 1)) return ATTN_EINVAL;
+  if (decode_supported(B, Hq, Hkv, Nq, d)) return ATTN_EUNSUPPORTED;   // prefill kernel only
+  if (lse && !aligned16(lse)) return ATTN_EALIGN;
+  if (!workspace || workspace_bytes < prefill_workspace_bytes()) return ATTN_EWORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return ATTN_EALIGN;
+  const int sms = current_sms();
+  if (sms <= 0) return ATTN_ECUDA;
+  return launch_prefill(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, window, align, scale,
+                        key_lens, nullptr, 0, workspace, sms, static_cast<cudaStream_t>(stream),
+                        trace);
+}
+
 size_t attn_rope_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   const size_t base = attn_workspace_size(B, Hq, Hkv, Nq, Nk, d);
   if (base == 0 || d <= 0) return 0;

@@ -29,6 +29,19 @@ __device__ __forceinline__ uint64_t globaltimer_ns() {
   return t;
 }
 
+// True in exactly one lane of the (fully active) warp: the lane that issues
+// an instruction meant to run once per warp, such as an MMA or a commit,
+// while the whole warp computes its operands.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\t"
+      "elect.sync _|P, 0xffffffff;\n\t"
+      "selp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 // ---------------------------------------------------------------- mbarrier
 
 __device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
@@ -90,6 +103,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity,
   return mbar_wait_for(bar, parity, abort_flag, kWaitLimitNs);
 }
 
+// mbar_wait by a whole warp with a warp-uniform result (false in every lane
+// if the wait gave up in any lane), so the warp stays converged.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity,
+                                               volatile int* abort_flag) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
 // Cache row of block-table entry `entry` for kv head h of a paged cache
 // [num_pages, Hkv, page_size, d] viewed as rows of d elements.  An entry
 // outside [0, num_pages) is never turned into an address: the row past the
@@ -102,6 +122,11 @@ __device__ __forceinline__ int paged_cache_row(int entry, int num_pages, int Hkv
     return oob_row;
   }
   return (entry * Hkv + h) * page_size;
+}
+
+// Barrier `id` (1..15) among `n` threads (a multiple of 32) of the CTA.
+__device__ __forceinline__ void named_bar_sync(int id, int n) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
 }
 
 // ---------------------------------------------------------------- TMA
@@ -170,6 +195,36 @@ __device__ __forceinline__ float exp2_approx(float x) {
   float y;
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
+}
+
+// 2^x for two values on the FMA and integer pipes (no SFU), so a softmax can
+// split its exponentials between the SFU and the FMA units.  Method: the
+// classic range reduction x = j + f with j = round(x), |f| <= 1/2 (Cody and
+// Waite's split), 2^f from a polynomial and 2^j added into the exponent field.
+//   - j comes from the rounding addition t = x + 1.5 * 2^23: in round-to-
+//     nearest the low mantissa bits of t hold j (two's complement), so
+//     (bits(t) << 23) is j in the exponent position and t - 1.5 * 2^23 is j
+//     exactly; f = x - j is exact.
+//   - 2^f ~ 1 + f (c1 + f (c2 + f c3)): a degree-3 fit with p(0) = 1 that
+//     minimises the maximum relative error over [-1/2, 1/2] (a linear
+//     programme over 4001 points, coefficients rounded to fp32); measured
+//     maximum relative error 1.01e-4 against exp2 over [-125, 10].
+//   - x is clamped to >= -125 so that j + exponent(p) stays a normal number:
+//     inputs below give about 2^-125 (~2e-38) instead of 0.  Callers use it
+//     only where no input is -inf (unmasked tiles).  x must be < 127.
+__device__ __forceinline__ float2 exp2_poly2(float2 x) {
+  constexpr float kC1 = 0x1.62f5fap-1f, kC2 = 0x1.f00c4cp-3f, kC3 = 0x1.c2a21ap-5f;
+  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
+  x.x = fmaxf(x.x, -125.f);
+  x.y = fmaxf(x.y, -125.f);
+  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
+  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
+  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
+  float2 p = __ffma2_rn(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
+  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
+  p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
+  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
+                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
 }
 
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half.

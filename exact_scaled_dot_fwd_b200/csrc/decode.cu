@@ -134,6 +134,9 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
+  // a programmatic dependent of the previous kernel in the stream (as the
+  // tcgen05 split kernel): global memory only after the previous grid
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // key lengths (clamped) and their exclusive prefix over b, by warp 0
   if (warp == 0) {
     long long carry = 0;
@@ -465,6 +468,9 @@ constexpr int kCombineThreads = 256;
 
 template <int D>
 __global__ void __launch_bounds__(kCombineThreads) decode_combine_kernel(CombineArgs a) {
+  // the next decode call's split kernel may start its set-up now (it waits
+  // for this grid before it touches global memory)
+  asm volatile("griddepcontrol.launch_dependents;");
   extern __shared__ float cs[];          // int flags [ns]: slots written by this launch
   __shared__ long long s_red[2][kCombineThreads / 32];
   __shared__ long long s_pb[2];
@@ -582,8 +588,7 @@ int launch_decode_t(const DecodePlan& p, const CUtensorMap& tk, const CUtensorMa
   const int smem = DecodeSmem<D>::kTotal;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ECUDA;
-  kern<<<p.grid, (MT * 4 + 1) * 32, smem, st>>>(tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+  return launch_programmatic(kern, dim3(p.grid), dim3((MT * 4 + 1) * 32), smem, st, tk, tv, a);
 }
 }  // namespace
 

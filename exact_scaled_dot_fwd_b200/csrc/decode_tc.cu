@@ -21,7 +21,13 @@
 // of tile j+2 and the loads run while the softmax works on tile j.
 //
 // Warp roles: warps 0-3 softmax (TMEM lane quarters 0-3), warp 4 MMA issuer
-// and TMEM allocator, warp 5 TMA producer.
+// (the whole warp runs its loop; one elected lane issues the tcgen05
+// instructions) and TMEM allocator, warp 5 TMA producer.
+//
+// Ring depths are chosen per launch: 3 K and 3 V tiles when they fit beside
+// the per-sequence arrays of the batch (most batches), else 2 + 3, else 2 + 2
+// (measured on the MQA decode workload: 2 + 3 with a single-lane MMA loop
+// 4736 GB/s, 3 + 3 4774, 3 + 3 with the warp-wide MMA loop 4834).
 //
 // Paged KV cache ("Attention mechanisms ...", section 20; "Transformer
 // internals", PagedAttention): key j of a sequence lives in physical block
@@ -48,15 +54,14 @@ constexpr int kD = 128;
 constexpr int kMaxB = 2048;
 constexpr float kRescaleLog2 = 8.0f;
 
-template <int N>
+template <int N, int KS_, int VS_>
 struct Smem {
   // Ring depths.  A K slot frees as soon as its S MMA has run, a V slot only
-  // after the softmax of its tile and the PV MMA, so V needs the deeper ring
-  // to keep enough loads in flight (two V slots held the producer waiting on
-  // V for half of the kernel at 32 heads).  At N = 64 the larger Q and P
-  // buffers leave room for two of each.
-  static constexpr int KS = 2;                 // K ring stages
-  static constexpr int VS = N <= 32 ? 3 : 2;   // V ring stages
+  // after the softmax of its tile and the PV MMA, so V needs at least as deep
+  // a ring as K to keep enough loads in flight.  The launch picks the
+  // deepest pair that fits beside the per-sequence arrays of its batch.
+  static constexpr int KS = KS_;                  // K ring stages
+  static constexpr int VS = VS_;                  // V ring stages
   static constexpr int kKV = kTile * kD * 2;   // one K or V tile (32 KB)
   static constexpr int kBox = kTile * 128;     // 64-column box of a K/V tile
   static constexpr int kQBox = N * 128;        // 64-column box of Q (N rows)
@@ -65,10 +70,7 @@ struct Smem {
   static constexpr int kV = kK + KS * kKV;
   static constexpr int kQ = kV + VS * kKV;
   static constexpr int kP = kQ + 2 * kQBox;    // P^T [2 buffers][2 boxes]
-  static constexpr int kScan = kP + 4 * kPBox; // int [kMaxB + 1] key prefix over b
-  static constexpr int kLens = kScan + (kMaxB + 1) * 4 + 4;   // int [kMaxB] keys per unit
-  static constexpr int kLo = kLens + kMaxB * 4;            // int [kMaxB] first key
-  static constexpr int kRed = kLo + kMaxB * 4;     // float [4][64]
+  static constexpr int kRed = kP + 4 * kPBox;      // float [4][64]
   static constexpr int kMs = kRed + 4 * 64 * 4;    // float [64] running max (log2 units)
   static constexpr int kAs = kMs + 64 * 4;         // float [64] this tile's rescale factor
   static constexpr int kLs = kAs + 64 * 4;         // float [64] segment row sums
@@ -88,8 +90,12 @@ struct Smem {
   };
   static constexpr int kTmemSlot = kBar + NUM_BARS * 8;
   static constexpr int kAbort = kTmemSlot + 16;
-  static constexpr int kTotal = kAbort + 16 + 1024;
-  static_assert(kTotal <= 232448, "shared memory over the 227 KB per-CTA limit");
+  // per-sequence arrays, sized by the launch's B: int [B + 1] key prefix over
+  // b, int [B] keys per unit, int [B] first key
+  static constexpr int kScan = kAbort + 16;
+  static constexpr int scan_bytes(int B) { return (3 * B + 2) * 4; }
+  static constexpr int total(int B) { return kScan + scan_bytes(B) + 1024; }   // + alignment slack
+  static constexpr bool fits(int B) { return total(B) <= 232448; }
 };
 
 struct Seg {
@@ -227,13 +233,13 @@ struct DecodeTcArgs {
   int max_pages, page_size, num_pages, oob_row;   // oob_row: first row past the cache
 };
 
-template <int N, bool kPaged>
+template <int N, bool kPaged, int KS_, int VS_>
 __global__ void __launch_bounds__(192, 1)
     decode_tc_kernel(const __grid_constant__ CUtensorMap tmap_q,
                      const __grid_constant__ CUtensorMap tmap_k,
                      const __grid_constant__ CUtensorMap tmap_v, DecodeTcArgs a) {
   using namespace dtc;
-  using L = Smem<N>;
+  using L = Smem<N, KS_, VS_>;
   constexpr int KS = L::KS, VS = L::VS;
   constexpr uint32_t kIdescS = tc::idesc_bf16(kTile, N, false, false);
   constexpr uint32_t kIdescPV = tc::idesc_bf16(kD, N, true, false);
@@ -241,9 +247,9 @@ __global__ void __launch_bounds__(192, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
-  int* pb = reinterpret_cast<int*>(smem + L::kScan);
-  int* lens_s = reinterpret_cast<int*>(smem + L::kLens);
-  int* lo_s = reinterpret_cast<int*>(smem + L::kLo);
+  int* pb = reinterpret_cast<int*>(smem + L::kScan);   // [B + 1]
+  int* lens_s = pb + a.B + 2;                          // [B]
+  int* lo_s = lens_s + a.B;                            // [B]
   float* red = reinterpret_cast<float*>(smem + L::kRed);
   float* m_s = reinterpret_cast<float*>(smem + L::kMs);
   float* a_s = reinterpret_cast<float*>(smem + L::kAs);
@@ -266,6 +272,12 @@ __global__ void __launch_bounds__(192, 1)
     tc::alloc(tmem_slot, 256);
     tc::relinquish();
   }
+  // Launched as a programmatic dependent of the previous kernel in the
+  // stream: the set-up above may overlap its tail (the previous decode
+  // call's combine pass releases its dependents early); nothing is read
+  // from or written to global memory before the previous grid has
+  // completed and its writes are visible.
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   // key lengths (clamped) and their exclusive prefix over b, by warp 5
   if (warp == 5) {
     int carry = 0;
@@ -414,7 +426,9 @@ __global__ void __launch_bounds__(192, 1)
     }
   } else if (warp == 4) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0 && start < end) {
+    // the whole warp runs the loop (warp-uniform waits and descriptors); one
+    // elected lane issues each group of tcgen05 instructions
+    if (start < end) {
       const uint32_t k_base = smem_u32(smem + L::kK), v_base = smem_u32(smem + L::kV);
       const uint32_t q_base = smem_u32(smem + L::kQ), p_base = smem_u32(smem + L::kP);
       // descriptors built once per call; a k-step only moves the start
@@ -423,57 +437,67 @@ __global__ void __launch_bounds__(192, 1)
         const uint64_t dk = tc::smem_desc_sw128(k_base + (g % KS) * L::kKV, 16, 1024);
         const uint64_t dq = tc::smem_desc_sw128(q_base, 16, 1024);
         const uint32_t dt = tmem + (uint32_t)((g & 1) * N);
-        tc::mma_ss(dt, dk, dq, kIdescS, 0u);
+        if (elect_one()) {
+          tc::mma_ss(dt, dk, dq, kIdescS, 0u);
 #pragma unroll
-        for (int kk = 1; kk < kD / 16; ++kk)
-          tc::mma_ss(dt, dk + (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4),
-                     dq + (uint64_t)(((kk >> 2) * L::kQBox + (kk & 3) * 32) >> 4), kIdescS, 1u);
+          for (int kk = 1; kk < kD / 16; ++kk)
+            tc::mma_ss(dt, dk + (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4),
+                       dq + (uint64_t)(((kk >> 2) * L::kQBox + (kk & 3) * 32) >> 4), kIdescS, 1u);
+        }
+        __syncwarp();
       };
       auto issue_pv = [&](int g, bool acc) {
         const uint64_t dv = tc::smem_desc_sw128(v_base + (g % VS) * L::kKV, L::kBox, 1024);
         const uint64_t dp = tc::smem_desc_sw128(p_base + (g & 1) * 2 * L::kPBox, 16, 1024);
-        tc::mma_ss(tmem + 2u * N, dv, dp, kIdescPV, acc ? 1u : 0u);
+        if (elect_one()) {
+          tc::mma_ss(tmem + 2u * N, dv, dp, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < kTile / 16; ++kk)
-          tc::mma_ss(tmem + 2u * N, dv + (uint64_t)((kk * 16 * 128) >> 4),
-                     dp + (uint64_t)(((kk >> 2) * L::kPBox + (kk & 3) * 32) >> 4), kIdescPV, 1u);
+          for (int kk = 1; kk < kTile / 16; ++kk)
+            tc::mma_ss(tmem + 2u * N, dv + (uint64_t)((kk * 16 * 128) >> 4),
+                       dp + (uint64_t)(((kk >> 2) * L::kPBox + (kk & 3) * 32) >> 4), kIdescPV, 1u);
+        }
+        __syncwarp();
+      };
+      auto commit = [&](int bar) {
+        if (elect_one()) tc::commit(&bars[bar]);
+        __syncwarp();
       };
       int u = u0, g = 0, qf = 0;
       Seg s;
       bool ok = true;
       while (ok && next_seg(u, s)) {
         const int n = s.n;
-        if (!mbar_wait(&bars[L::Q_FULL], qf & 1, abort_flag)) break;
+        if (!mbar_wait_warp(&bars[L::Q_FULL], qf & 1, abort_flag)) break;
         ++qf;
         for (int t = 0; t < 2 && t < n && ok; ++t) {
           const int gt = g + t;
-          if (!mbar_wait(&bars[L::K_FULL + gt % KS], (gt / KS) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bars[L::K_FULL + gt % KS], (gt / KS) & 1, abort_flag)) { ok = false; break; }
           tc::fence_after();
           issue_s(gt);
-          tc::commit(&bars[L::S_FULL + (gt & 1)]);
-          tc::commit(&bars[L::K_EMPTY + gt % KS]);
+          commit(L::S_FULL + (gt & 1));
+          commit(L::K_EMPTY + gt % KS);
         }
-        if (ok && n <= 2) tc::commit(&bars[L::Q_EMPTY]);
+        if (ok && n <= 2) commit(L::Q_EMPTY);
         for (int j = 0; ok && j < n; ++j, ++g) {
-          if (!mbar_wait(&bars[L::P_FULL + (g & 1)], (g >> 1) & 1, abort_flag)) { ok = false; break; }
-          if (!mbar_wait(&bars[L::V_FULL + g % VS], (g / VS) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bars[L::P_FULL + (g & 1)], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bars[L::V_FULL + g % VS], (g / VS) & 1, abort_flag)) { ok = false; break; }
           tc::fence_after();
           issue_pv(g, j > 0);
-          tc::commit(&bars[L::PV_DONE + (g & 1)]);
-          tc::commit(&bars[L::V_EMPTY + g % VS]);
+          commit(L::PV_DONE + (g & 1));
+          commit(L::V_EMPTY + g % VS);
           if (j + 2 < n) {
             const int g2 = g + 2;
-            if (!mbar_wait(&bars[L::K_FULL + g2 % KS], (g2 / KS) & 1, abort_flag)) { ok = false; break; }
+            if (!mbar_wait_warp(&bars[L::K_FULL + g2 % KS], (g2 / KS) & 1, abort_flag)) { ok = false; break; }
             tc::fence_after();
             issue_s(g2);
-            tc::commit(&bars[L::S_FULL + (g2 & 1)]);
-            tc::commit(&bars[L::K_EMPTY + g2 % KS]);
-            if (j + 2 == n - 1) tc::commit(&bars[L::Q_EMPTY]);
+            commit(L::S_FULL + (g2 & 1));
+            commit(L::K_EMPTY + g2 % KS);
+            if (j + 2 == n - 1) commit(L::Q_EMPTY);
           }
         }
       }
-      tc::commit(&bars[L::MMA_DONE]);
-      mbar_wait(&bars[L::MMA_DONE], 0, nullptr);
+      commit(L::MMA_DONE);
+      mbar_wait_warp(&bars[L::MMA_DONE], 0, nullptr);
     }
   } else {
     // ------------------------------------------------------------ softmax
@@ -636,15 +660,24 @@ __global__ void __launch_bounds__(192, 1)
 }
 
 namespace {
-template <int N, bool kPaged>
+template <int N, bool kPaged, int KS, int VS>
 int launch_tc_t(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                 const DecodeTcArgs& a, cudaStream_t st) {
-  auto kern = decode_tc_kernel<N, kPaged>;
-  const int smem = dtc::Smem<N>::kTotal;
+  auto kern = decode_tc_kernel<N, kPaged, KS, VS>;
+  const int smem = dtc::Smem<N, KS, VS>::total(a.B);
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ECUDA;
-  kern<<<grid, 192, smem, st>>>(tq, tk, tv, a);
-  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+  return launch_programmatic(kern, dim3(grid), dim3(192), smem, st, tq, tk, tv, a);
+}
+
+// The deepest rings that fit with the batch's per-sequence arrays:
+// 3 K + 3 V tiles, else 2 + 3, else 2 + 2.
+template <int N, bool kPaged>
+int launch_tc_rings(int grid, const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                    const DecodeTcArgs& a, cudaStream_t st) {
+  if (dtc::Smem<N, 3, 3>::fits(a.B)) return launch_tc_t<N, kPaged, 3, 3>(grid, tq, tk, tv, a, st);
+  if (dtc::Smem<N, 2, 3>::fits(a.B)) return launch_tc_t<N, kPaged, 2, 3>(grid, tq, tk, tv, a, st);
+  return launch_tc_t<N, kPaged, 2, 2>(grid, tq, tk, tv, a, st);
 }
 }  // namespace
 
@@ -683,13 +716,13 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   a.seg_cost = mk.seg_cost;
   a.scale_log2 = scale * kLog2e;
   if (pg) {
-    if (N == 16) return launch_tc_t<16, true>(grid, tq, tk, tv, a, st);
-    if (N == 32) return launch_tc_t<32, true>(grid, tq, tk, tv, a, st);
-    return launch_tc_t<64, true>(grid, tq, tk, tv, a, st);
+    if (N == 16) return launch_tc_rings<16, true>(grid, tq, tk, tv, a, st);
+    if (N == 32) return launch_tc_rings<32, true>(grid, tq, tk, tv, a, st);
+    return launch_tc_rings<64, true>(grid, tq, tk, tv, a, st);
   }
-  if (N == 16) return launch_tc_t<16, false>(grid, tq, tk, tv, a, st);
-  if (N == 32) return launch_tc_t<32, false>(grid, tq, tk, tv, a, st);
-  return launch_tc_t<64, false>(grid, tq, tk, tv, a, st);
+  if (N == 16) return launch_tc_rings<16, false>(grid, tq, tk, tv, a, st);
+  if (N == 32) return launch_tc_rings<32, false>(grid, tq, tk, tv, a, st);
+  return launch_tc_rings<64, false>(grid, tq, tk, tv, a, st);
 }
 
 }  // namespace attn

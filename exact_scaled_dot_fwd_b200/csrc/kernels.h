@@ -22,6 +22,27 @@ int make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_
 int make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                       uint64_t mats, uint32_t box_cols, uint32_t box_rows);
 
+// Launch `kern` as a programmatic dependent of the previous kernel in the
+// stream (cudaLaunchAttributeProgrammaticStreamSerialization): it may start
+// once that kernel has called griddepcontrol.launch_dependents (or ended) and
+// must execute griddepcontrol.wait before it touches global memory.
+template <typename... P, typename... A>
+int launch_programmatic(void (*kern)(P...), dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                        A&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, static_cast<A&&>(args)...) != cudaSuccess) return ATTN_ECUDA;
+  return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
+}
+
 // ---- decode (R = (Hq / Hkv) * Nq <= 64 query rows per kv head)
 struct DecodePlan {
   int grid = 0;          // CTAs of the split kernel (one wave)
@@ -65,10 +86,14 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
 bool prefill_supported(int d);
 size_t prefill_workspace_bytes();   // scheduler counter
 void prefill_tile_shape(int d, int* Br, int* Bc);
+// trace (test hook, may be null): int32 [B * Hq * ceil(Nq / 128)][3], per query
+// tile {first, last, count} of the KV tiles whose scores the kernel computes;
+// tiles it computes none for are left as they are.
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
                    float scale, const int32_t* key_lens, const float2* rope_tab,
-                   int rope_pairing, void* workspace, int num_sms, cudaStream_t st);
+                   int rope_pairing, void* workspace, int num_sms, cudaStream_t st,
+                   int32_t* trace = nullptr);
 int launch_tile_plan(int B, int Nq, int Nk, int d, int causal, int window, int align,
                      const int32_t* key_lens, int32_t* first, int32_t* count, cudaStream_t st);
 

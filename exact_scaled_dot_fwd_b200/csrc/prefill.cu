@@ -37,19 +37,25 @@
 // than 8 (log2 units); otherwise the stale max is kept (P <= 2^8, exact in
 // the final O / l because O and l share the same reference).
 //
-// Fused RoPE of Q (kRope instantiation): after a Q tile lands, the softmax
-// warpgroup of its slot -- idle until the tile's first scores exist --
-// rotates it in shared memory, one row per thread (row i at position
-// q_pos_offset + i, cos/sin from a table built for the call, the arithmetic
-// of rope_math.cuh), and releases it to the MMA issuer on Q_READY.  K is
-// expected rotated (a KV cache stores keys rotated once); rotating K here
-// would redo the work for every query tile that reads the K tile.
+// Fused RoPE of Q (kRope instantiation, one more warp): after a Q tile
+// lands, warps 10-11 rotate it in shared memory, two rows per thread (row i
+// at position q_pos_offset + i, cos/sin from a table built for the call, the
+// arithmetic of rope_math.cuh), and release it to the MMA issuer on Q_READY;
+// the softmax warps never wait for it.  K is expected rotated (a KV cache
+// stores keys rotated once); rotating K here would redo the work for every
+// query tile that reads the K tile.
 //
 // Sliding window ("Attention mechanisms ...", section 11): a query tile
 // visits the contiguous KV-tile range that covers its rows' windows.  When
-// the two tiles of an item start at different KV tiles, both walk the union
-// of their ranges (one or two extra tiles per item, fully masked for the
-// tile they do not belong to), so the slots stay on one KV stream.
+// the two tiles of an item start at different KV tiles, the item's K/V
+// stream covers the union of their ranges and each slot joins it at its own
+// first tile and leaves after its own last: no scores are computed for a
+// tile outside a query tile's range.
+
+//
+// Trace (FwdArgs::trace, a test hook): the MMA issuer records for every
+// query tile the first and last KV tile whose scores it computed and how
+// many, as it issues them.
 #include <cuda_bf16.h>
 
 #include <cmath>
@@ -69,10 +75,14 @@ constexpr int kN = 128;        // keys per KV tile
 // K/V ring stages: d = 128 fits three K and two V tiles beside the two Q
 // tiles (224 KB); d = 64 fits three of each.
 template <int D> struct Stages { static constexpr int K = 3, V = D == 128 ? 2 : 3; };
-constexpr int kThreads = 352;   // 11 warps
+// 11 warps; the fused-RoPE instantiation adds a 12th, so that warps 10-11
+// rotate the Q tiles (below)
+constexpr int threads(bool rope) { return rope ? 384 : 352; }
 constexpr int kItemSlots = 4;   // depth of the shared-memory ring of work items
-// arrivals that free an item slot: MMA thread, Q producer, 256 softmax threads
-constexpr int kItemReaders = 2 + 256;
+// arrivals that free an item slot: MMA warp, the Q warp (fused RoPE: both Q
+// warps, every thread), 256 softmax threads (every softmax thread arrives:
+// measured faster than one elected arrival per warp after a warp barrier)
+constexpr int item_readers(bool rope) { return rope ? 1 + 64 + 256 : 2 + 256; }
 constexpr float kRescaleLog2 = 8.0f;
 
 template <int D>
@@ -109,6 +119,7 @@ struct Smem {
 
 struct Tile {
   int row_tile, head, count;
+  int first;              // step of the item's KV stream at which this tile joins it
   int um_begin, um_end;   // KV tiles (absolute index) that need no element mask
 };
 
@@ -137,15 +148,16 @@ struct FwdArgs {
   int band;         // ranks per band (item order: band, unit, rank in band)
   int total;        // number of items
   float scale_log2;
+  int32_t* trace;   // test hook: per query tile {first, last, count} of the KV tiles scored, or null
 };
 
 namespace pf {
 
 struct Item {
   Tile tl[2];       // tl[0] has the fewer KV tiles
-  int b, n, L;
+  int b, n, L;      // n: steps of the item's KV stream
   int off;          // key position of query row i is i + off
-  int kv_begin;     // KV tile of step 0 (both slots)
+  int kv_begin;     // KV tile of stream step 0
   int kv_row0;      // cache row of KV tile kv_begin
 };
 
@@ -199,22 +211,24 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window)
     it.tl[t].um_begin = r.um_begin;
     it.tl[t].um_end = r.um_end;
   }
-  it.kv_begin = 0;
-  if (it.tl[0].count > 0 && it.tl[1].count > 0 && begin[0] != begin[1]) {
-    // different first tiles (sliding window): both walk the union
-    const int b0 = begin[0] < begin[1] ? begin[0] : begin[1];
-    const int e0 = begin[0] + it.tl[0].count, e1 = begin[1] + it.tl[1].count;
-    it.kv_begin = b0;
-    it.tl[0].count = it.tl[1].count = (e0 > e1 ? e0 : e1) - b0;
-  } else {
+  // the stream starts at the earlier first tile (only a window makes the two
+  // differ); each tile joins it at its own offset
+  if (it.tl[0].count > 0 && it.tl[1].count > 0)
+    it.kv_begin = begin[0] < begin[1] ? begin[0] : begin[1];
+  else
     it.kv_begin = it.tl[0].count > 0 ? begin[0] : begin[1];
+  it.n = 0;
+#pragma unroll
+  for (int t = 0; t < 2; ++t) {
+    it.tl[t].first = it.tl[t].count > 0 ? begin[t] - it.kv_begin : 0;
+    const int e = it.tl[t].first + it.tl[t].count;
+    if (e > it.n) it.n = e;
   }
   if (it.tl[0].count > it.tl[1].count) {
     const Tile x = it.tl[0];
     it.tl[0] = it.tl[1];
     it.tl[1] = x;
   }
-  it.n = it.tl[1].count;
   const int hk = it.tl[1].head / (a.Hq / a.Hkv);
   it.kv_row0 = (it.b * a.Hkv + hk) * a.Nk + it.kv_begin * kN;
   return it;
@@ -303,12 +317,19 @@ __device__ __forceinline__ void rope_q_row(uint8_t* qs, int r, int pos_row, cons
 }
 
 template <int D, bool kWindow, bool kRope>
-__global__ void __launch_bounds__(pf::kThreads, 1)
+__global__ void __launch_bounds__(pf::threads(kRope), 1)
     prefill_tc_kernel(const __grid_constant__ CUtensorMap tq, const __grid_constant__ CUtensorMap tk,
                       const __grid_constant__ CUtensorMap tv, FwdArgs a) {
   using namespace pf;
   using L = Smem<D>;
   constexpr int kBoxes = D / 64;
+  // Exponentials of unmasked tiles: at d = 64 the MMAs take half the time
+  // per score that they take at d = 128 while the exponentials stay, so 3 of
+  // every 8 score pairs take 2^x from a polynomial on the FMA pipe
+  // (exp2_poly2) and the SFU does the rest (measured +4% on the padded
+  // cross-attention workload; at d = 128 the split measured slower and the
+  // SFU does all of them)
+  constexpr int kPolyPairs = D == 64 ? 3 : 0;
   const int window = kWindow ? a.window : 0;
   constexpr int kKS = L::kKS, kVS = L::kVS;
   // TMEM columns: S of tile t at 128 t, O of tile t at 256 + D t
@@ -325,7 +346,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* items = reinterpret_cast<volatile int*>(smem + L::kItems);
   // next item index from the ring (every reader calls it once per item);
-  // -1 ends the stream
+  // -1 ends the stream.  One thread, one arrival.
   auto next_item = [&](int& k) -> int {
     const int slot = k % kItemSlots;
     if (!mbar_wait(&bars[L::ITEM_FULL + slot], (k / kItemSlots) & 1, abort_flag)) return -1;
@@ -335,12 +356,13 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     return idx;
   };
 
+
   if (threadIdx.x == 0) {
     for (int i = 0; i < L::NUM_BARS; ++i) {
       uint32_t cnt = 1;
       if (i == L::P_FULL || i == L::P_FULL + 1) cnt = 128;
-      if (i >= L::ITEM_EMPTY && i < L::ITEM_EMPTY + kItemSlots) cnt = kItemReaders;
-      if (i == L::Q_READY || i == L::Q_READY + 1) cnt = 128;   // a slot's softmax warpgroup
+      if (i >= L::ITEM_EMPTY && i < L::ITEM_EMPTY + kItemSlots) cnt = item_readers(kRope);
+      if (i == L::Q_READY || i == L::Q_READY + 1) cnt = 64;    // the two Q warps
       mbar_init(&bars[i], cnt);
     }
     *abort_flag = 0;
@@ -404,6 +426,45 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       for (int j = g - kVS > 0 ? g - kVS : 0; j < g; ++j)
         mbar_wait(&bars[L::V_FULL + j % kVS], (j / kVS) & 1, nullptr);
     }
+  } else if (kRope && warp >= 10) {
+    // ------------------------------------------------- Q producer + RoPE of Q
+    // Lane 0 of warp 10 loads each Q tile; once it lands, the 64 threads of
+    // warps 10-11 rotate it in place (rows q and q + 64 each, row i at
+    // position q_pos_offset + i, cos/sin from the call's table, the
+    // arithmetic of rope_math.cuh) and release it to the MMA issuer on
+    // Q_READY.  The rotation runs while the softmax warps finish the
+    // previous item, off their critical path.
+    const int q = (warp - 10) * 32 + lane;
+    if (warp == 10 && lane == 0) tma_prefetch_desc(&tq);
+    int qn[2] = {0, 0}, k = 0;
+    bool ok = true;
+    for (int idx; ok && (idx = next_item(k)) >= 0;) {
+      const Item it = make_item(a, idx, window);
+      if (it.n == 0) continue;
+      for (int t = 0; t < 2 && ok; ++t) {
+        if (it.tl[t].count == 0) continue;
+        if (q == 0) {
+          if (qn[t] > 0 && !mbar_wait(&bars[L::Q_EMPTY + t], (qn[t] - 1) & 1, abort_flag)) {
+            ok = false;
+          } else {
+            mbar_arrive_expect_tx(&bars[L::Q_FULL + t], L::kTile);
+            for (int bx = 0; bx < kBoxes; ++bx)
+              tma_load_3d(smem + L::kQ + t * L::kTile + bx * L::kBox, &tq, bx * 64,
+                          it.tl[t].row_tile * kM, it.b * a.Hq + it.tl[t].head,
+                          &bars[L::Q_FULL + t]);
+          }
+        }
+        if (!mbar_wait(&bars[L::Q_FULL + t], qn[t] & 1, abort_flag)) { ok = false; break; }
+        ++qn[t];
+#pragma unroll
+        for (int h = 0; h < 2; ++h) {
+          const int r = q + 64 * h, row = it.tl[t].row_tile * kM + r;
+          if (row < a.Nq) rope_q_row<D>(smem + L::kQ + t * L::kTile, r, row, a);
+        }
+        fence_proxy_async_smem();   // the tensor core reads what this thread wrote
+        mbar_arrive(&bars[L::Q_READY + t]);
+      }
+    }
   } else if (warp == 10) {
     // ------------------------------------------------------------ Q producer
     if (lane == 0) {
@@ -431,102 +492,156 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     }
   } else if (warp == 8) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
+    // The whole warp runs the issue loop -- waits, item bookkeeping and the
+    // MMA descriptors are warp-uniform -- and one elected lane issues each
+    // group of tcgen05 instructions.  (A loop run by a single lane made
+    // every MMA issue cost about 100 cycles, which capped the tensor core
+    // below the rate its 64-cycle 128x128x16 MMAs allow.)
+    {
       const uint32_t q_base = smem_u32(smem + L::kQ);
       const uint32_t k_base = smem_u32(smem + L::kK);
       const uint32_t v_base = smem_u32(smem + L::kV);
       // Descriptors are built once per call; a k-step only moves the start
       // address field (bits 0-13 hold address >> 4, and shared memory stays
-      // below 256 KB, so the add never carries out of it).  The issuing
-      // thread is on the critical path: about 600 cycles per call were
-      // measured with per-step descriptor construction.
+      // below 256 KB, so the add never carries out of it).
       auto issue_s = [&](int t, int ks) {
         const uint64_t da = tc::smem_desc_sw128(q_base + t * L::kTile, 16, 1024);
         const uint64_t db = tc::smem_desc_sw128(k_base + ks * L::kTile, 16, 1024);
         const uint32_t dt = tmem + 128u * t;
-        tc::mma_ss(dt, da, db, kIdescS, 0u);
+        if (elect_one()) {
+          tc::mma_ss(dt, da, db, kIdescS, 0u);
 #pragma unroll
-        for (int kk = 1; kk < D / 16; ++kk) {
-          const uint64_t off = (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4);
-          tc::mma_ss(dt, da + off, db + off, kIdescS, 1u);
+          for (int kk = 1; kk < D / 16; ++kk) {
+            const uint64_t off = (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4);
+            tc::mma_ss(dt, da + off, db + off, kIdescS, 1u);
+          }
         }
+        __syncwarp();
       };
       auto issue_pv = [&](int t, int vs, bool acc) {
         const uint64_t dv = tc::smem_desc_sw128(v_base + vs * L::kTile, L::kBox, 1024);
         const uint32_t dt = tmem + 256u + D * t, pa = tmem + 128u * t;
-        tc::mma_ts(dt, pa, dv, kIdescPV, acc ? 1u : 0u);
+        if (elect_one()) {
+          tc::mma_ts(dt, pa, dv, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-        for (int kk = 1; kk < kN / 16; ++kk)
-          tc::mma_ts(dt, pa + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, 1u);
+          for (int kk = 1; kk < kN / 16; ++kk)
+            tc::mma_ts(dt, pa + kk * 8, dv + (uint64_t)((kk * 16 * 128) >> 4), kIdescPV, 1u);
+        }
+        __syncwarp();
+      };
+      auto commit = [&](int bar) {
+        if (elect_one()) tc::commit(&bars[bar]);
+        __syncwarp();
+      };
+      // next item index, read by lane 0 and handed to the warp (one arrival)
+      auto next_item_w = [&](int& k) -> int {
+        int idx = -1;
+        if (lane == 0) idx = next_item(k);
+        idx = __shfl_sync(0xffffffffu, idx, 0);
+        k = __shfl_sync(0xffffffffu, k, 0);
+        return idx;
       };
       // Each slot's work is one stream of KV tiles across items: in the step
-      // that finishes item i for one slot, the S MMA of item i+1's first
-      // tile is issued for every slot that is done with item i, so a slot
-      // with fewer tiles moves on while the other one finishes.
+      // that finishes item i, the S MMA of item i+1's first tile is issued
+      // for every slot that starts item i+1 on its first stream step, so a
+      // slot with fewer tiles moves on while the other one finishes.  Slot t
+      // takes part in stream steps [f[t], f[t] + c[t]) of an item.
       int qf[2] = {0, 0}, pw[2] = {0, 0}, g = 0, k = 0;
+      int tr_first[2] = {0, 0}, tr_cnt[2] = {0, 0};
       bool ok = true;
-      struct Counts { int c[2], n; };   // all the issuer needs of an item
+      struct Counts { int c[2], f[2], n, kv_begin, qid[2]; };   // all the issuer needs of an item
       auto fetch = [&](Counts& it) -> bool {   // next item that has KV tiles
-        for (int idx; (idx = next_item(k)) >= 0;) {
+        for (int idx; (idx = next_item_w(k)) >= 0;) {
           const Item full = make_item(a, idx, window);
-          it.c[0] = full.tl[0].count;
-          it.c[1] = full.tl[1].count;
+#pragma unroll
+          for (int t = 0; t < 2; ++t) {
+            it.c[t] = full.tl[t].count;
+            it.f[t] = full.tl[t].first;
+            it.qid[t] = (full.b * a.Hq + full.tl[t].head) * a.ntq + full.tl[t].row_tile;
+          }
           it.n = full.n;
+          it.kv_begin = full.kv_begin;
           if (it.n > 0) return true;
         }
         return false;
       };
+      // trace hook: the KV tile of stream step `step` was scored for slot t
+      auto trace_s = [&](const Counts& it, int t, int step) {
+        if (a.trace == nullptr) return;
+        const int kt = it.kv_begin + step;
+        if (tr_cnt[t] == 0) tr_first[t] = kt;
+        ++tr_cnt[t];
+        if (step == it.f[t] + it.c[t] - 1) {
+          if (lane == 0) {
+            int32_t* r = a.trace + 3 * (size_t)it.qid[t];
+            r[0] = tr_first[t];
+            r[1] = kt;
+            r[2] = tr_cnt[t];
+          }
+          tr_cnt[t] = 0;
+        }
+      };
       auto issue_first_s = [&](const Counts& it, int t, int ks) -> bool {
-        if (!mbar_wait(&bars[(kRope ? L::Q_READY : L::Q_FULL) + t], qf[t] & 1, abort_flag))
+        if (!mbar_wait_warp(&bars[(kRope ? L::Q_READY : L::Q_FULL) + t], qf[t] & 1, abort_flag))
           return false;
         ++qf[t];
         tc::fence_after();
         issue_s(t, ks);
-        tc::commit(&bars[L::S_FULL + t]);
-        if (it.c[t] == 1) tc::commit(&bars[L::Q_EMPTY + t]);
+        commit(L::S_FULL + t);
+        if (it.c[t] == 1) commit(L::Q_EMPTY + t);
+        trace_s(it, t, it.f[t]);
         return true;
       };
       Counts cur, nxt;
       if (fetch(cur)) {
-        ok = mbar_wait(&bars[L::K_FULL + 0], 0, abort_flag);
+        ok = mbar_wait_warp(&bars[L::K_FULL + 0], 0, abort_flag);
         for (int t = 0; t < 2 && ok; ++t)
-          if (cur.c[t] > 0) ok = issue_first_s(cur, t, 0);
-        if (ok) tc::commit(&bars[L::K_EMPTY + 0]);
+          if (cur.c[t] > 0 && cur.f[t] == 0) ok = issue_first_s(cur, t, 0);
+        if (ok) commit(L::K_EMPTY + 0);
         int j = 0;
         while (ok) {
           const int vs = g % kVS, ksn = (g + 1) % kKS;
           const bool last = j == cur.n - 1;
           const bool more = last ? fetch(nxt) : true;
-          if (!mbar_wait(&bars[L::V_FULL + vs], (g / kVS) & 1, abort_flag)) { ok = false; break; }
+          if (!mbar_wait_warp(&bars[L::V_FULL + vs], (g / kVS) & 1, abort_flag)) { ok = false; break; }
           bool k_next = false;
           auto need_k = [&]() -> bool {
             if (k_next) return true;
-            if (!mbar_wait(&bars[L::K_FULL + ksn], ((g + 1) / kKS) & 1, abort_flag)) return false;
+            if (!mbar_wait_warp(&bars[L::K_FULL + ksn], ((g + 1) / kKS) & 1, abort_flag)) return false;
             tc::fence_after();
             k_next = true;
             return true;
           };
           for (int t = 0; t < 2 && ok; ++t) {
-            const int cnt = cur.c[t];
-            if (j < cnt) {
-              if (!mbar_wait(&bars[L::P_FULL + t], pw[t] & 1, abort_flag)) { ok = false; break; }
+            const int f = cur.f[t], e = f + cur.c[t];
+            if (j >= f && j < e) {
+              if (!mbar_wait_warp(&bars[L::P_FULL + t], pw[t] & 1, abort_flag)) { ok = false; break; }
               ++pw[t];
               tc::fence_after();
-              issue_pv(t, vs, j > 0);
-              if (j == cnt - 1) tc::commit(&bars[L::O_FULL + t]);
+              issue_pv(t, vs, j > f);
+              if (j == e - 1) commit(L::O_FULL + t);
             }
-            if (j + 1 < cnt) {                                 // same item, next tile
+            if (j + 1 >= f && j + 1 < e) {                    // same item, next tile
               if (!need_k()) { ok = false; break; }
-              issue_s(t, ksn);
-              tc::commit(&bars[L::S_FULL + t]);
-              if (j + 2 == cnt) tc::commit(&bars[L::Q_EMPTY + t]);
-            } else if (last && more && nxt.c[t] > 0) {  // next item, first tile
+              if (j + 1 == f) {                               // this slot joins the stream
+                if (!issue_first_s(cur, t, ksn)) { ok = false; break; }
+              } else {
+                issue_s(t, ksn);
+                commit(L::S_FULL + t);
+                if (j + 2 == e) commit(L::Q_EMPTY + t);
+                trace_s(cur, t, j + 1);
+              }
+            } else if (last && more && nxt.c[t] > 0 && nxt.f[t] == 0) {   // next item, first tile
               if (!need_k() || !issue_first_s(nxt, t, ksn)) { ok = false; break; }
             }
           }
           if (!ok) break;
-          tc::commit(&bars[L::V_EMPTY + vs]);
-          if (k_next) tc::commit(&bars[L::K_EMPTY + ksn]);
+          // every K tile the producer loads is released once, even one that
+          // no slot scored (the ranges of an item's tiles leave no gap, so
+          // this does not happen; it keeps the ring in step regardless)
+          if (!k_next && (!last || more) && !need_k()) { ok = false; break; }
+          commit(L::V_EMPTY + vs);
+          if (k_next) commit(L::K_EMPTY + ksn);
           ++g;
           if (!last) {
             ++j;
@@ -538,8 +653,8 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         }
       }
       // every MMA of this CTA must be complete before TMEM is released
-      tc::commit(&bars[L::MMA_DONE]);
-      mbar_wait(&bars[L::MMA_DONE], 0, nullptr);
+      commit(L::MMA_DONE);
+      mbar_wait_warp(&bars[L::MMA_DONE], 0, nullptr);
     }
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax
@@ -548,37 +663,76 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t scol = 128u * t, ocol = 256u + D * t;
     const float sl2 = a.scale_log2;
-    int sw = 0, ow = 0, k = 0, rq = 0;
+    int sw = 0, ow = 0, k = 0;
     bool ok = true;
-    for (int idx; ok && (idx = next_item(k)) >= 0;) {
+    int idx = next_item(k);
+    while (ok && idx >= 0) {
       const Item it = make_item(a, idx, window);
       const Tile T = t == 0 ? it.tl[0] : it.tl[1];
-      if (T.row_tile >= a.ntq) continue;
+      const bool mine = T.row_tile < a.ntq;
       const int row = T.row_tile * kM + r;
-      if constexpr (kRope) {
-        if (T.count > 0) {   // this slot loaded a Q tile for the item: rotate it
-          if (!mbar_wait(&bars[L::Q_FULL + t], rq & 1, abort_flag)) { ok = false; break; }
-          ++rq;
-          if (row < a.Nq) rope_q_row<D>(smem + L::kQ + t * L::kTile, r, row, a);
-          fence_proxy_async_smem();   // the tensor core reads what this thread wrote
-          mbar_arrive(&bars[L::Q_READY + t]);
-        }
-      }
       int vlo, vhi;   // this row's visible keys [vlo, vhi)
       visible_range(row, it.off, a.causal, it.L, window, &vlo, &vhi);
       float m_run = -INFINITY, l_run = 0.f;
 
-      for (int j = 0; j < T.count; ++j) {
+      for (int j = 0; mine && j < T.count; ++j) {
         if (!mbar_wait(&bars[L::S_FULL + t], sw & 1, abort_flag)) { ok = false; break; }
         ++sw;
         tc::fence_after();
-        const int kt = it.kv_begin + j;   // KV tile index
-        const bool masked = kWindow ? (kt < T.um_begin || kt >= T.um_end) : j >= T.um_end;
+        const int kt = it.kv_begin + T.first + j;   // KV tile index
+        const bool masked = kWindow ? (kt < T.um_begin || kt >= T.um_end) : kt >= T.um_end;
         const int lim = vhi - kt * kN;    // keys [base, lim) of this tile are visible
         const int base = vlo - kt * kN;
+        // Unmasked tiles after a row's first: the running max usually stands
+        // (the lazy rescale keeps it unless a score passes it by more than 8
+        // in log2 units), so P is computed with it from a single read of S,
+        // the tile's max taken on the way, and P is written only if no row of
+        // the warp needs a rescale.  Otherwise S is still intact in TMEM and
+        // the two-pass path below runs.  When P is written it is bit for bit
+        // what the two-pass path writes.  (Not in the window instantiation:
+        // there the extra registers spilled and it measured 6% slower.)
+        if (!kWindow && !masked && j > 0) {
+          const float2 c_sl2 = make_float2(sl2, sl2), c_m = make_float2(-m_run, -m_run);
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
+          uint32_t pk[64];
+          float rsum = 0.f;
+#pragma unroll
+          for (int c8 = 0; c8 < kN / 64; ++c8) {
+            float sv[64];
+            tc::ld32f(tmem + lane_off + scol + 64 * c8, sv);
+            tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
+            tc::wait_ld();
+            float2 rs2 = make_float2(0.f, 0.f), rs3 = make_float2(0.f, 0.f);
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              m4[e & 3] = max3(m4[e & 3], sv[2 * e], sv[2 * e + 1]);
+              const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), c_sl2, c_m);
+              const float2 p = (e & 7) < kPolyPairs
+                                   ? exp2_poly2(x)
+                                   : make_float2(exp2_approx(x.x), exp2_approx(x.y));
+              if (e & 1) rs3 = __fadd2_rn(rs3, p); else rs2 = __fadd2_rn(rs2, p);
+              pk[32 * c8 + e] = pack_bf16x2(p.x, p.y);
+            }
+            rs2 = __fadd2_rn(rs2, rs3);
+            rsum += rs2.x + rs2.y;
+          }
+          const float m_tile = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])) * sl2;
+          const bool keep = m_run != -INFINITY && !(m_tile > m_run + kRescaleLog2);
+          if (__all_sync(0xffffffffu, keep)) {
+#pragma unroll
+            for (int c = 0; c < 4; ++c) tc::st16(tmem + lane_off + scol + 16 * c, pk + 16 * c);
+            l_run += rsum;
+            tc::wait_st();
+            tc::fence_before();
+            mbar_arrive(&bars[L::P_FULL + t]);
+            continue;
+          }
+        }
         // pass 1: row max of the (masked) scores
         float mx = -INFINITY;
         if (!masked) {
+          // four independent max chains: the reduction's latency is a quarter
+          float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
           for (int c8 = 0; c8 < kN / 64; ++c8) {
             float sv[64];
@@ -586,8 +740,9 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
             tc::wait_ld();
 #pragma unroll
-            for (int e = 0; e < 32; ++e) mx = max3(mx, sv[2 * e], sv[2 * e + 1]);
+            for (int e = 0; e < 32; ++e) m4[e & 3] = max3(m4[e & 3], sv[2 * e], sv[2 * e + 1]);
           }
+          mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         } else {
 #pragma unroll
           for (int c4 = 0; c4 < kN / 32; ++c4) {
@@ -636,14 +791,17 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
             tc::ld32f(tmem + lane_off + scol + 64 * c8 + 32, sv + 32);
             tc::wait_ld();
             uint32_t pk[32];
-            float2 rs2 = make_float2(0.f, 0.f);
+            float2 rs2 = make_float2(0.f, 0.f), rs3 = make_float2(0.f, 0.f);   // two sum chains
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), c_sl2, c_m);
-              const float2 p = make_float2(exp2_approx(x.x), exp2_approx(x.y));
-              rs2 = __fadd2_rn(rs2, p);
+              const float2 p = (e & 7) < kPolyPairs
+                                   ? exp2_poly2(x)
+                                   : make_float2(exp2_approx(x.x), exp2_approx(x.y));
+              if (e & 1) rs3 = __fadd2_rn(rs3, p); else rs2 = __fadd2_rn(rs2, p);
               pk[e] = pack_bf16x2(p.x, p.y);
             }
+            rs2 = __fadd2_rn(rs2, rs3);
             rs += rs2.x + rs2.y;
             tc::st16(tmem + lane_off + scol + 32 * c8, pk);
             tc::st16(tmem + lane_off + scol + 32 * c8 + 16, pk + 16);
@@ -674,6 +832,11 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
         mbar_arrive(&bars[L::P_FULL + t]);
       }
       if (!ok) break;
+      const int nidx = next_item(k);
+      if (!mine) {
+        idx = nidx;
+        continue;
+      }
 
       // ---- epilogue: O / l -> bf16 straight to global; lse
       const bool have = T.count > 0;
@@ -710,6 +873,7 @@ __global__ void __launch_bounds__(pf::kThreads, 1)
       if (a.lse && row < a.Nq)
         a.lse[((size_t)it.b * a.Hq + T.head) * a.Nq + row] =
             l_run > 0.f ? (m_run + __log2f(l_run)) * kLn2 : -INFINITY;
+      idx = nidx;
     }
   }
 
@@ -736,7 +900,8 @@ void prefill_tile_shape(int d, int* Br, int* Bc) {
 int launch_prefill(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq,
                    int Hkv, int Nq, int Nk, int d, int causal, int window, int align,
                    float scale, const int32_t* key_lens, const float2* rope_tab,
-                   int rope_pairing, void* workspace, int num_sms, cudaStream_t st) {
+                   int rope_pairing, void* workspace, int num_sms, cudaStream_t st,
+                   int32_t* trace) {
   CUtensorMap tq, tk, tv;
   if (make_tmap_3d_bf16(&tq, q, d, Nq, (uint64_t)B * Hq, 64, pf::kM) != ATTN_OK) return ATTN_ECUDA;
   if (make_tmap_2d_bf16(&tk, k, d, (uint64_t)B * Hkv * Nk, 64, pf::kN) != ATTN_OK) return ATTN_ECUDA;
@@ -751,6 +916,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   a.align = align;
   a.rope_tab = rope_tab;
   a.rope_pairing = rope_pairing;
+  a.trace = trace;
   a.ntq = (Nq + pf::kM - 1) / pf::kM;
   a.head_pairs = ((Hq / Hkv) % 2 == 0) ? 1 : 0;
   a.scale_log2 = scale * kLog2e;
@@ -788,7 +954,7 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   const int smem = d == 128 ? pf::Smem<128>::kTotal : pf::Smem<64>::kTotal;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess)
     return ATTN_ECUDA;
-  kern<<<grid, pf::kThreads, smem, st>>>(tq, tk, tv, a);
+  kern<<<grid, pf::threads(rope), smem, st>>>(tq, tk, tv, a);
   return cudaGetLastError() == cudaSuccess ? ATTN_OK : ATTN_ECUDA;
 }
 

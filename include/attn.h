@@ -117,8 +117,9 @@ ATTN_API int attn_fwd_ws(const void* q, const void* k, const void* v, void* o,
  *   causal = 1, row i sees the L - Nq cached keys and new tokens 0..i.  With
  *   L = Nk for every sequence both alignments agree.  The ABI's other entry
  *   points use ATTN_ALIGN_NK.
- *   The prefill kernel visits only the KV tiles that hold visible keys
- *   (attn_fwd_tile_plan_ex reports them); the decode kernels read each
+ *   The prefill kernel scores only the KV tiles that hold visible keys
+ *   (attn_fwd_tile_plan_ex gives them, attn_fwd_trace observes them); the
+ *   decode kernels read each
  *   sequence's keys from the first one its first row sees up to L.
  *   Workspace: attn_workspace_size(...) bytes, as for attn_fwd_ws.
  * Errors: as attn_fwd_ws. */
@@ -233,21 +234,43 @@ ATTN_API size_t attn_rope_workspace_size(int B, int Hq, int Hkv, int Nq, int Nk,
  * dimension d.  Returns ATTN_EUNSUPPORTED for other d. */
 ATTN_API int attn_prefill_tile_shape(int d, int* Br, int* Bc);
 
-/* The KV-tile range the prefill kernel visits for every (b, query tile):
- * writes first[b * nqt + qt] and count[b * nqt + qt] (nqt = ceil(Nq / Br);
- * first = -1, count = 0 when the tile sees no key).  Runs the same device
- * function the prefill kernel uses.  first/count: DEVICE int32 [B * nqt]. */
+/* The closed-form KV-tile range of every (b, query tile): the tiles that
+ * hold a key visible to one of the tile's rows (the causal, key-length,
+ * window and alignment rules of attn_fwd_ex).  Writes first[b * nqt + qt]
+ * and count[b * nqt + qt] (nqt = ceil(Nq / Br); first = -1, count = 0 when
+ * the tile sees no key).  Evaluates the device function the prefill kernel's
+ * scheduler uses; what the kernel itself computes is observed by
+ * attn_fwd_trace.  first/count: DEVICE int32 [B * nqt]. */
 ATTN_API int attn_fwd_tile_plan(int B, int Nq, int Nk, int d, int causal,
                        const int32_t* key_lens, int32_t* first,
                        int32_t* count, void* stream);
 
 /* attn_fwd_tile_plan under a sliding window of `window` keys (0 = none) and
- * a query alignment (as attn_fwd_ex): first = the first KV tile a query tile
- * visits, count = how many in a row (the range covers every visible key of
- * the tile's rows and no tile without one). */
+ * a query alignment (as attn_fwd_ex): first = the first KV tile holding a
+ * key visible to one of the tile's rows, count = how many in a row (the
+ * range covers every visible key of the tile's rows and no tile without
+ * one).  The prefill kernel scores exactly these tiles (attn_fwd_trace). */
 ATTN_API int attn_fwd_tile_plan_ex(int B, int Nq, int Nk, int d, int causal,
                                    int window, int align, const int32_t* key_lens,
                                    int32_t* first, int32_t* count, void* stream);
+
+/* attn_fwd_ex on the prefill kernel with a trace of the work it does (a
+ * test hook; the pages define no such interface): for every query tile
+ * (b, h, qt) of Br rows, the MMA-issuing thread records the first and last
+ * KV tile whose scores it computed for that tile and how many, as it issues
+ * them: trace[((b * Hq + h) * nqt + qt) * 3 + {0, 1, 2}] = {first, last,
+ * count}, nqt = ceil(Nq / Br).  Entries of query tiles that score no KV tile
+ * are not written (initialise them, e.g. to {-1, -1, 0}).  Output as
+ * attn_fwd_ex.
+ *   trace: DEVICE int32 [B * Hq * nqt * 3].  Shapes the decode kernels take
+ *   ((Hq / Hkv) * Nq <= 64, B <= 2048) return ATTN_EUNSUPPORTED.
+ *   Workspace as attn_fwd_ws (attn_workspace_size bytes).
+ * Errors: ATTN_EINVAL for a null trace, else as attn_fwd_ex. */
+ATTN_API int attn_fwd_trace(const void* q, const void* k, const void* v, void* o, float* lse,
+                            int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal,
+                            int window, int align, float scale, const int32_t* key_lens,
+                            void* workspace, size_t workspace_bytes, int32_t* trace,
+                            void* stream);
 
 /* attn_fwd_tile_plan_ex with align = ATTN_ALIGN_NK. */
 ATTN_API int attn_fwd_tile_plan_window(int B, int Nq, int Nk, int d, int causal,

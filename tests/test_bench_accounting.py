@@ -126,3 +126,17 @@ def test_reference_arm_reports_the_same_config(capsys):
         assert per_copy == nbytes
         assert copies * per_copy >= min(2 * bench.L2_BYTES, 8 * per_copy)
         assert copies == 1 or (copies - 1) * per_copy < 2 * bench.L2_BYTES
+
+
+def test_profile_case_keeps_the_group_size():
+    import pytest
+    w = synth.WORKLOADS["long_causal"]
+    c = bench.profile_case(w, 8)
+    assert (c.Hq, c.Hkv, c.Nq, c.Nk, c.d, c.causal) == (8, 8, w.Nq, w.Nk, w.d, w.causal)
+    g = bench.profile_case(synth.WORKLOADS["gqa_rope_prefill"], 8)
+    assert (g.Hq, g.Hkv) == (8, 2)
+    assert bench.profile_case(w, 0) is w
+    # FLOPs scale with the heads (the capture's traffic is scaled the same way)
+    assert c.flops() * 4 == w.flops()
+    with pytest.raises(SystemExit):
+        bench.profile_case(synth.WORKLOADS["gqa_rope_prefill"], 6)
