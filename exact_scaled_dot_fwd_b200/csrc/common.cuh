@@ -124,11 +124,6 @@ __device__ __forceinline__ int paged_cache_row(int entry, int num_pages, int Hkv
   return (entry * Hkv + h) * page_size;
 }
 
-// Barrier `id` (1..15) among `n` threads (a multiple of 32) of the CTA.
-__device__ __forceinline__ void named_bar_sync(int id, int n) {
-  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(n) : "memory");
-}
-
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {
