@@ -58,17 +58,22 @@ KERNEL_SOURCES = {
     "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
 }
 # workload: (kernel, source hash, DRAM bytes read + written per launch).
+# long_causal was captured on its 8-head cut (bench.py --profile-heads 8; the
+# full launch holds 805 MB of inputs) and is scaled by 32 / 8: every head is
+# an independent set of items over its own K/V.
 NCU_TRAFFIC = {
-    "mha_prefill": ("prefill", "2196b26240cb2407", 131482624 + 11721472),
-    "mqa_decode": ("decode", "3f64d81e21fa07a0", 322994688 + 4797952),
+    "long_causal": ("prefill", "1602c19261e2b8d3", (366046464 + 51195136) * 4),
+    "mha_prefill": ("prefill", "1602c19261e2b8d3", 131365632 + 11902208),
+    "mqa_decode": ("decode", "24157ee3a1c5877b", 323002112 + 4591872),
 }
 # Further counters of the same captures (same keys and hash rule): the
 # tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
 # % of peak over the launch) and the DRAM throughput of a decode launch
 # (dram__bytes.sum.per_second, GB/s).
 NCU_COUNTERS = {
-    "mha_prefill": ("prefill", "2196b26240cb2407", {"tensor_pipe_pct": 31.5}),
-    "mqa_decode": ("decode", "3f64d81e21fa07a0", {"dram_gbs": 5534.0}),
+    "long_causal": ("prefill", "1602c19261e2b8d3", {"tensor_pipe_pct": 57.8}),
+    "mha_prefill": ("prefill", "1602c19261e2b8d3", {"tensor_pipe_pct": 32.5}),
+    "mqa_decode": ("decode", "24157ee3a1c5877b", {"dram_gbs": 5480.4}),
 }
 
 
