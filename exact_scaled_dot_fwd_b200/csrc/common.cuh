@@ -124,6 +124,14 @@ __device__ __forceinline__ int paged_cache_row(int entry, int num_pages, int Hkv
   return (entry * Hkv + h) * page_size;
 }
 
+// 32 bytes to global memory in one instruction (a full sector); p must be
+// 32-byte aligned.
+__device__ __forceinline__ void st_global_32B(void* p, uint4 a, uint4 b) {
+  asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x),
+               "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

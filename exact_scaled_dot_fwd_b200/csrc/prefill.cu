@@ -663,6 +663,9 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
     const uint32_t lane_off = (uint32_t)((warp & 3) * 32) << 16;
     const uint32_t scol = 128u * t, ocol = 256u + D * t;
     const float sl2 = a.scale_log2;
+    // (not in the fused-RoPE instantiation: the extra store path made it
+    // spill and measured 1.7% slower there)
+    const bool o_32B = !kRope && (reinterpret_cast<uintptr_t>(a.o) & 31) == 0;
     int sw = 0, ow = 0, k = 0;
     bool ok = true;
     int idx = next_item(k);
@@ -728,6 +731,23 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
             continue;
           }
         }
+        // A masked tile is taken in 32-key chunks, each classified for the
+        // whole warp from the range of its rows' bounds: a chunk no row sees
+        // any key of is skipped (P = 0 without reading S), a chunk every row
+        // sees in full takes no mask, and only the rest is masked per key.
+        // (A causal diagonal tile is one skipped, partial or full chunk per
+        // warp and chunk; a window's edge tile likewise.)
+        int lmin = 0, lmax = 0, bmin = 0, bmax = 0;
+        if (masked) {
+          lmin = __reduce_min_sync(0xffffffffu, lim);
+          lmax = __reduce_max_sync(0xffffffffu, lim);
+          if (kWindow) {
+            bmin = __reduce_min_sync(0xffffffffu, base);
+            bmax = __reduce_max_sync(0xffffffffu, base);
+          }
+        }
+        auto chunk_dead = [&](int c0) { return c0 >= lmax || (kWindow && c0 + 32 <= bmin); };
+        auto chunk_full = [&](int c0) { return c0 + 32 <= lmin && (!kWindow || c0 >= bmax); };
         // pass 1: row max of the (masked) scores
         float mx = -INFINITY;
         if (!masked) {
@@ -744,15 +764,24 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
           }
           mx = fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3]));
         } else {
-#pragma unroll
+#pragma unroll 1
           for (int c4 = 0; c4 < kN / 32; ++c4) {
+            const int c0 = 32 * c4;
+            if (chunk_dead(c0)) continue;
             float sv[32];
-            tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
+            tc::ld32f(tmem + lane_off + scol + c0, sv);
             tc::wait_ld();
+            if (chunk_full(c0)) {
+              float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
-            for (int e = 0; e < 32; ++e) {
-              const int c = 32 * c4 + e;
-              mx = fmaxf(mx, (c >= lim || (kWindow && c < base)) ? -INFINITY : sv[e]);
+              for (int e = 0; e < 16; ++e) m4[e & 3] = max3(m4[e & 3], sv[2 * e], sv[2 * e + 1]);
+              mx = fmaxf(mx, fmaxf(fmaxf(m4[0], m4[1]), fmaxf(m4[2], m4[3])));
+            } else {
+#pragma unroll
+              for (int e = 0; e < 32; ++e) {
+                const int c = c0 + e;
+                mx = fmaxf(mx, (c >= lim || (kWindow && c < base)) ? -INFINITY : sv[e]);
+              }
             }
           }
         }
@@ -807,21 +836,41 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
             tc::st16(tmem + lane_off + scol + 32 * c8 + 16, pk + 16);
           }
         } else {
-#pragma unroll
+#pragma unroll 1
           for (int c4 = 0; c4 < kN / 32; ++c4) {
-            float sv[32];
-            tc::ld32f(tmem + lane_off + scol + 32 * c4, sv);
-            tc::wait_ld();
+            const int c0 = 32 * c4;
             uint32_t pk[16];
+            if (chunk_dead(c0)) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = 32 * c4 + 2 * e;
-              const float x0 = (c >= lim || (kWindow && c < base)) ? -INFINITY : sv[2 * e];
-              const float x1 = (c + 1 >= lim || (kWindow && c + 1 < base)) ? -INFINITY : sv[2 * e + 1];
-              const float p0 = exp2_approx(fmaf(x0, sl2, -m_use));
-              const float p1 = exp2_approx(fmaf(x1, sl2, -m_use));
-              rs += p0 + p1;
-              pk[e] = pack_bf16x2(p0, p1);
+              for (int e = 0; e < 16; ++e) pk[e] = 0u;
+            } else {
+              float sv[32];
+              tc::ld32f(tmem + lane_off + scol + c0, sv);
+              tc::wait_ld();
+              if (chunk_full(c0)) {
+                const float2 c_sl2 = make_float2(sl2, sl2), c_m = make_float2(-m_use, -m_use);
+                float2 rs2 = make_float2(0.f, 0.f), rs3 = make_float2(0.f, 0.f);
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), c_sl2, c_m);
+                  const float2 p = make_float2(exp2_approx(x.x), exp2_approx(x.y));
+                  if (e & 1) rs3 = __fadd2_rn(rs3, p); else rs2 = __fadd2_rn(rs2, p);
+                  pk[e] = pack_bf16x2(p.x, p.y);
+                }
+                rs2 = __fadd2_rn(rs2, rs3);
+                rs += rs2.x + rs2.y;
+              } else {
+#pragma unroll
+                for (int e = 0; e < 16; ++e) {
+                  const int c = c0 + 2 * e;
+                  const float x0 = (c >= lim || (kWindow && c < base)) ? -INFINITY : sv[2 * e];
+                  const float x1 = (c + 1 >= lim || (kWindow && c + 1 < base)) ? -INFINITY : sv[2 * e + 1];
+                  const float p0 = exp2_approx(fmaf(x0, sl2, -m_use));
+                  const float p1 = exp2_approx(fmaf(x1, sl2, -m_use));
+                  rs += p0 + p1;
+                  pk[e] = pack_bf16x2(p0, p1);
+                }
+              }
             }
             tc::st16(tmem + lane_off + scol + 16 * c4, pk);
           }
@@ -858,14 +907,22 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
           for (int e = 0; e < 32; ++e) o[e] = 0.f;
         }
         if (row < a.Nq) {
+          uint4 v[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            uint4 v;
-            v.x = pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
-            v.y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
-            v.z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
-            v.w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
-            *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = v;
+            v[q].x = pack_bf16x2(o[8 * q + 0] * inv, o[8 * q + 1] * inv);
+            v[q].y = pack_bf16x2(o[8 * q + 2] * inv, o[8 * q + 3] * inv);
+            v[q].z = pack_bf16x2(o[8 * q + 4] * inv, o[8 * q + 5] * inv);
+            v[q].w = pack_bf16x2(o[8 * q + 6] * inv, o[8 * q + 7] * inv);
+          }
+          // a row is D * 2 bytes, so its 32-column chunks are 32-byte
+          // aligned whenever o is: one full sector per store
+          if (o_32B) {
+            st_global_32B(orow + 32 * c, v[0], v[1]);
+            st_global_32B(orow + 32 * c + 16, v[2], v[3]);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 4; ++q) *reinterpret_cast<uint4*>(orow + 32 * c + 8 * q) = v[q];
           }
         }
       }
