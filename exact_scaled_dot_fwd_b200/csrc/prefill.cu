@@ -72,6 +72,7 @@ namespace pf {
 
 constexpr int kM = 128;        // query rows per tile (= TMEM lanes)
 constexpr int kN = 128;        // keys per KV tile
+constexpr int kMaxSortB = 64;  // batches up to this size are ordered by key length
 // K/V ring stages: d = 128 fits three K and two V tiles beside the two Q
 // tiles (224 KB); d = 64 fits three of each.
 template <int D> struct Stages { static constexpr int K = 3, V = D == 128 ? 2 : 3; };
@@ -113,7 +114,8 @@ struct Smem {
   static constexpr int kItems = kBar + NUM_BARS * 8;      // int [kItemSlots]
   static constexpr int kTmemSlot = kItems + kItemSlots * 4;
   static constexpr int kAbort = kTmemSlot + 16;
-  static constexpr int kTotal = kAbort + 16 + 1024;   // + alignment slack
+  static constexpr int kPerm = kAbort + 16;              // int [kMaxSortB]
+  static constexpr int kTotal = kPerm + kMaxSortB * 4 + 1024;   // + alignment slack
   static_assert(kTotal <= 232448, "shared memory over the 227 KB per-CTA limit");
 };
 
@@ -146,6 +148,7 @@ struct FwdArgs {
   int units;        // items per cost rank (head_pairs: B*Hq/2, else B*Hq)
   int ranks;        // cost ranks (row tiles, or row-tile pairs)
   int band;         // ranks per band (item order: band, unit, rank in band)
+  int sort_b;       // 1: sequences in the order of their key lengths, longest first
   int total;        // number of items
   float scale_log2;
   int32_t* trace;   // test hook: per query tile {first, last, count} of the KV tiles scored, or null
@@ -165,8 +168,13 @@ struct Item {
 // callers pass a compile-time 0 when the launch has no window).  Ranks walk the row tiles (row pairs)
 // from the most KV tiles to the fewest when causal; bands of `band` ranks
 // keep one unit's (head's) items next to each other so the CTAs that run at
-// the same time share its K/V in L2 (band = 1: plain rank-major order).
-__device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window) {
+// the same time share its K/V in L2 (band = 1: plain rank-major order; a
+// non-causal launch, whose ranks all cost the same, takes one band: unit-
+// major order).  With sort_b the units' sequences come longest first
+// (perm: the sequences by decreasing key length), so the list runs from the
+// most expensive items to the cheapest and the dynamic claim is greedy
+// longest-first across ragged batches too.
+__device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window, const int* perm) {
   Item it;
   const int per_band = a.units * a.band;
   const int full = a.ranks / a.band;
@@ -183,16 +191,18 @@ __device__ __forceinline__ Item make_item(const FwdArgs& a, int idx, int window)
   if (a.head_pairs) {
     const int rt = a.causal ? (a.ntq - 1 - rank) : rank;
     const int hp2 = a.Hq >> 1;
-    it.b = unit / hp2;
-    const int hp = unit - it.b * hp2;
+    const int bs = unit / hp2;
+    const int hp = unit - bs * hp2;
+    it.b = (perm != nullptr && a.sort_b) ? perm[bs] : bs;
     it.tl[0].row_tile = it.tl[1].row_tile = rt;
     it.tl[0].head = 2 * hp;
     it.tl[1].head = 2 * hp + 1;
   } else {
     const int np = (a.ntq + 1) >> 1;
     const int p = a.causal ? (np - 1 - rank) : rank;
-    it.b = unit / a.Hq;
-    const int h = unit - it.b * a.Hq;
+    const int bs = unit / a.Hq;
+    const int h = unit - bs * a.Hq;
+    it.b = (perm != nullptr && a.sort_b) ? perm[bs] : bs;
     it.tl[0].row_tile = 2 * p;
     it.tl[1].row_tile = 2 * p + 1;
     it.tl[0].head = it.tl[1].head = h;
@@ -342,6 +352,9 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::kBar);
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + L::kTmemSlot);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::kAbort);
+  // (the fused-RoPE instantiation keeps the plain order: the lookup pushed
+  // its register allocation into spills, 1.8% slower)
+  const int* perm = kRope ? nullptr : reinterpret_cast<int*>(smem + L::kPerm);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* items = reinterpret_cast<volatile int*>(smem + L::kItems);
@@ -367,6 +380,16 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
     }
     *abort_flag = 0;
     fence_mbar_init();
+  }
+  if (!kRope && a.sort_b && threadIdx.x < a.B) {   // perm[rank] = sequence, longest first, ties by index
+    const int i = threadIdx.x;
+    const int li = clamp_len(a.key_lens[i], a.Nk);
+    int rank = 0;
+    for (int j = 0; j < a.B; ++j) {
+      const int lj = clamp_len(a.key_lens[j], a.Nk);
+      rank += (lj > li || (lj == li && j < i)) ? 1 : 0;
+    }
+    reinterpret_cast<int*>(smem + L::kPerm)[rank] = i;
   }
   if (warp == 8) {
     tc::alloc(tmem_slot, 512);
@@ -394,7 +417,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
         mbar_arrive(&bars[L::ITEM_FULL + slot]);
         ++k;
         if (idx < 0) break;
-        const Item it = make_item(a, idx, window);
+        const Item it = make_item(a, idx, window, perm);
         // claim the next item only while issuing this item's last tile, so
         // no CTA sits on a claimed item (greedy longest-first stays greedy);
         // the atomic's latency hides behind the last loads
@@ -439,7 +462,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
     int qn[2] = {0, 0}, k = 0;
     bool ok = true;
     for (int idx; ok && (idx = next_item(k)) >= 0;) {
-      const Item it = make_item(a, idx, window);
+      const Item it = make_item(a, idx, window, perm);
       if (it.n == 0) continue;
       for (int t = 0; t < 2 && ok; ++t) {
         if (it.tl[t].count == 0) continue;
@@ -472,7 +495,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
       int qn[2] = {0, 0}, k = 0;
       bool ok = true;
       for (int idx; ok && (idx = next_item(k)) >= 0;) {
-        const Item it = make_item(a, idx, window);
+        const Item it = make_item(a, idx, window, perm);
         if (it.n == 0) continue;
         for (int t = 0; t < 2 && ok; ++t) {
           if (it.tl[t].count == 0) continue;
@@ -552,7 +575,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
       struct Counts { int c[2], f[2], n, kv_begin, qid[2]; };   // all the issuer needs of an item
       auto fetch = [&](Counts& it) -> bool {   // next item that has KV tiles
         for (int idx; (idx = next_item_w(k)) >= 0;) {
-          const Item full = make_item(a, idx, window);
+          const Item full = make_item(a, idx, window, perm);
 #pragma unroll
           for (int t = 0; t < 2; ++t) {
             it.c[t] = full.tl[t].count;
@@ -670,7 +693,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
     bool ok = true;
     int idx = next_item(k);
     while (ok && idx >= 0) {
-      const Item it = make_item(a, idx, window);
+      const Item it = make_item(a, idx, window, perm);
       const Tile T = t == 0 ? it.tl[0] : it.tl[1];
       const bool mine = T.row_tile < a.ntq;
       const int row = T.row_tile * kM + r;
@@ -989,12 +1012,15 @@ int launch_prefill(const void* q, const void* k, const void* v, void* o, float* 
   const double kv_head = 4.0 * (double)Nk * d;   // K + V bytes of one kv head
   const double kv_all = kv_head * B * Hkv;
   int band = 1;
-  if (kv_all > 64.0 * (1 << 20)) {
+  if (!causal) {
+    band = a.ranks;
+  } else if (kv_all > 64.0 * (1 << 20)) {
     band = (int)ceil(grid * kv_head / (64.0 * (1 << 20)));
     if (band > a.ranks) band = a.ranks;
     if (band < 1) band = 1;
   }
   a.band = band;
+  a.sort_b = (key_lens != nullptr && B > 1 && B <= pf::kMaxSortB) ? 1 : 0;
   // the item counter starts every launch at zero (stream-ordered)
   if (cudaMemsetAsync(workspace, 0, sizeof(unsigned int), st) != cudaSuccess) return ATTN_ECUDA;
   // a window shifts each tile's first visible key: a separate instantiation
