@@ -62,18 +62,18 @@ KERNEL_SOURCES = {
 # full launch holds 805 MB of inputs) and is scaled by 32 / 8: every head is
 # an independent set of items over its own K/V.
 NCU_TRAFFIC = {
-    "long_causal": ("prefill", "1602c19261e2b8d3", (366046464 + 51195136) * 4),
-    "mha_prefill": ("prefill", "1602c19261e2b8d3", 131365632 + 11902208),
-    "mqa_decode": ("decode", "24157ee3a1c5877b", 323002112 + 4591872),
+    "long_causal": ("prefill", "24333d3b4d07f8e8", (367769344 + 53481984) * 4),
+    "mha_prefill": ("prefill", "24333d3b4d07f8e8", 136520704 + 14329856),
+    "mqa_decode": ("decode", "ec123ff4f7ce4730", 323008256 + 4574976),
 }
 # Further counters of the same captures (same keys and hash rule): the
 # tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
 # % of peak over the launch) and the DRAM throughput of a decode launch
 # (dram__bytes.sum.per_second, GB/s).
 NCU_COUNTERS = {
-    "long_causal": ("prefill", "1602c19261e2b8d3", {"tensor_pipe_pct": 57.8}),
-    "mha_prefill": ("prefill", "1602c19261e2b8d3", {"tensor_pipe_pct": 32.5}),
-    "mqa_decode": ("decode", "24157ee3a1c5877b", {"dram_gbs": 5480.4}),
+    "long_causal": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 59.0}),
+    "mha_prefill": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 35.4}),
+    "mqa_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 5337.3}),
 }
 
 

@@ -132,6 +132,22 @@ __device__ __forceinline__ void st_global_32B(void* p, uint4 a, uint4 b) {
                : "memory");
 }
 
+// Named barrier `id` over `n` threads (a multiple of 32) that also ORs `pred`
+// across them: every thread gets the same answer, so a decision taken on it
+// (leave a loop) is taken by all of them together.
+__device__ __forceinline__ bool bar_vote_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
 // ---------------------------------------------------------------- TMA
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* map) {

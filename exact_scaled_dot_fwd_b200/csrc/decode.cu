@@ -379,7 +379,6 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&empty[st]);
     }
-    if (!alive) break;
 
     // ---- merge the four key quarters of each head tile
 #pragma unroll
@@ -391,7 +390,13 @@ __global__ void __launch_bounds__((MT * 4 + 1) * 32, 1)
       mbuf[(kq * 4 + mt) * 16 + g] = m[0];
       mbuf[(kq * 4 + mt) * 16 + g + 8] = m[1];
     }
-    asm volatile("bar.sync 1, %0;" ::"n"(kConsumerThreads));
+    // A wait that gave up ends the tile loop of its warp only; the consumer
+    // warps leave together here, on a vote at the barrier (one that left
+    // alone would strand the others at it).
+    if (bar_vote_or(1, kConsumerThreads, !alive)) {
+      alive = false;
+      break;
+    }
     float f[2], M[2];
 #pragma unroll
     for (int r = 0; r < 2; ++r) {

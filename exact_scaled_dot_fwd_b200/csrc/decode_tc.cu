@@ -204,18 +204,6 @@ __device__ __forceinline__ void tmem_st_row(uint32_t taddr, const float (&v)[N])
   }
 }
 
-__device__ __forceinline__ bool bar_or(int id, bool pred) {
-  uint32_t r;
-  asm volatile(
-      "{\n\t.reg .pred p, q;\n\t"
-      "setp.ne.u32 p, %1, 0;\n\t"
-      "bar.red.or.pred q, %2, 128, p;\n\t"
-      "selp.u32 %0, 1, 0, q;\n\t}"
-      : "=r"(r)
-      : "r"((uint32_t)pred), "r"(id)
-      : "memory");
-  return r != 0;
-}
 
 }  // namespace dtc
 
@@ -522,7 +510,10 @@ __global__ void __launch_bounds__(192, 1)
       asm volatile("bar.sync 1, 128;" ::: "memory");
       for (int j = 0; j < n; ++j, ++g) {
         const int buf = g & 1;
-        if (!mbar_wait(&bars[L::S_FULL + buf], (g >> 1) & 1, abort_flag)) { ok = false; break; }
+        // A wait that gives up only clears ok: the thread carries on to the
+        // next barrier, where all four warps vote (bar_or) and leave
+        // together -- one that left alone would strand the others at it.
+        if (!mbar_wait(&bars[L::S_FULL + buf], (g >> 1) & 1, abort_flag)) ok = false;
         tc::fence_after();
         float sv[N];
         tmem_ld_row<N>(tmem + lane_off + (uint32_t)(buf * N), sv);
@@ -562,8 +553,10 @@ __global__ void __launch_bounds__(192, 1)
         {
           col_max_to_red<N>(red, warp, lane, sv);
         }
-        if (*abort_flag) { ok = false; break; }
-        asm volatile("bar.sync 1, 128;" ::: "memory");
+        if (bar_vote_or(1, 128, !ok || *abort_flag != 0)) {   // (also orders the red[] writes)
+          ok = false;
+          break;
+        }
         bool need = false;
         if (Lr < N) {
           const float mt = fmaxf(fmaxf(red[Lr], red[64 + Lr]), fmaxf(red[128 + Lr], red[192 + Lr])) * sl2;
@@ -573,7 +566,7 @@ __global__ void __launch_bounds__(192, 1)
           a_s[Lr] = (need && mo != -INFINITY) ? exp2_approx(mo - mn) : 1.f;
           m_s[Lr] = mn;
         }
-        const bool any = bar_or(1, need);
+        const bool any = bar_vote_or(1, 128, need);
         float mu[N];
 #pragma unroll
         for (int h = 0; h < N; ++h) {
@@ -588,26 +581,22 @@ __global__ void __launch_bounds__(192, 1)
             lp[h] *= al[h];
           }
           if (j > 0) {   // O^T holds tiles < j: wait for PV of tile j-1, then rescale
-            if (!mbar_wait(&bars[L::PV_DONE + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag)) {
-              ok = false;
-              break;
-            }
-            tc::fence_after();
-            float o[N];
-            tmem_ld_row<N>(tmem + lane_off + 2u * N, o);
-            tc::wait_ld();
+            if (mbar_wait(&bars[L::PV_DONE + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag)) {
+              tc::fence_after();
+              float o[N];
+              tmem_ld_row<N>(tmem + lane_off + 2u * N, o);
+              tc::wait_ld();
 #pragma unroll
-            for (int h = 0; h < N; ++h) o[h] *= al[h];
-            tmem_st_row<N>(tmem + lane_off + 2u * N, o);
-            tc::wait_st();
+              for (int h = 0; h < N; ++h) o[h] *= al[h];
+              tmem_st_row<N>(tmem + lane_off + 2u * N, o);
+              tc::wait_st();
+            } else {
+              ok = false;
+            }
           }
         }
         // P^T buffer `buf` was read by PV of tile g-2
-        if (g >= 2 &&
-            !mbar_wait(&bars[L::PV_DONE + buf], ((g - 2) >> 1) & 1, abort_flag)) {
-          ok = false;
-          break;
-        }
+        if (g >= 2 && !mbar_wait(&bars[L::PV_DONE + buf], ((g - 2) >> 1) & 1, abort_flag)) ok = false;
         uint8_t* pb_ = p_smem + buf * 2 * L::kPBox + (Lr >> 6) * L::kPBox;
         const int kc = (Lr & 63) >> 3, kb = (Lr & 7) * 2;
 #pragma unroll
@@ -621,18 +610,24 @@ __global__ void __launch_bounds__(192, 1)
         tc::fence_before();
         mbar_arrive(&bars[L::P_FULL + buf]);
       }
-      if (!ok) break;
+      if (bar_vote_or(1, 128, !ok)) {
+        ok = false;
+        break;
+      }
 
       // ---- segment end: per-head sums, O^T / l, partial results
       const int glast = g - 1;
-      if (!mbar_wait(&bars[L::PV_DONE + (glast & 1)], (glast >> 1) & 1, abort_flag)) { ok = false; break; }
+      if (!mbar_wait(&bars[L::PV_DONE + (glast & 1)], (glast >> 1) & 1, abort_flag)) ok = false;
       tc::fence_after();
       float o[N];
       tmem_ld_row<N>(tmem + lane_off + 2u * N, o);
       tc::wait_ld();
       bfly_reduce<N, true>(lp, lane);
       put_red<N>(red, warp, lane, lp);
-      asm volatile("bar.sync 1, 128;" ::: "memory");
+      if (bar_vote_or(1, 128, !ok)) {
+        ok = false;
+        break;
+      }
       if (Lr < N) l_s[Lr] = (red[Lr] + red[64 + Lr]) + (red[128 + Lr] + red[192 + Lr]);
       asm volatile("bar.sync 1, 128;" ::: "memory");
       const size_t slot = (size_t)blockIdx.x + s.u;
