@@ -211,6 +211,28 @@ def test_large_scores_stay_finite(torch):
     check_workload(x, (B, H, N, d), True, 1.0, what="large scores")
 
 
+@pytest.mark.parametrize("B,H,N,d,causal,window", [(2, 2, 1000, 128, True, 0),
+                                                  (1, 2, 700, 64, False, 0),
+                                                  (1, 2, 1200, 128, True, 300)])
+def test_max_rises_inside_a_tile(torch, B, H, N, d, causal, window):
+    """Scores 12 t (natural units, scale 1) on the second half of KV tile t's
+    keys and about 0 on the first: in every unmasked tile after a row's first
+    the max rises by ~17 log2 units within the tile's second half, the case in
+    which the kernel rescales the first half's P in place.  Compared with the
+    oracle (fp64, the definition without any running max) on every row."""
+    rng = np.random.default_rng(77 + d)
+    q = rng.normal(0.0, 0.25, (B, H, N, d))
+    k = rng.normal(0.0, 0.25, (B, H, N, d))
+    v = rng.normal(0.0, 1.0, (B, H, N, d))
+    q[..., 0] = 1.0
+    j = np.arange(N)
+    k[..., 0] = np.where(j % 128 >= 64, 12.0 * (j // 128), 0.0)
+    x = {"q": synth.bf16_bits_from_f32(q.astype(np.float32)),
+         "k": synth.bf16_bits_from_f32(k.astype(np.float32)),
+         "v": synth.bf16_bits_from_f32(v.astype(np.float32)), "key_lens": None}
+    check_workload(x, (B, H, N, d), causal, 1.0, what="max rising in a tile", window=window)
+
+
 def test_deterministic(torch):
     w = synth.WORKLOADS["tiny_causal"]
     x = synth.make_inputs(w)
