@@ -58,13 +58,18 @@ KERNEL_SOURCES = {
     "decode": ["decode_tc.cu", "tcgen05.cuh", "common.cuh", "tile_plan.cuh"],
 }
 # workload: (kernel, source hash, DRAM bytes read + written per launch).
-# long_causal was captured on its 8-head cut (bench.py --profile-heads 8; the
-# full launch holds 805 MB of inputs) and is scaled by 32 / 8: every head is
-# an independent set of items over its own K/V.
+# long_causal and long_window were captured on their 8-head cuts (bench.py
+# --profile-heads 8; a full launch holds 805 MB of inputs) and are scaled by
+# 32 / 8: every head is an independent set of items over its own K/V.
+# paged_decode is mqa_decode over a cache of 16-token pages (the bench's
+# paged_decode object).
 NCU_TRAFFIC = {
     "long_causal": ("prefill", "24333d3b4d07f8e8", (367769344 + 53481984) * 4),
     "mha_prefill": ("prefill", "24333d3b4d07f8e8", 136520704 + 14329856),
+    "long_window": ("prefill", "24333d3b4d07f8e8", (240082944 + 48610304) * 4),
     "mqa_decode": ("decode", "ec123ff4f7ce4730", 323008256 + 4574976),
+    "spec_decode": ("decode", "ec123ff4f7ce4730", 508930816 + 4898048),
+    "paged_decode": ("decode", "ec123ff4f7ce4730", 319074304 + 4990208),
 }
 # Further counters of the same captures (same keys and hash rule): the
 # tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
@@ -73,7 +78,10 @@ NCU_TRAFFIC = {
 NCU_COUNTERS = {
     "long_causal": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 59.0}),
     "mha_prefill": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 35.4}),
+    "long_window": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 46.5}),
     "mqa_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 5337.3}),
+    "spec_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 6152.2}),
+    "paged_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 4247.9}),
 }
 
 
@@ -576,7 +584,8 @@ def run_decode(torch, eb, device, stream, peaks, peak_src, steps=None, name="mqa
             "page_size": page_size or None,
             "algorithmic_bytes": decode_bytes(w, x["key_lens"]),
             "l2": f"{copies} rotating KV caches ({copies * per_copy / 1e6:.0f} MB allocated)",
-            "roofline": roofline("hbm", gbs, peaks, peak_src, w.name),
+            "roofline": roofline("hbm", gbs, peaks, peak_src,
+                                 "paged_decode" if page_size else w.name),
             "gpu_launches": 2 * n}
 
 
