@@ -216,36 +216,6 @@ __device__ __forceinline__ float exp2_approx(float x) {
   return y;
 }
 
-// 2^x for two values on the FMA and integer pipes (no SFU), so a softmax can
-// split its exponentials between the SFU and the FMA units.  Method: the
-// classic range reduction x = j + f with j = round(x), |f| <= 1/2 (Cody and
-// Waite's split), 2^f from a polynomial and 2^j added into the exponent field.
-//   - j comes from the rounding addition t = x + 1.5 * 2^23: in round-to-
-//     nearest the low mantissa bits of t hold j (two's complement), so
-//     (bits(t) << 23) is j in the exponent position and t - 1.5 * 2^23 is j
-//     exactly; f = x - j is exact.
-//   - 2^f ~ 1 + f (c1 + f (c2 + f c3)): a degree-3 fit with p(0) = 1 that
-//     minimises the maximum relative error over [-1/2, 1/2] (a linear
-//     programme over 4001 points, coefficients rounded to fp32); measured
-//     maximum relative error 1.01e-4 against exp2 over [-125, 10].
-//   - x is clamped to >= -125 so that j + exponent(p) stays a normal number:
-//     inputs below give about 2^-125 (~2e-38) instead of 0.  Callers use it
-//     only where no input is -inf (unmasked tiles).  x must be < 127.
-__device__ __forceinline__ float2 exp2_poly2(float2 x) {
-  constexpr float kC1 = 0x1.62f5fap-1f, kC2 = 0x1.f00c4cp-3f, kC3 = 0x1.c2a21ap-5f;
-  constexpr float kRound = 12582912.0f;   // 1.5 * 2^23
-  x.x = fmaxf(x.x, -125.f);
-  x.y = fmaxf(x.y, -125.f);
-  const float2 t = __fadd2_rn(x, make_float2(kRound, kRound));
-  const float2 j = __fadd2_rn(t, make_float2(-kRound, -kRound));
-  const float2 f = __ffma2_rn(j, make_float2(-1.f, -1.f), x);
-  float2 p = __ffma2_rn(f, make_float2(kC3, kC3), make_float2(kC2, kC2));
-  p = __ffma2_rn(p, f, make_float2(kC1, kC1));
-  p = __ffma2_rn(p, f, make_float2(1.f, 1.f));
-  return make_float2(__uint_as_float(__float_as_uint(p.x) + (__float_as_uint(t.x) << 23)),
-                     __uint_as_float(__float_as_uint(p.y) + (__float_as_uint(t.y) << 23)));
-}
-
 // Two fp32 -> packed bf16x2 (round to nearest even); `lo` in the low half.
 __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   uint32_t r;

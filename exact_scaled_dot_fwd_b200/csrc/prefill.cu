@@ -333,13 +333,6 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
   using namespace pf;
   using L = Smem<D>;
   constexpr int kBoxes = D / 64;
-  // Exponentials of unmasked tiles: at d = 64 the MMAs take half the time
-  // per score that they take at d = 128 while the exponentials stay, so 3 of
-  // every 8 score pairs take 2^x from a polynomial on the FMA pipe
-  // (exp2_poly2) and the SFU does the rest (measured +4% on the padded
-  // cross-attention workload; at d = 128 the split measured slower and the
-  // SFU does all of them)
-  constexpr int kPolyPairs = D == 64 ? 3 : 0;
   const int window = kWindow ? a.window : 0;
   constexpr int kKS = L::kKS, kVS = L::kVS;
   // TMEM columns: S of tile t at 128 t, O of tile t at 256 + D t
@@ -733,9 +726,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
             for (int e = 0; e < 32; ++e) {
               m4[e & 3] = max3(m4[e & 3], sv[2 * e], sv[2 * e + 1]);
               const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), c_sl2, c_m);
-              const float2 p = (e & 7) < kPolyPairs
-                                   ? exp2_poly2(x)
-                                   : make_float2(exp2_approx(x.x), exp2_approx(x.y));
+              const float2 p = make_float2(exp2_approx(x.x), exp2_approx(x.y));
               if (e & 1) rs3 = __fadd2_rn(rs3, p); else rs2 = __fadd2_rn(rs2, p);
               pk[32 * c8 + e] = pack_bf16x2(p.x, p.y);
             }
@@ -847,9 +838,7 @@ __global__ void __launch_bounds__(pf::threads(kRope), 1)
 #pragma unroll
             for (int e = 0; e < 32; ++e) {
               const float2 x = __ffma2_rn(make_float2(sv[2 * e], sv[2 * e + 1]), c_sl2, c_m);
-              const float2 p = (e & 7) < kPolyPairs
-                                   ? exp2_poly2(x)
-                                   : make_float2(exp2_approx(x.x), exp2_approx(x.y));
+              const float2 p = make_float2(exp2_approx(x.x), exp2_approx(x.y));
               if (e & 1) rs3 = __fadd2_rn(rs3, p); else rs2 = __fadd2_rn(rs2, p);
               pk[e] = pack_bf16x2(p.x, p.y);
             }
