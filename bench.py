@@ -64,24 +64,24 @@ KERNEL_SOURCES = {
 # paged_decode is mqa_decode over a cache of 16-token pages (the bench's
 # paged_decode object).
 NCU_TRAFFIC = {
-    "long_causal": ("prefill", "24333d3b4d07f8e8", (367769344 + 53481984) * 4),
-    "mha_prefill": ("prefill", "24333d3b4d07f8e8", 136520704 + 14329856),
-    "long_window": ("prefill", "24333d3b4d07f8e8", (240082944 + 48610304) * 4),
-    "mqa_decode": ("decode", "ec123ff4f7ce4730", 323008256 + 4574976),
-    "spec_decode": ("decode", "ec123ff4f7ce4730", 508930816 + 4898048),
-    "paged_decode": ("decode", "ec123ff4f7ce4730", 319074304 + 4990208),
+    "long_causal": ("prefill", "cf9fb7b089ed0128", (362489088 + 53635072) * 4),
+    "mha_prefill": ("prefill", "cf9fb7b089ed0128", 132578304 + 13372928),
+    "long_window": ("prefill", "cf9fb7b089ed0128", (241136128 + 48871424) * 4),
+    "mqa_decode": ("decode", "cb6f97e893d32d89", 323006976 + 4521216),
+    "spec_decode": ("decode", "cb6f97e893d32d89", 508926464 + 4657920),
+    "paged_decode": ("decode", "cb6f97e893d32d89", 319148032 + 5268992),
 }
 # Further counters of the same captures (same keys and hash rule): the
 # tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
 # % of peak over the launch) and the DRAM throughput of a decode launch
 # (dram__bytes.sum.per_second, GB/s).
 NCU_COUNTERS = {
-    "long_causal": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 59.0}),
-    "mha_prefill": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 35.4}),
-    "long_window": ("prefill", "24333d3b4d07f8e8", {"tensor_pipe_pct": 46.5}),
-    "mqa_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 5337.3}),
-    "spec_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 6152.2}),
-    "paged_decode": ("decode", "ec123ff4f7ce4730", {"dram_gbs": 4247.9}),
+    "long_causal": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 58.9}),
+    "mha_prefill": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 35.5}),
+    "long_window": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 46.5}),
+    "mqa_decode": ("decode", "cb6f97e893d32d89", {"dram_gbs": 5424.1}),
+    "spec_decode": ("decode", "cb6f97e893d32d89", {"dram_gbs": 6079.4}),
+    "paged_decode": ("decode", "cb6f97e893d32d89", {"dram_gbs": 4286.7}),
 }
 
 
