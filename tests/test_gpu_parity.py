@@ -233,6 +233,17 @@ def test_max_rises_inside_a_tile(torch, B, H, N, d, causal, window):
     check_workload(x, (B, H, N, d), causal, 1.0, what="max rising in a tile", window=window)
 
 
+@pytest.mark.parametrize("B,causal", [(64, True), (65, False)])
+def test_ragged_batch_at_the_ordering_limit(torch, B, causal):
+    """Batches of up to 64 sequences with key lengths run longest first (the
+    kernel ranks them at launch), larger ones in index order: both sides of
+    that limit, ragged lengths, every row against the oracle."""
+    rng = np.random.default_rng(900 + B)
+    kl = [int(x) for x in rng.integers(0, 301, size=B)]
+    x = rand_inputs(B, 2, 2, 300, 300, 64, seed=61 + B, key_lens=kl)
+    check_workload(x, (B, 2, 300, 64), causal, 0.125, what=f"B={B} ragged")
+
+
 def test_deterministic(torch):
     w = synth.WORKLOADS["tiny_causal"]
     x = synth.make_inputs(w)
