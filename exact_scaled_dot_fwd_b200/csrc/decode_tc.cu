@@ -492,6 +492,11 @@ __global__ void __launch_bounds__(192, 1)
     const int Lr = warp * 32 + lane;                 // key row of S^T, dimension of O^T
     const uint32_t lane_off = (uint32_t)(warp * 32) << 16;
     const float sl2 = a.scale_log2;
+    // Above 32 rows a thread cannot keep its whole row of S^T in registers
+    // beside its N running sums: it reads S^T from TMEM in 32-column parts,
+    // once for the maxima and again for P.
+    constexpr bool kReload = N > 32;
+    constexpr int NC = kReload ? 32 : N;
     uint8_t* p_smem = smem + L::kP;
     int u = u0, g = 0;
     Seg s;
@@ -515,15 +520,8 @@ __global__ void __launch_bounds__(192, 1)
         // together -- one that left alone would strand the others at it.
         if (!mbar_wait(&bars[L::S_FULL + buf], (g >> 1) & 1, abort_flag)) ok = false;
         tc::fence_after();
-        float sv[N];
-        tmem_ld_row<N>(tmem + lane_off + (uint32_t)(buf * N), sv);
-        tc::wait_ld();
         const int kfirst = s.base + j * kTile;   // absolute key of this tile's row 0
         const bool valid = kfirst + Lr < s.end && (!kPaged || kfirst + Lr >= s.start);
-        if (!valid) {
-#pragma unroll
-          for (int h = 0; h < N; ++h) sv[h] = -INFINITY;
-        }
         // rows (tokens) that do not see every key of this tile: causal keys
         // past row 0's position, window keys before the last row's window
         const int klast = kfirst + kTile - 1;
@@ -531,27 +529,41 @@ __global__ void __launch_bounds__(192, 1)
             (a.causal && klast > off) ||
             (a.window > 0 && ((long long)kfirst < (long long)off + a.Nq - a.window ||
                               (!a.causal && (long long)klast >= (long long)off + a.window)));
+        // this key is visible to the rows whose token index t satisfies
+        // t >= key - off (causal) and |off + t - key| < window
+        int tlo = -(1 << 30), thi = 1 << 30;
         if (tile_mask) {
-          // this key is visible to the rows whose token index t satisfies
-          // t >= key - off (causal) and |off + t - key| < window
           const int key = kfirst + Lr;
-          int tlo = a.causal ? key - off : -(1 << 30);
-          int thi = 1 << 30;
+          if (a.causal) tlo = key - off;
           if (a.window > 0) {
             const int wlo = key - off - a.window + 1;
             tlo = tlo > wlo ? tlo : wlo;
             thi = key - off + a.window - 1;
           }
-          int t = 0;
-#pragma unroll
-          for (int h = 0; h < N; ++h) {
-            if (t < tlo || t > thi) sv[h] = -INFINITY;
-            t = t + 1 == a.Nq ? 0 : t + 1;
-          }
         }
+        // S^T columns h0 .. h0 + NC of buffer `buf`, masked
+        float sv[NC];
+        auto load_s = [&](int h0) {
+          tmem_ld_row<NC>(tmem + lane_off + (uint32_t)(buf * N + h0), sv);
+          tc::wait_ld();
+          if (!valid) {
+#pragma unroll
+            for (int h = 0; h < NC; ++h) sv[h] = -INFINITY;
+          }
+          if (tile_mask) {
+            int t = h0 % a.Nq;
+#pragma unroll
+            for (int h = 0; h < NC; ++h) {
+              if (t < tlo || t > thi) sv[h] = -INFINITY;
+              t = t + 1 == a.Nq ? 0 : t + 1;
+            }
+          }
+        };
         // per-head max over the tile's keys
-        {
-          col_max_to_red<N>(red, warp, lane, sv);
+#pragma unroll
+        for (int h0 = 0; h0 < N; h0 += NC) {
+          load_s(h0);
+          col_max_to_red<NC>(red + h0, warp, lane, sv);
         }
         if (bar_vote_or(1, 128, !ok || *abort_flag != 0)) {   // (also orders the red[] writes)
           ok = false;
@@ -567,12 +579,15 @@ __global__ void __launch_bounds__(192, 1)
           m_s[Lr] = mn;
         }
         const bool any = bar_vote_or(1, 128, need);
-        float mu[N];
+        float mu[NC];
+        auto load_mu = [&](int h0) {
 #pragma unroll
-        for (int h = 0; h < N; ++h) {
-          const float m = m_s[h];
-          mu[h] = m == -INFINITY ? 0.f : m;
-        }
+          for (int h = 0; h < NC; ++h) {
+            const float m = m_s[h0 + h];
+            mu[h] = m == -INFINITY ? 0.f : m;
+          }
+        };
+        if (!kReload) load_mu(0);
         if (any) {
           float al[N];
 #pragma unroll
@@ -583,12 +598,15 @@ __global__ void __launch_bounds__(192, 1)
           if (j > 0) {   // O^T holds tiles < j: wait for PV of tile j-1, then rescale
             if (mbar_wait(&bars[L::PV_DONE + ((g - 1) & 1)], ((g - 1) >> 1) & 1, abort_flag)) {
               tc::fence_after();
-              float o[N];
-              tmem_ld_row<N>(tmem + lane_off + 2u * N, o);
-              tc::wait_ld();
 #pragma unroll
-              for (int h = 0; h < N; ++h) o[h] *= al[h];
-              tmem_st_row<N>(tmem + lane_off + 2u * N, o);
+              for (int h0 = 0; h0 < N; h0 += NC) {
+                float o[NC];
+                tmem_ld_row<NC>(tmem + lane_off + 2u * N + h0, o);
+                tc::wait_ld();
+#pragma unroll
+                for (int h = 0; h < NC; ++h) o[h] *= al[h0 + h];
+                tmem_st_row<NC>(tmem + lane_off + 2u * N + h0, o);
+              }
               tc::wait_st();
             } else {
               ok = false;
@@ -600,11 +618,19 @@ __global__ void __launch_bounds__(192, 1)
         uint8_t* pb_ = p_smem + buf * 2 * L::kPBox + (Lr >> 6) * L::kPBox;
         const int kc = (Lr & 63) >> 3, kb = (Lr & 7) * 2;
 #pragma unroll
-        for (int h = 0; h < N; ++h) {
-          const float p = exp2_approx(fmaf(sv[h], sl2, -mu[h]));
-          lp[h] += p;
-          const uint32_t off = (uint32_t)h * 128u + (uint32_t)((kc ^ (h & 7)) << 4) + kb;
-          *reinterpret_cast<__nv_bfloat16*>(pb_ + off) = __float2bfloat16_rn(p);
+        for (int h0 = 0; h0 < N; h0 += NC) {
+          if (kReload) {   // S^T is still in TMEM: its buffer is reused after P_FULL
+            load_s(h0);
+            load_mu(h0);   // before this part's P stores
+          }
+#pragma unroll
+          for (int h = 0; h < NC; ++h) {
+            const float p = exp2_approx(fmaf(sv[h], sl2, -mu[h]));
+            lp[h0 + h] += p;
+            const int hh = h0 + h;
+            const uint32_t off = (uint32_t)hh * 128u + (uint32_t)((kc ^ (hh & 7)) << 4) + kb;
+            *reinterpret_cast<__nv_bfloat16*>(pb_ + off) = __float2bfloat16_rn(p);
+          }
         }
         fence_proxy_async_smem();
         tc::fence_before();

@@ -38,6 +38,8 @@ CASES = [
     (2, 8, 8, 7, 500, 128, True, 0, 1, [500, 260]),                 # 7 tokens, MHA
     (3, 16, 4, 5, 1000, 64, True, 0, 1, [1000, 640, 77]),           # d = 64 (mma.sync)
     (2, 4, 1, 16, 900, 64, True, 0, 1, [900, 333]),                 # d = 64, 64 rows
+    (2, 16, 1, 3, 1500, 128, True, 0, 1, [1500, 777]),              # 48 rows: S read in two parts, 32 % Nq != 0
+    (3, 8, 1, 5, 1200, 128, True, 150, 1, [1200, 600, 40]),         # 40 rows, sliding window
     (2, 16, 2, 8, 1024, 128, True, 0, 0, None),                     # full caches, align 0
     (2, 8, 2, 3, 700, 128, False, 0, 1, [700, 300]),                # not causal
     (3, 16, 4, 4, 2000, 128, True, 300, 1, [2000, 1000, 200]),      # sliding window

@@ -55,6 +55,7 @@ CASES = [
     (2, 32, 8, 1, 1000, 128, 128, True, 0, [1000, 127]),             # one page per tile
     (3, 32, 8, 4, 2500, 128, 16, True, 0, [2500, 5, 1024]),          # multi-token, GQA
     (2, 16, 4, 2, 3000, 128, 16, True, 500, [3000, 700]),            # window
+    (2, 16, 1, 3, 1800, 128, 32, True, 0, [1800, 900]),              # 48 rows per kv head
     (3, 16, 4, 1, 1200, 64, 16, True, 0, [1200, 33, 64]),            # d = 64 (mma.sync)
     (2, 8, 2, 3, 900, 64, 64, True, 0, [900, 100]),                  # d = 64, multi-token
     (2, 8, 2, 1, 900, 64, 8, False, 200, [900, 500]),                # d = 64, window
