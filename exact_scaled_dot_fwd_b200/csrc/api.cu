@@ -117,6 +117,21 @@ int make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_
   return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ECUDA;
 }
 
+int make_tmap_grouped_bf16(CUtensorMap* map, const void* base, uint64_t rows,
+                           uint32_t box_groups) {
+  EncodeTiledFn fn = encode_fn();
+  if (!fn || rows % 8 != 0) return ATTN_ECUDA;
+  // (64 columns, 8 rows, 2 halves, rows / 8 groups); a row is 256 bytes
+  cuuint64_t dims[4] = {64, 8, 2, rows / 8};
+  cuuint64_t strides[3] = {256, 128, 2048};
+  cuuint32_t box[4] = {64, 8, 2, box_groups};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? ATTN_OK : ATTN_ECUDA;
+}
+
 // Failure-detection hook: one thread waits on an mbarrier that nothing ever
 // arrives on, with a short limit; the wait gives up, records ATTN_ETIMEOUT and
 // the kernel returns.  No fault, no hang.

@@ -63,7 +63,13 @@ struct Smem {
   static constexpr int KS = KS_;                  // K ring stages
   static constexpr int VS = VS_;                  // V ring stages
   static constexpr int kKV = kTile * kD * 2;   // one K or V tile (32 KB)
+  // A K/V tile of a contiguous cache lands as two 64-column halves of 128
+  // keys (kBox apart); one of a paged cache as 16 groups of 8 keys, each
+  // [half 0 | half 1] of 1 KB, so that a page is one TMA box.  In both, each
+  // half is a column of 1 KB 128-byte-swizzled atoms at a uniform stride.
   static constexpr int kBox = kTile * 128;     // 64-column box of a K/V tile
+  static constexpr uint32_t half_step(bool paged) { return paged ? 1024u : (uint32_t)kBox; }
+  static constexpr uint32_t group_stride(bool paged) { return paged ? 2048u : 1024u; }
   static constexpr int kQBox = N * 128;        // 64-column box of Q (N rows)
   static constexpr int kPBox = N * 128;        // 64-key box of P^T (N rows)
   static constexpr int kK = 0;
@@ -374,7 +380,7 @@ __global__ void __launch_bounds__(192, 1)
                      : a.oob_row;
         };
         int prow = kPaged ? page_row(0) : 0;
-        const uint32_t so = kPaged ? (uint32_t)(lane * a.page_size * 128) : 0u;
+        const uint32_t so = kPaged ? (uint32_t)(lane * a.page_size * 256) : 0u;   // page's groups
         for (int j = 0; j < n; ++j, ++g) {
           const int ks = g % KS, vs = g % VS;
           const int pnext = (kPaged && j + 1 < n) ? page_row(j + 1) : 0;
@@ -385,20 +391,32 @@ __global__ void __launch_bounds__(192, 1)
           }
           if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
           ++gk;
-          if (issuer)
-            for (int bx = 0; bx < 2; ++bx)
-              tma_load_2d(smem + L::kK + ks * L::kKV + bx * L::kBox + so, &tmap_k, bx * 64, r,
+          if (issuer) {
+            if constexpr (kPaged) {
+              tma_load_4d(smem + L::kK + ks * L::kKV + so, &tmap_k, 0, 0, 0, r >> 3,
                           &bars[L::K_FULL + ks]);
+            } else {
+              for (int bx = 0; bx < 2; ++bx)
+                tma_load_2d(smem + L::kK + ks * L::kKV + bx * L::kBox, &tmap_k, bx * 64, r,
+                            &bars[L::K_FULL + ks]);
+            }
+          }
           if (lane == 0) {
             w = mbar_wait(&bars[L::V_EMPTY + vs], ((g / VS) & 1) ^ 1, abort_flag);
             if (w) mbar_arrive_expect_tx(&bars[L::V_FULL + vs], L::kKV);
           }
           if (!__shfl_sync(0xffffffffu, w, 0)) { ok = false; break; }
           ++gv;
-          if (issuer)
-            for (int bx = 0; bx < 2; ++bx)
-              tma_load_2d(smem + L::kV + vs * L::kKV + bx * L::kBox + so, &tmap_v, bx * 64, r,
+          if (issuer) {
+            if constexpr (kPaged) {
+              tma_load_4d(smem + L::kV + vs * L::kKV + so, &tmap_v, 0, 0, 0, r >> 3,
                           &bars[L::V_FULL + vs]);
+            } else {
+              for (int bx = 0; bx < 2; ++bx)
+                tma_load_2d(smem + L::kV + vs * L::kKV + bx * L::kBox, &tmap_v, bx * 64, r,
+                            &bars[L::V_FULL + vs]);
+            }
+          }
           prow = pnext;
         }
       }
@@ -421,27 +439,29 @@ __global__ void __launch_bounds__(192, 1)
       const uint32_t q_base = smem_u32(smem + L::kQ), p_base = smem_u32(smem + L::kP);
       // descriptors built once per call; a k-step only moves the start
       // address field (address >> 4 in bits 0-13, no carry below 256 KB)
+      // a k-step of 16 keys is two 8-key groups; one of 64 columns a half
+      constexpr uint32_t kHalf = L::half_step(kPaged), kGroup = L::group_stride(kPaged);
       auto issue_s = [&](int g) {
-        const uint64_t dk = tc::smem_desc_sw128(k_base + (g % KS) * L::kKV, 16, 1024);
+        const uint64_t dk = tc::smem_desc_sw128(k_base + (g % KS) * L::kKV, 16, kGroup);
         const uint64_t dq = tc::smem_desc_sw128(q_base, 16, 1024);
         const uint32_t dt = tmem + (uint32_t)((g & 1) * N);
         if (elect_one()) {
           tc::mma_ss(dt, dk, dq, kIdescS, 0u);
 #pragma unroll
           for (int kk = 1; kk < kD / 16; ++kk)
-            tc::mma_ss(dt, dk + (uint64_t)(((kk >> 2) * L::kBox + (kk & 3) * 32) >> 4),
+            tc::mma_ss(dt, dk + (uint64_t)(((kk >> 2) * kHalf + (kk & 3) * 32) >> 4),
                        dq + (uint64_t)(((kk >> 2) * L::kQBox + (kk & 3) * 32) >> 4), kIdescS, 1u);
         }
         __syncwarp();
       };
       auto issue_pv = [&](int g, bool acc) {
-        const uint64_t dv = tc::smem_desc_sw128(v_base + (g % VS) * L::kKV, L::kBox, 1024);
+        const uint64_t dv = tc::smem_desc_sw128(v_base + (g % VS) * L::kKV, kHalf, kGroup);
         const uint64_t dp = tc::smem_desc_sw128(p_base + (g & 1) * 2 * L::kPBox, 16, 1024);
         if (elect_one()) {
           tc::mma_ss(tmem + 2u * N, dv, dp, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
           for (int kk = 1; kk < kTile / 16; ++kk)
-            tc::mma_ss(tmem + 2u * N, dv + (uint64_t)((kk * 16 * 128) >> 4),
+            tc::mma_ss(tmem + 2u * N, dv + (uint64_t)((kk * 2 * kGroup) >> 4),
                        dp + (uint64_t)(((kk >> 2) * L::kPBox + (kk & 3) * 32) >> 4), kIdescPV, 1u);
         }
         __syncwarp();
@@ -713,15 +733,20 @@ int launch_decode_split_tc(const void* q, const void* k, const void* v, int B, i
   const int G = Hq / Hkv, R = G * Nq;
   const int N = R <= 16 ? 16 : (R <= 32 ? 32 : 64);
   CUtensorMap tq, tk, tv;
-  // contiguous: [B * Hkv * Nk, d] in 128-row boxes; paged: [num_pages * Hkv *
-  // page_size, d] in page_size-row boxes
+  // contiguous: [B * Hkv * Nk, d] in 128-row, 64-column boxes; paged:
+  // [num_pages * Hkv * page_size, d] in 8-row groups, one page per box
   const uint64_t rows = pg ? (uint64_t)pg->num_pages * Hkv * pg->page_size
                            : (uint64_t)B * Hkv * Nk;
-  const uint32_t box = pg ? (uint32_t)pg->page_size : (uint32_t)dtc::kTile;
   if (make_tmap_2d_bf16(&tq, q, dtc::kD, (uint64_t)B * Hq * Nq, 64, (uint32_t)N) != ATTN_OK)
     return ATTN_ECUDA;
-  if (make_tmap_2d_bf16(&tk, k, dtc::kD, rows, 64, box) != ATTN_OK) return ATTN_ECUDA;
-  if (make_tmap_2d_bf16(&tv, v, dtc::kD, rows, 64, box) != ATTN_OK) return ATTN_ECUDA;
+  if (pg) {
+    const uint32_t groups = (uint32_t)pg->page_size / 8;
+    if (make_tmap_grouped_bf16(&tk, k, rows, groups) != ATTN_OK) return ATTN_ECUDA;
+    if (make_tmap_grouped_bf16(&tv, v, rows, groups) != ATTN_OK) return ATTN_ECUDA;
+  } else {
+    if (make_tmap_2d_bf16(&tk, k, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
+    if (make_tmap_2d_bf16(&tv, v, dtc::kD, rows, 64, dtc::kTile) != ATTN_OK) return ATTN_ECUDA;
+  }
   DecodeTcArgs a;
   a.block_table = pg ? pg->block_table : nullptr;
   a.max_pages = pg ? pg->max_pages : 0;

@@ -22,6 +22,14 @@ int make_tmap_2d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_
 int make_tmap_3d_bf16(CUtensorMap* map, const void* base, uint64_t cols, uint64_t rows,
                       uint64_t mats, uint32_t box_cols, uint32_t box_rows);
 
+// 4D bf16 tensor map over a row-major [rows, 128] matrix (rows % 8 == 0)
+// seen as groups of 8 rows: a box of box_groups groups lands in shared memory
+// group after group, each as [64-column half 0 | half 1] of 8 rows x 128 B,
+// 128-byte swizzled.  One box thus covers whole rows (both halves) while each
+// half keeps a uniform 2 KB stride between its 8-row groups.
+int make_tmap_grouped_bf16(CUtensorMap* map, const void* base, uint64_t rows,
+                           uint32_t box_groups);
+
 // Launch `kern` as a programmatic dependent of the previous kernel in the
 // stream (cudaLaunchAttributeProgrammaticStreamSerialization): it may start
 // once that kernel has called griddepcontrol.launch_dependents (or ended) and
