@@ -175,16 +175,6 @@ __device__ __forceinline__ void tma_load_3d(void* smem_dst, const CUtensorMap* m
       : "memory");
 }
 
-// 4D tiled load (no multicast): coordinates (x inner, y, z, w).
-__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, int x, int y,
-                                            int z, int w, uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
-      : "memory");
-}
-
 // Byte offset of 16-byte chunk `chunk` (0..7) of row `row` inside a tile
 // written by TMA with 128-byte swizzling (rows of 128 bytes, 1024-byte atoms).
 __device__ __forceinline__ uint32_t sw128_offset(uint32_t row, uint32_t chunk) {

@@ -54,6 +54,17 @@ constexpr int kD = 128;
 constexpr int kMaxB = 2048;
 constexpr float kRescaleLog2 = 8.0f;
 
+// 4D tiled load (no multicast): coordinates (x inner, y, z, w); the paged
+// cache's grouped boxes.
+__device__ __forceinline__ void tma_load_4d(void* smem_dst, const CUtensorMap* map, int x, int y,
+                                            int z, int w, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.4d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%2, %3, %4, %5}], [%6];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(z), "r"(w), "r"(smem_u32(bar))
+      : "memory");
+}
+
 template <int N, int KS_, int VS_>
 struct Smem {
   // Ring depths.  A K slot frees as soon as its S MMA has run, a V slot only
