@@ -67,9 +67,9 @@ NCU_TRAFFIC = {
     "long_causal": ("prefill", "cf9fb7b089ed0128", (362489088 + 53635072) * 4),
     "mha_prefill": ("prefill", "cf9fb7b089ed0128", 132578304 + 13372928),
     "long_window": ("prefill", "cf9fb7b089ed0128", (241136128 + 48871424) * 4),
-    "mqa_decode": ("decode", "cb6f97e893d32d89", 323006976 + 4521216),
-    "spec_decode": ("decode", "cb6f97e893d32d89", 508926464 + 4657920),
-    "paged_decode": ("decode", "cb6f97e893d32d89", 319148032 + 5268992),
+    "mqa_decode": ("decode", "beb446c09c64c3bb", 323024896 + 4561152),
+    "spec_decode": ("decode", "beb446c09c64c3bb", 508933888 + 4384512),
+    "paged_decode": ("decode", "beb446c09c64c3bb", 319095552 + 4556800),
 }
 # Further counters of the same captures (same keys and hash rule): the
 # tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
@@ -79,9 +79,9 @@ NCU_COUNTERS = {
     "long_causal": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 58.9}),
     "mha_prefill": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 35.5}),
     "long_window": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 46.5}),
-    "mqa_decode": ("decode", "cb6f97e893d32d89", {"dram_gbs": 5424.1}),
-    "spec_decode": ("decode", "cb6f97e893d32d89", {"dram_gbs": 6079.4}),
-    "paged_decode": ("decode", "cb6f97e893d32d89", {"dram_gbs": 4286.7}),
+    "mqa_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 5500.8}),
+    "spec_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 5956.6}),
+    "paged_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 4874.3}),
 }
 
 
