@@ -62,11 +62,14 @@ KERNEL_SOURCES = {
 # --profile-heads 8; a full launch holds 805 MB of inputs) and are scaled by
 # 32 / 8: every head is an independent set of items over its own K/V.
 # paged_decode is mqa_decode over a cache of 16-token pages (the bench's
-# paged_decode object).
+# paged_decode object); gqa_rope_prefill is its attention kernel on rotated
+# inputs (the rotation passes are separate kernels).
 NCU_TRAFFIC = {
     "long_causal": ("prefill", "cf9fb7b089ed0128", (362489088 + 53635072) * 4),
     "mha_prefill": ("prefill", "cf9fb7b089ed0128", 132578304 + 13372928),
     "long_window": ("prefill", "cf9fb7b089ed0128", (241136128 + 48871424) * 4),
+    "cross_padded": ("prefill", "cf9fb7b089ed0128", 122257152 + 8826624),
+    "gqa_rope_prefill": ("prefill", "cf9fb7b089ed0128", 406414848 + 104055808),
     "mqa_decode": ("decode", "beb446c09c64c3bb", 323024896 + 4561152),
     "spec_decode": ("decode", "beb446c09c64c3bb", 508933888 + 4384512),
     "paged_decode": ("decode", "beb446c09c64c3bb", 319095552 + 4556800),
@@ -79,6 +82,8 @@ NCU_COUNTERS = {
     "long_causal": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 58.9}),
     "mha_prefill": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 35.5}),
     "long_window": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 46.5}),
+    "cross_padded": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 27.2}),
+    "gqa_rope_prefill": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 57.0}),
     "mqa_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 5500.8}),
     "spec_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 5956.6}),
     "paged_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 4874.3}),
