@@ -247,7 +247,12 @@ __global__ void __launch_bounds__(192, 1)
   using L = Smem<N, KS_, VS_>;
   constexpr int KS = L::KS, VS = L::VS;
   constexpr uint32_t kIdescS = tc::idesc_bf16(kTile, N, false, false);
-  constexpr uint32_t kIdescPV = tc::idesc_bf16(kD, N, true, false);
+  // P^T, the PV MMA's B operand: K-major up to 32 rows (each head's keys
+  // contiguous, two boxes of 64 keys; a thread stores its key's P head by
+  // head); MN-major at N = 64, where a key's 64 heads are one 128-byte row
+  // and a thread stores them as eight 16-byte chunks.
+  constexpr bool kPMn = N == 64;
+  constexpr uint32_t kIdescPV = tc::idesc_bf16(kD, N, true, kPMn);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -467,13 +472,18 @@ __global__ void __launch_bounds__(192, 1)
       };
       auto issue_pv = [&](int g, bool acc) {
         const uint64_t dv = tc::smem_desc_sw128(v_base + (g % VS) * L::kKV, kHalf, kGroup);
-        const uint64_t dp = tc::smem_desc_sw128(p_base + (g & 1) * 2 * L::kPBox, 16, 1024);
+        // MN-major P^T: one 64-head atom across, 8-key groups 1 KB apart
+        const uint64_t dp = tc::smem_desc_sw128(p_base + (g & 1) * 2 * L::kPBox,
+                                                kPMn ? 2u * L::kPBox : 16u, 1024);
         if (elect_one()) {
           tc::mma_ss(tmem + 2u * N, dv, dp, kIdescPV, acc ? 1u : 0u);
 #pragma unroll
-          for (int kk = 1; kk < kTile / 16; ++kk)
+          for (int kk = 1; kk < kTile / 16; ++kk) {
+            const uint32_t pk = kPMn ? (uint32_t)(kk * 2048)
+                                     : (uint32_t)((kk >> 2) * L::kPBox + (kk & 3) * 32);
             tc::mma_ss(tmem + 2u * N, dv + (uint64_t)((kk * 2 * kGroup) >> 4),
-                       dp + (uint64_t)(((kk >> 2) * L::kPBox + (kk & 3) * 32) >> 4), kIdescPV, 1u);
+                       dp + (uint64_t)(pk >> 4), kIdescPV, 1u);
+          }
         }
         __syncwarp();
       };
@@ -654,13 +664,35 @@ __global__ void __launch_bounds__(192, 1)
             load_s(h0);
             load_mu(h0);   // before this part's P stores
           }
+          if constexpr (kPMn) {
+            // this key's row of P^T: heads h0 .. h0 + 32 are 16-byte chunks
+            // h0 / 8 .. h0 / 8 + 3, swizzled with the key's row in its atom
+            uint8_t* prow = p_smem + buf * 2 * L::kPBox + Lr * 128;
 #pragma unroll
-          for (int h = 0; h < NC; ++h) {
-            const float p = exp2_approx(fmaf(sv[h], sl2, -mu[h]));
-            lp[h0 + h] += p;
-            const int hh = h0 + h;
-            const uint32_t off = (uint32_t)hh * 128u + (uint32_t)((kc ^ (hh & 7)) << 4) + kb;
-            *reinterpret_cast<__nv_bfloat16*>(pb_ + off) = __float2bfloat16_rn(p);
+            for (int c = 0; c < NC / 8; ++c) {
+              uint32_t w[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                const int h = 8 * c + 2 * i;
+                const float p0 = exp2_approx(fmaf(sv[h], sl2, -mu[h]));
+                const float p1 = exp2_approx(fmaf(sv[h + 1], sl2, -mu[h + 1]));
+                lp[h0 + h] += p0;
+                lp[h0 + h + 1] += p1;
+                w[i] = pack_bf16x2(p0, p1);
+              }
+              const int cc = h0 / 8 + c;
+              *reinterpret_cast<uint4*>(prow + ((cc ^ (Lr & 7)) << 4)) =
+                  make_uint4(w[0], w[1], w[2], w[3]);
+            }
+          } else {
+#pragma unroll
+            for (int h = 0; h < NC; ++h) {
+              const float p = exp2_approx(fmaf(sv[h], sl2, -mu[h]));
+              lp[h0 + h] += p;
+              const int hh = h0 + h;
+              const uint32_t off = (uint32_t)hh * 128u + (uint32_t)((kc ^ (hh & 7)) << 4) + kb;
+              *reinterpret_cast<__nv_bfloat16*>(pb_ + off) = __float2bfloat16_rn(p);
+            }
           }
         }
         fence_proxy_async_smem();
