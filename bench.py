@@ -70,9 +70,9 @@ NCU_TRAFFIC = {
     "long_window": ("prefill", "cf9fb7b089ed0128", (241136128 + 48871424) * 4),
     "cross_padded": ("prefill", "cf9fb7b089ed0128", 122257152 + 8826624),
     "gqa_rope_prefill": ("prefill", "cf9fb7b089ed0128", 406414848 + 104055808),
-    "mqa_decode": ("decode", "beb446c09c64c3bb", 323024896 + 4561152),
-    "spec_decode": ("decode", "beb446c09c64c3bb", 508933888 + 4384512),
-    "paged_decode": ("decode", "beb446c09c64c3bb", 319095552 + 4556800),
+    "mqa_decode": ("decode", "5707f1bdfff62684", 322999296 + 4343040),
+    "spec_decode": ("decode", "5707f1bdfff62684", 508918784 + 4852480),
+    "paged_decode": ("decode", "5707f1bdfff62684", 319074560 + 4551936),
 }
 # Further counters of the same captures (same keys and hash rule): the
 # tensor-pipe utilisation of a prefill launch (sm__pipe_tensor_cycles_active,
@@ -84,9 +84,9 @@ NCU_COUNTERS = {
     "long_window": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 46.5}),
     "cross_padded": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 27.2}),
     "gqa_rope_prefill": ("prefill", "cf9fb7b089ed0128", {"tensor_pipe_pct": 57.0}),
-    "mqa_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 5500.8}),
-    "spec_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 5956.6}),
-    "paged_decode": ("decode", "beb446c09c64c3bb", {"dram_gbs": 4874.3}),
+    "mqa_decode": ("decode", "5707f1bdfff62684", {"dram_gbs": 5470.3}),
+    "spec_decode": ("decode", "5707f1bdfff62684", {"dram_gbs": 6081.6}),
+    "paged_decode": ("decode", "5707f1bdfff62684", {"dram_gbs": 4926.1}),
 }
 
 
